@@ -1,0 +1,478 @@
+#!/usr/bin/env python
+"""Benchmark of one MLA absorbed-decode step on B200.
+
+A step is one pass of the whole hot path over one batch: the cache append of
+the batch's new tokens (down-projection, RMSNorm, RoPE, paged write) and the
+absorbed decode of those tokens (query absorption, split-KV attention over
+the paged latent cache, log-sum-exp combine, value up-projection).
+
+Default workload: DeepSeek-V3 shapes (128 heads, latent 512 + RoPE 64),
+batch 64, one new token per sequence, context lengths uniform in
+[1024, 8192], 64-token pages with a shuffled block table. The cache is filled
+before timing by the library's own append from x ~ N(0,1) hidden states and
+a kv_a weight ~ N(0, 1/7168), so every row is an RMS-normalised latent plus
+a RoPE-rotated key, as the workload prescribes.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun (N > 1) every rank runs its own replica (independent batches,
+no collective on the data path): weak scaling, timed as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MLA absorbed decode µs/step, cache GB/s & TFLOPS as fraction of B200 roofline"
+UNIT = "µs/step"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+L2_FLUSH_BYTES = 256 << 20
+HIDDEN = 7168
+
+
+# ----------------------------------------------------------- distributed
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def init_dist(backend: str, world: int, timeout_s: float = 120.0):
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return dist
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank's replica draws its own batch."""
+    return base + 7919 * rank
+
+
+def max_over_ranks(value: float, device) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and getattr(device, "type", "cpu") == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ------------------------------------------------------------- roofline
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            m = json.load(f)
+        return {"hbm_gbs": float(m["hbm_gbs"]), "bf16_tflops": float(m["bf16_tflops"]), "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS)
+
+
+def workload_totals(w, lengths):
+    """Algorithmic units of one decode step (measurement)."""
+    d = w.dims
+    L = [int(v) for v in lengths]
+    T = sum(L)  # unique cached tokens read
+    V = sum(Lb - w.q_len + s + 1 for Lb in L for s in range(w.q_len))  # visible (query, token) pairs
+    G = w.batch * w.q_len
+    row = d.row_width * 2  # bytes per cached token
+    attn_bytes = T * row + G * d.num_heads * row  # cache rows + absorbed queries
+    attn_flops = 2 * d.num_heads * (d.row_width + d.kv_lora_rank) * V
+    w_bytes = 2 * d.num_heads * (d.qk_nope_dim + d.v_head_dim) * d.kv_lora_rank * 2
+    step_bytes = T * row + w_bytes + G * d.num_heads * (d.qk_nope_dim + d.rope_dim + d.v_head_dim) * 2
+    step_flops = attn_flops + 2 * G * d.num_heads * (d.qk_nope_dim + d.v_head_dim) * d.kv_lora_rank
+    # every step appends its G new tokens (x [G, 7168] times W_kva [7168, 576])
+    step_bytes += HIDDEN * d.row_width * 2 + G * HIDDEN * 2
+    step_flops += 2 * G * HIDDEN * d.row_width
+    return dict(T=T, V=V, G=G, attn_bytes=attn_bytes, attn_flops=attn_flops, step_bytes=step_bytes,
+                step_flops=step_flops)
+
+
+def roofline(bytes_, flops, seconds, peaks):
+    gbs = bytes_ / seconds / 1e9
+    tfs = flops / seconds / 1e12
+    t_hbm = bytes_ / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    if t_hbm >= t_tc:
+        return dict(bound="hbm", achieved=round(gbs, 1), peak=peaks["hbm_gbs"], unit="GB/s",
+                    frac=round(gbs / peaks["hbm_gbs"], 4)), gbs, tfs
+    return dict(bound="tensor", achieved=round(tfs, 2), peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                frac=round(tfs / peaks["bf16_tflops"], 4)), gbs, tfs
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 100):
+        self.proc = None
+        self.lines = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 f"-lms", str(period_ms), "-i", str(gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------- CPU (oracle)
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample_seconds(w, lengths, seqs, heads):
+    """Times the fp64 oracle (explicit decode + append rows) on a few sequences and heads.
+
+    Inputs are drawn on the host from the same seeded generators (the
+    oracle never reads device data); only the timed calls are the oracle's.
+    """
+    import numpy as np
+
+    from mla_latent_kv_29_b200 import inputs as I
+    from oracle import mla_oracle as O
+
+    d = w.dims
+    q_nope, q_pe = I.queries(w)
+    w_uk, w_uv = I.up_weights(w)
+    x_new = I.normal((w.q_len, HIDDEN), 1.0, w.seed, 7)
+    w_kva = I.normal((HIDDEN, d.row_width), HIDDEN ** -0.5, w.seed, 8)
+    total = 0.0
+    tokens = 0
+    for b in seqs:
+        L = int(lengths[b])
+        c_raw, pe_raw = I.cache_raw(w, b, L)
+        c = O.rmsnorm(c_raw)
+        kpe = O.rope(pe_raw, np.arange(L))
+        qn = I.bf16(q_nope[b][:, heads]).double().numpy()
+        qp = I.bf16(q_pe[b][:, heads]).double().numpy()
+        wk = I.bf16(w_uk[heads]).double().numpy()
+        wv = I.bf16(w_uv[heads]).double().numpy()
+        t0 = time.perf_counter()
+        O.append_rows(x_new, w_kva, np.arange(L - w.q_len, L), d.kv_lora_rank)
+        O.decode_sequence(qn, qp, c, kpe, wk, wv, w.softmax_scale)
+        total += time.perf_counter() - t0
+        tokens += L
+    return total, tokens
+
+
+def cpu_baseline(w, lengths, budget_s: float = 12.0):
+    """Oracle µs/step for the whole workload, extrapolated from a bounded sample."""
+    H = w.dims.num_heads
+    heads = list(range(0, H, 4))  # a quarter of the heads
+    T = sum(int(v) for v in lengths)
+    spent, tok, seqs = 0.0, 0, []
+    for b in range(w.batch):
+        s, t = oracle_sample_seconds(w, lengths, [b], heads)
+        spent += s
+        tok += t
+        seqs.append(b)
+        if spent >= budget_s:
+            break
+    per_step_s = spent * (T / tok) * (H / len(heads))
+    return {"value": round(per_step_s * 1e6, 1), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 explicit oracle on {len(seqs)} of {w.batch} sequences ({tok} of {T} cached "
+                      f"tokens), {len(heads)} of {H} heads, plus their append rows; scaled by tokens and "
+                      f"heads to the full step ({spent:.1f} s measured)"}
+
+
+# -------------------------------------------------------------- GPU leg
+def setup_gpu(w, device, rank):
+    import torch
+
+    from mla_latent_kv_29_b200 import inputs as I
+    from mla_latent_kv_29_b200 import lib
+
+    d = w.dims
+    lengths = I.context_lengths(w)
+    table, nblk = I.block_table(w, lengths)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed)
+    pool = torch.empty(nblk, d.block_size, d.row_width, dtype=torch.bfloat16, device=device)
+    table_d = table.to(device)
+    w_kva = (torch.randn(HIDDEN, d.row_width, generator=gen, device=device) * HIDDEN ** -0.5).to(torch.bfloat16)
+    # fill positions 0 .. L_b - q_len - 1 of every sequence through the library's append
+    seq_ids = torch.cat([torch.full((int(L) - w.q_len,), b, dtype=torch.int32) for b, L in enumerate(lengths)])
+    pos = torch.cat([torch.arange(int(L) - w.q_len, dtype=torch.int32) for L in lengths])
+    chunk = 16384
+    ws = torch.empty(lib.append_workspace_size(d, chunk, HIDDEN) + 256, dtype=torch.uint8, device=device)
+    for i in range(0, seq_ids.numel(), chunk):
+        n = min(chunk, seq_ids.numel() - i)
+        x = torch.randn(n, HIDDEN, generator=gen, device=device).to(torch.bfloat16)
+        lib.append_kv(d, x, w_kva, seq_ids[i:i + n].to(device), pos[i:i + n].to(device), table_d, pool,
+                      workspace=ws)
+    torch.cuda.synchronize(device)
+    assert lib.device_error() == 0
+    G = w.batch * w.q_len
+    new_seq = torch.arange(w.batch, dtype=torch.int32).repeat_interleave(w.q_len)
+    new_pos = (lengths.repeat_interleave(w.q_len) - w.q_len +
+               torch.arange(w.q_len, dtype=torch.int32).repeat(w.batch)).to(torch.int32)
+    st = dict(
+        d=d, lengths=lengths, lengths_d=lengths.to(device), table=table_d, pool=pool, w_kva=w_kva,
+        x_new=torch.randn(G, HIDDEN, generator=gen, device=device).to(torch.bfloat16),
+        new_seq=new_seq.to(device), new_pos=new_pos.to(device),
+        q_nope=torch.randn(w.batch, w.q_len, d.num_heads, d.qk_nope_dim, generator=gen, device=device).to(torch.bfloat16),
+        q_pe=torch.randn(w.batch, w.q_len, d.num_heads, d.rope_dim, generator=gen, device=device).to(torch.bfloat16),
+        w_uk=(torch.randn(d.num_heads, d.qk_nope_dim, d.kv_lora_rank, generator=gen, device=device) * w.w_std).to(torch.bfloat16),
+        w_uv=(torch.randn(d.num_heads, d.v_head_dim, d.kv_lora_rank, generator=gen, device=device) * w.w_std).to(torch.bfloat16),
+        out=torch.empty(w.batch, w.q_len, d.num_heads, d.v_head_dim, dtype=torch.bfloat16, device=device),
+        max_len=int(lengths.max()),
+    )
+    st["ws_append"] = torch.empty(lib.append_workspace_size(d, G, HIDDEN) + 256, dtype=torch.uint8, device=device)
+    st["ws_decode"] = torch.empty(lib.decode_workspace_size(d, w.softmax_scale, w.batch, w.q_len, st["max_len"]),
+                                  dtype=torch.uint8, device=device)
+    return st
+
+
+def make_step(w, st, kernel):
+    from mla_latent_kv_29_b200 import lib
+
+    d = st["d"]
+
+    def step(x_new=None, q_nope=None, q_pe=None, events=None):
+        lib.append_kv(d, st["x_new"] if x_new is None else x_new, st["w_kva"], st["new_seq"], st["new_pos"],
+                      st["table"], st["pool"], workspace=st["ws_append"])
+        lib.decode(d, w.softmax_scale, st["q_nope"] if q_nope is None else q_nope,
+                   st["q_pe"] if q_pe is None else q_pe, st["pool"], st["table"], st["lengths_d"], st["max_len"],
+                   st["w_uk"], st["w_uv"], out=st["out"], workspace=st["ws_decode"], kernel=kernel,
+                   attn_events=events)
+
+    return step
+
+
+LAUNCHES_PER_STEP = 2 + 4  # append: GEMM + epilogue; decode: plan, absorb, attention, combine+W_UV
+
+
+def run_ours(args, w):
+    import torch
+
+    rank, world, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    init_dist("nccl", world)
+    from mla_latent_kv_29_b200 import lib
+
+    lib.load()
+    st = setup_gpu(w, device, rank)
+    step = make_step(w, st, args.kernel)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    assert lib.device_error() == 0, "device fault during warm-up"
+
+    sampler = ClockSampler(device.index)
+    soak_end = time.time() + args.soak
+    while time.time() < soak_end:  # holds the GPU under the step's load while the sampler starts
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize(device)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ea = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(device)
+    torch.cuda.synchronize(device)
+    for k in range(K):
+        flush.zero_()  # evicts L2 (126 MB) between timed steps
+        ev[k][0].record()
+        step(events=ea[k])
+        ev[k][1].record()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    attn_ms = [a.elapsed_time(b) for a, b in ea]
+    assert lib.device_error() == 0, "device fault during the timed steps"
+
+    # end to end through the public API with host buffers (pinned)
+    h_x = st["x_new"].cpu().pin_memory()
+    h_qn = st["q_nope"].cpu().pin_memory()
+    h_qp = st["q_pe"].cpu().pin_memory()
+    h_seq = st["new_seq"].cpu().pin_memory()
+    h_pos = st["new_pos"].cpu().pin_memory()
+    h_out = torch.empty(st["out"].shape, dtype=torch.bfloat16).pin_memory()
+    d_x, d_qn, d_qp = torch.empty_like(st["x_new"]), torch.empty_like(st["q_nope"]), torch.empty_like(st["q_pe"])
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(device)
+    torch.cuda.synchronize(device)
+    for k in range(K):
+        flush.zero_()
+        e2e_ev[k][0].record()
+        d_x.copy_(h_x, non_blocking=True)
+        d_qn.copy_(h_qn, non_blocking=True)
+        d_qp.copy_(h_qp, non_blocking=True)
+        st["new_seq"].copy_(h_seq, non_blocking=True)
+        st["new_pos"].copy_(h_pos, non_blocking=True)
+        step(x_new=d_x, q_nope=d_qn, q_pe=d_qp)
+        h_out.copy_(st["out"], non_blocking=True)
+        e2e_ev[k][1].record()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e2e_ms = [a.elapsed_time(b) for a, b in e2e_ev]
+
+    t_step = max_over_ranks(statistics.mean(step_ms), device)
+    t_attn = max_over_ranks(statistics.mean(attn_ms), device)
+    t_e2e = max_over_ranks(statistics.mean(e2e_ms), device)
+    if rank != 0:
+        return None
+    tot = workload_totals(w, st["lengths"].tolist())
+    peaks = load_peaks()
+    roof, attn_gbs, attn_tfs = roofline(tot["attn_bytes"], tot["attn_flops"], t_attn / 1e3, peaks)
+    roof["traffic"] = None
+    roof["kernel"] = "split-KV attention" + (" (CUDA cores)" if args.kernel == 2 else "")
+    roof["peak_source"] = peaks["source"]
+    nominal_step = max(tot["step_bytes"] / (NOMINAL["hbm_gbs"] * 1e9), tot["step_flops"] / (NOMINAL["bf16_tflops"] * 1e12))
+    line = {
+        "metric": METRIC, "value": round(t_step * 1e3, 2), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch_per_gpu": w.batch, "q_len": w.q_len,
+                   "context": f"U[{w.length_range[0]},{w.length_range[1]}]", "cached_tokens_per_gpu": tot["T"],
+                   "heads": w.dims.num_heads, "latent": w.dims.kv_lora_rank, "rope": w.dims.rope_dim,
+                   "page": w.dims.block_size, "paged": "shuffled", "l2": "flushed (256 MB write) before each step",
+                   "step": "append of the batch's new tokens + absorbed decode"},
+        "roofline": roof,
+        "attn_us": round(t_attn * 1e3, 2),
+        "attn_hbm_gbs": round(attn_gbs, 1), "attn_tflops": round(attn_tfs, 2),
+        "cache_tokens_per_s": round(world * tot["T"] / (t_step / 1e3), 1),
+        "decode_tokens_per_s": round(world * tot["G"] / (t_step / 1e3), 1),
+        "step_roofline_nominal_us": round(nominal_step * 1e6, 2),
+        "step_frac_of_nominal_roofline": round(nominal_step / (t_step / 1e3), 4),
+        "e2e": {"value": round(t_e2e * 1e3, 2), "unit": UNIT,
+                "h2d_bytes_per_step": (h_x.numel() + h_qn.numel() + h_qp.numel()) * 2
+                                      + (h_seq.numel() + h_pos.numel()) * 4,
+                "d2h_bytes_per_step": h_out.numel() * 2},
+        "gpu_launches": LAUNCHES_PER_STEP * K,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, st["lengths"].tolist(), args.cpu_seconds)
+    return line
+
+
+def run_reference(args, w):
+    """The oracle timed on the host cores (the reference arm)."""
+    from mla_latent_kv_29_b200 import inputs as I
+
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    lengths = I.context_lengths(w).tolist()
+    H = w.dims.num_heads
+    heads = list(range(0, H, 4))
+    T = sum(lengths)
+    per_step = []
+    for k in range(args.warmup + args.steps):
+        b = k % w.batch
+        s, tok = oracle_sample_seconds(w, lengths, [b], heads)
+        if k >= args.warmup:
+            per_step.append(s * (T / tok) * (H / len(heads)))
+    v = statistics.mean(per_step) * 1e6
+    sample = (f"each step: fp64 explicit oracle on 1 of {w.batch} sequences and {len(heads)} of {H} heads "
+              f"plus its append rows, scaled by tokens and heads to the full step")
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v / 1e3, 3),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch_per_gpu": w.batch, "q_len": w.q_len,
+                       "context": f"U[{w.length_range[0]},{w.length_range[1]}]"},
+            "cpu_baseline": {"value": round(v, 1), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="v3_b64_l1k_8k")
+    ap.add_argument("--kernel", type=int, default=0, help="0 auto, 1 sm100 tensor-core, 2 CUDA-core")
+    ap.add_argument("--soak", type=float, default=1.5, help="seconds of untimed steps while clocks are sampled")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from mla_latent_kv_29_b200 import inputs as I
+
+    rank, world, _ = dist_env()
+    w = I.WORKLOADS[args.workload]
+    import dataclasses
+
+    w = dataclasses.replace(w, seed=rank_seed(w.seed, rank))
+    line = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    if args.impl == "ours" and world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,205 @@
+/*
+ * mla_b200.h -- C ABI of the B200 (sm_100a) MLA absorbed-decode library.
+ *
+ * Multi-head Latent Attention (DeepSeek-V3 style) keeps one latent row per
+ * cached token: c_kv (kv_lora_rank values, RMS-normalised) followed by a
+ * decoupled RoPE key k_pe (rope_dim values) shared by every head.
+ * Sources, cited by page title and section:
+ *   [MLA-arch] "MLA架构：低秩注意力机制优化LLM显存与计算效率": section 1
+ *              (128 heads, qk_head_dim 128 + 64, the RoPE part broadcast to
+ *              all heads), 2.2 (kv_a_proj_with_mqa hidden -> 512 + 64,
+ *              kv_a_layernorm, kv_b_proj), 3.1 (absorption = matrix
+ *              associativity), 3.2 (cache = c_kv + shared pe), 4.2 (fuse
+ *              RoPE with the cache update).
+ *   [MQA-MLA]  "一次讲透MHA、GQA、MQA、MLA", section "MLA的实现": RoPE module,
+ *              forward_training (explicit K/V) and forward_inference_absorbed
+ *              (scores = q_absorbed . c_kv + q_r . k_r; output from P . c_kv).
+ *
+ * Conventions for every entry point:
+ *   - bf16 means IEEE bfloat16 stored as uint16; all tensors are dense,
+ *     row-major, with the shapes given below.
+ *   - Pointers are DEVICE pointers unless the argument says "host". The
+ *     caller allocates and owns every buffer; the library never allocates,
+ *     frees or synchronises. Work is enqueued on `stream` (a cudaStream_t;
+ *     NULL = legacy default stream) and runs asynchronously.
+ *   - Return value: MLA_OK (0) or a negative mla_status_t. Host-side
+ *     validation failures return before anything is enqueued. Nothing
+ *     aborts, throws or prints across this boundary.
+ *   - Faults found by a kernel (a block id outside the pool, a position
+ *     outside the block table, a bounded device wait that expired) do not
+ *     trap: the offending access is skipped and a device error word is set;
+ *     read and clear it with mla_get_device_error().
+ */
+#ifndef MLA_B200_H
+#define MLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mla_status {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = -1,         /* null pointer, non-positive size, bad stride */
+    MLA_ERR_UNSUPPORTED_DIMS = -2,    /* dims outside what the kernels implement */
+    MLA_ERR_WORKSPACE_TOO_SMALL = -3, /* workspace_bytes < the *_workspace_size() answer */
+    MLA_ERR_CUDA = -4,                /* a CUDA runtime call or launch failed */
+    MLA_ERR_DEVICE_FAULT = -5,        /* device error word: bad block id / slot / position */
+    MLA_ERR_DEVICE_TIMEOUT = -6,      /* device error word: a bounded wait expired */
+    MLA_ERR_NO_DEVICE = -7            /* no sm_100 device is current */
+} mla_status_t;
+
+/* Per-layer sizes. DeepSeek-V3: {128, 512, 64, 128, 128, 64, 1/sqrt(192)}
+ * ([MLA-arch] 1 and 2.2). softmax_scale multiplies the summed score
+ * q_nope.k_nope + q_pe.k_pe; the pages use (d_nope + d_rope)^-1/2
+ * ([MQA-MLA] "MLA的实现", self.scale). */
+typedef struct mla_dims {
+    int32_t num_heads;    /* H */
+    int32_t kv_lora_rank; /* d_c: latent values per token */
+    int32_t rope_dim;     /* d_r: shared RoPE key values per token */
+    int32_t qk_nope_dim;  /* d_n: per-head query/key width without RoPE */
+    int32_t v_head_dim;   /* d_v: per-head value width */
+    int32_t block_size;   /* tokens per cache page */
+    float softmax_scale;
+} mla_dims_t;
+
+/* Kernel choice, split control and timing hooks for mla_decode. Pass NULL
+ * for defaults. */
+typedef struct mla_decode_opts {
+    int32_t kernel;      /* 0 auto; 1 sm100 tensor-core kernel (V3 dims only);
+                            2 CUDA-core kernel (any supported dims) */
+    int32_t num_workers; /* 0 auto; else the number of split-KV workers the
+                            balanced schedule targets (>= 1) */
+    void* event_attn_begin; /* NULL or a cudaEvent_t recorded on `stream` right
+                               before the split-KV attention kernel */
+    void* event_attn_end;   /* NULL or a cudaEvent_t recorded right after it */
+} mla_decode_opts_t;
+
+/* Paged latent cache ("pool"), [MLA-arch] 3.2 kept as one row per token:
+ *   pool        bf16 [num_blocks, block_size, kv_lora_rank + rope_dim]
+ *               row = c_kv (kv_lora_rank) then k_pe (rope_dim)
+ *   block_table int32 [batch, max_blocks_per_seq]; page j of sequence b is
+ *               pool block block_table[b*max_blocks_per_seq + j]
+ *   token t of sequence b lives in pool row
+ *               block_table[b][t / block_size] * block_size + t % block_size
+ * A contiguous cache is block_size >= context length with block b for
+ * sequence b. */
+
+/* ------------------------------------------------------------------ */
+/* Cache append: [MLA-arch] 2.2 (kv_a_proj_with_mqa, kv_a_layernorm) and
+ * 4.2 (RoPE fused with the cache update); RoPE as in [MQA-MLA] "MLA的实现".
+ *   kv   = x . w_kva                       (fp32 accumulate)
+ *   c    = kv[:d_c] / sqrt(mean(kv[:d_c]^2) + rms_eps) * gamma
+ *   k_pe = rotate-half RoPE of kv[d_c:] at positions[i], base rope_base
+ *   pool[row(seq_ids[i], positions[i])] = bf16(c) ++ bf16(k_pe)
+ * Arguments:
+ *   x          bf16 [n_tokens, hidden]
+ *   w_kva      bf16 [hidden, kv_lora_rank + rope_dim]
+ *   rms_gamma  bf16 [kv_lora_rank] or NULL (= ones)
+ *   seq_ids    int32 [n_tokens] in [0, num_seqs), positions int32 [n_tokens]
+ *   block_table int32 [num_seqs, max_blocks_per_seq]; pool as above (written
+ *              only at the target rows)
+ *   workspace  >= mla_append_workspace_size(dims, n_tokens, hidden) bytes,
+ *              256-byte aligned, contents need not be initialised.
+ * A (seq, position) whose sequence is outside [0, num_seqs), whose page is
+ * missing (-1 / >= num_blocks) or outside max_blocks_per_seq is skipped and
+ * flags MLA_ERR_DEVICE_FAULT. Rows of distinct tokens must not coincide. */
+MLA_API int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t hidden,
+                  const void* w_kva, const void* rms_gamma, float rms_eps, float rope_base,
+                  const int32_t* seq_ids, const int32_t* positions,
+                  const int32_t* block_table, int32_t num_seqs, int32_t max_blocks_per_seq,
+                  void* pool, int64_t num_blocks,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+MLA_API size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t n_tokens, int32_t hidden);
+
+/* ------------------------------------------------------------------ */
+/* Absorbed decode: [MQA-MLA] "MLA的实现" forward_inference_absorbed with the
+ * query absorption of [MLA-arch] 3.1, restated for q_len new tokens per
+ * sequence over the paged cache. For sequence b (context_lens[b] = L
+ * cached tokens, the q_len new ones included), new token s, head h:
+ *   q_lat  = W_UK[h]^T q_nope[b,s,h]                       (d_c)
+ *   z_t    = scale * (q_lat . c_t + q_pe[b,s,h] . k_pe_t),  t = 0 .. L-q_len+s
+ *   o_lat  = softmax(z) . c                                 (d_c)
+ *   out[b,s,h] = W_UV[h] o_lat                              (d_v)
+ * computed as split-KV partials merged by a log-sum-exp combine.
+ * Arguments:
+ *   q_nope  bf16 [batch, q_len, H, qk_nope_dim]
+ *   q_pe    bf16 [batch, q_len, H, rope_dim]   (RoPE already applied)
+ *   pool, block_table: as above (read only)
+ *   context_lens int32 [batch] on the device; every value must be in
+ *           [q_len, max_context_len] and covered by the block table
+ *   max_context_len  host int, an upper bound of context_lens (sizes the
+ *           launch and the workspace)
+ *   w_uk    bf16 [H, qk_nope_dim, kv_lora_rank]
+ *   w_uv    bf16 [H, v_head_dim, kv_lora_rank]
+ *   out     bf16 [batch, q_len, H, v_head_dim]
+ *   workspace >= mla_decode_workspace_size(...) bytes, 256-byte aligned,
+ *           contents need not be initialised
+ *   opts    NULL or kernel / split overrides
+ * Rounding: q_lat is rounded to bf16 before the score product and the
+ * softmax weights to bf16 before the value product; accumulation, partials
+ * and the combine are fp32; out is rounded to bf16 once. */
+MLA_API int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe,
+               int32_t batch, int32_t q_len,
+               const void* pool, int64_t num_blocks,
+               const int32_t* block_table, int32_t max_blocks_per_seq,
+               const int32_t* context_lens, int32_t max_context_len,
+               const void* w_uk, const void* w_uv, void* out,
+               void* workspace, size_t workspace_bytes,
+               const mla_decode_opts_t* opts, void* stream);
+
+MLA_API size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t batch, int32_t q_len,
+                                 int32_t max_context_len, const mla_decode_opts_t* opts);
+
+/* ------------------------------------------------------------------ */
+/* Log-sum-exp combine of split-KV partials (the merge the split decode
+ * needs; no page states it, it is exact softmax algebra). For group g
+ * (= b*q_len + s) and head h, with parts i in [part_offsets[g],
+ * part_offsets[g+1]):
+ *   M = max_i lse_i;  w_i = exp(lse_i - M)  (0 when lse_i = -inf)
+ *   o_lat[g,h] = sum_i w_i o_part[i,h] / sum_i w_i
+ *   lse_out[g,h] = M + log(sum_i w_i)
+ * A group whose parts all have lse = -inf (or that has none) gets zeros and
+ * lse = -inf.
+ *   o_part   fp32 [n_parts, H, kv_lora_rank]   (each part normalised)
+ *   lse_part fp32 [n_parts, H]                 (natural log)
+ *   part_offsets int32 [n_groups + 1], non-decreasing, device memory
+ *   o_lat    fp32 [n_groups, H, kv_lora_rank]
+ *   lse_out  fp32 [n_groups, H] or NULL */
+MLA_API int mla_combine(const mla_dims_t* dims, const float* o_part, const float* lse_part,
+                const int32_t* part_offsets, int32_t n_groups,
+                float* o_lat, float* lse_out, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* Test hook: the pool row of (seq_ids[i], positions[i]) from the same
+ * device resolver the append and decode kernels use; -1 where the sequence,
+ * page or block id is out of range. rows: int64 [n] device. */
+MLA_API int mla_debug_resolve_slots(const mla_dims_t* dims, const int32_t* block_table, int32_t num_seqs,
+                            int32_t max_blocks_per_seq, int64_t num_blocks,
+                            const int32_t* seq_ids, const int32_t* positions, int32_t n,
+                            int64_t* rows, void* stream);
+
+/* Reads and clears the device error word of the current device after
+ * synchronising `stream`. *device_status receives MLA_OK or the first
+ * MLA_ERR_DEVICE_* recorded since the last call. */
+MLA_API int mla_get_device_error(int* device_status, void* stream);
+
+/* Static description of a status code (never NULL). */
+MLA_API const char* mla_error_string(int status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+MLA_API int mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_B200_H */

@@ -1,0 +1,322 @@
+// C ABI of the MLA decode library: argument validation, workspace layout and
+// kernel launches. Every entry point returns an mla_status_t and never
+// allocates, frees or synchronises (except mla_get_device_error, whose job
+// is to synchronise and read the device status word).
+#include <cmath>
+#include <cstring>
+
+#include "mla_b200.h"
+#include "common.cuh"
+#include "plan.cuh"
+#include "absorb.cuh"
+#include "combine.cuh"
+#include "decode_generic.cuh"
+#include "append.cuh"
+
+namespace mla {
+namespace {
+
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Dims the CUDA-core kernels implement.
+int check_dims(const mla_dims_t* d) {
+    if (!d) return MLA_ERR_INVALID_ARG;
+    if (d->num_heads < 1 || d->kv_lora_rank < 8 || d->rope_dim < 2 || d->qk_nope_dim < 1 ||
+        d->v_head_dim < 1 || d->block_size < 1 || !(d->softmax_scale > 0.f) || !std::isfinite(d->softmax_scale))
+        return MLA_ERR_INVALID_ARG;
+    if (d->num_heads > 1024 || d->kv_lora_rank > 16 * kGenMaxCols || d->rope_dim > 128 ||
+        d->qk_nope_dim > 512 || d->v_head_dim > 512)
+        return MLA_ERR_UNSUPPORTED_DIMS;
+    if ((d->kv_lora_rank + d->rope_dim) % 8 != 0 || d->rope_dim % 2 != 0) return MLA_ERR_UNSUPPORTED_DIMS;
+    return MLA_OK;
+}
+
+int device_ok() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return MLA_ERR_NO_DEVICE; }
+    static int cached[64] = {0};  // 0 unknown, 1 ok, 2 not sm_100
+    if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev] == 1 ? MLA_OK : MLA_ERR_NO_DEVICE;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_NO_DEVICE;
+    }
+    const int ok = major == 10 ? 1 : 2;
+    if (dev >= 0 && dev < 64) cached[dev] = ok;
+    return ok == 1 ? MLA_OK : MLA_ERR_NO_DEVICE;
+}
+
+int launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int num_sms() {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+// ---- decode workspace ------------------------------------------------
+struct DecodeLayout {
+    size_t hdr, tile_prefix, part_offsets, q, o_part, lse_part, total;
+    int32_t workers, max_parts, kernel, tile;
+};
+
+int pick_kernel(const mla_dims_t* d, const mla_decode_opts_t* o) {
+    (void)d;
+    const int k = o ? o->kernel : 0;
+    if (k == 0 || k == 2) return 2;
+    return -1;
+}
+
+int default_workers(const mla_dims_t* d, int kernel) {
+    (void)kernel;
+    const int hb = (d->num_heads + kGenHeads - 1) / kGenHeads;
+    const int target = 4 * num_sms();
+    return target / hb > 0 ? target / hb : 1;
+}
+
+int decode_layout(const mla_dims_t* d, int32_t batch, int32_t q_len, int32_t max_len,
+                  const mla_decode_opts_t* o, DecodeLayout* L) {
+    int rc = check_dims(d);
+    if (rc) return rc;
+    if (batch < 1 || q_len < 1 || max_len < q_len) return MLA_ERR_INVALID_ARG;
+    const int kernel = pick_kernel(d, o);
+    if (kernel < 0) return MLA_ERR_UNSUPPORTED_DIMS;
+    L->kernel = kernel;
+    L->tile = kGenTokens;
+    const int64_t G = static_cast<int64_t>(batch) * q_len;
+    const int64_t tiles_per_group = (max_len + L->tile - 1) / L->tile;
+    if (G * tiles_per_group >= (int64_t(1) << 31) || G * d->num_heads >= (int64_t(1) << 31))
+        return MLA_ERR_UNSUPPORTED_DIMS;
+    int64_t workers = (o && o->num_workers > 0) ? o->num_workers : default_workers(d, kernel);
+    if (workers > (int64_t(1) << 20)) workers = int64_t(1) << 20;
+    L->workers = static_cast<int32_t>(workers);
+    L->max_parts = static_cast<int32_t>(G + workers);
+    const size_t D = static_cast<size_t>(d->kv_lora_rank) + d->rope_dim;
+    size_t off = 0;
+    L->hdr = off; off = align_up(off + sizeof(PlanHeader));
+    L->tile_prefix = off; off = align_up(off + sizeof(int32_t) * (G + 1));
+    L->part_offsets = off; off = align_up(off + sizeof(int32_t) * (G + 1));
+    L->q = off; off = align_up(off + sizeof(uint16_t) * G * d->num_heads * D);
+    L->o_part = off; off = align_up(off + sizeof(float) * static_cast<size_t>(L->max_parts) * d->num_heads * d->kv_lora_rank);
+    L->lse_part = off; off = align_up(off + sizeof(float) * static_cast<size_t>(L->max_parts) * d->num_heads);
+    L->total = off;
+    return MLA_OK;
+}
+
+template <typename K>
+int ensure_smem(K kernel, size_t bytes) {
+    if (bytes <= 48 * 1024) return MLA_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    return MLA_OK;
+}
+
+// ---- append workspace ------------------------------------------------
+int append_splits(int32_t n_tokens, int32_t hidden, int32_t N) {
+    const int64_t tiles = static_cast<int64_t>((N + kApTileN - 1) / kApTileN) * ((n_tokens + kApTileT - 1) / kApTileT);
+    const int64_t target = 2 * num_sms();
+    int64_t s = tiles >= target ? 1 : (target + tiles - 1) / tiles;
+    const int64_t max_s = (hidden + kApTileK - 1) / kApTileK;
+    if (s > max_s) s = max_s;
+    if (s > 64) s = 64;
+    return static_cast<int>(s < 1 ? 1 : s);
+}
+
+}  // namespace
+}  // namespace mla
+
+using namespace mla;
+
+extern "C" {
+
+int mla_version(void) { return 100; }
+
+const char* mla_error_string(int s) {
+    switch (s) {
+        case MLA_OK: return "ok";
+        case MLA_ERR_INVALID_ARG: return "invalid argument";
+        case MLA_ERR_UNSUPPORTED_DIMS: return "dims not supported by the selected kernel";
+        case MLA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case MLA_ERR_CUDA: return "CUDA runtime or launch error";
+        case MLA_ERR_DEVICE_FAULT: return "device fault: block id, slot or position out of range";
+        case MLA_ERR_DEVICE_TIMEOUT: return "device timeout: a bounded wait expired";
+        case MLA_ERR_NO_DEVICE: return "no sm_100 CUDA device is current";
+        default: return "unknown status";
+    }
+}
+
+int mla_get_device_error(int* device_status, void* stream) {
+    if (!device_status) return MLA_ERR_INVALID_ARG;
+    if (int rc = device_ok()) return rc;
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+    *device_status = v;
+    return MLA_OK;
+}
+
+size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t n_tokens, int32_t hidden) {
+    if (check_dims(dims) || n_tokens < 1 || hidden < 1) return 0;
+    const int N = dims->kv_lora_rank + dims->rope_dim;
+    const int s = append_splits(n_tokens, hidden, N);
+    return align_up(sizeof(float) * static_cast<size_t>(s) * n_tokens * N);
+}
+
+int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t hidden, const void* w_kva,
+                  const void* rms_gamma, float rms_eps, float rope_base, const int32_t* seq_ids,
+                  const int32_t* positions, const int32_t* block_table, int32_t num_seqs,
+                  int32_t max_blocks_per_seq, void* pool, int64_t num_blocks, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+    if (int rc = check_dims(dims)) return rc;
+    if (!x || !w_kva || !seq_ids || !positions || !block_table || !pool || !workspace) return MLA_ERR_INVALID_ARG;
+    if (n_tokens < 1 || hidden < 1 || num_seqs < 1 || max_blocks_per_seq < 1 || num_blocks < 1)
+        return MLA_ERR_INVALID_ARG;
+    if (!(rms_eps >= 0.f) || !(rope_base > 0.f)) return MLA_ERR_INVALID_ARG;
+    if (!aligned(workspace, kAlign) || !aligned(pool, 16)) return MLA_ERR_INVALID_ARG;
+    if (workspace_bytes < mla_append_workspace_size(dims, n_tokens, hidden)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+    if (int rc = device_ok()) return rc;
+    const int N = dims->kv_lora_rank + dims->rope_dim;
+    const int splits = append_splits(n_tokens, hidden, N);
+    int k_per_split = (hidden + splits - 1) / splits;
+    k_per_split = (k_per_split + kApTileK - 1) / kApTileK * kApTileK;
+    float* part = static_cast<float*>(workspace);
+    cudaStream_t st = as_stream(stream);
+    dim3 g1((N + kApTileN - 1) / kApTileN, (n_tokens + kApTileT - 1) / kApTileT, splits);
+    append_gemm_kernel<<<g1, 256, 0, st>>>(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w_kva),
+                                           part, n_tokens, hidden, N, k_per_split);
+    if (int rc = launch_status()) return rc;
+    AppendEpilogueParams P;
+    P.part = part;
+    P.gamma = static_cast<const uint16_t*>(rms_gamma);
+    P.seq_ids = seq_ids;
+    P.positions = positions;
+    P.block_table = block_table;
+    P.pool = static_cast<uint16_t*>(pool);
+    P.num_blocks = num_blocks;
+    P.splits = splits;
+    P.T = n_tokens;
+    P.dc = dims->kv_lora_rank;
+    P.dr = dims->rope_dim;
+    P.num_seqs = num_seqs;
+    P.max_blocks_per_seq = max_blocks_per_seq;
+    P.block_size = dims->block_size;
+    P.eps = rms_eps;
+    P.rope_base = rope_base;
+    append_epilogue_kernel<<<n_tokens, 256, sizeof(float) * N, st>>>(P);
+    return launch_status();
+}
+
+size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t batch, int32_t q_len, int32_t max_context_len,
+                                 const mla_decode_opts_t* opts) {
+    DecodeLayout L;
+    if (decode_layout(dims, batch, q_len, max_context_len, opts, &L)) return 0;
+    return L.total;
+}
+
+int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int32_t batch, int32_t q_len,
+               const void* pool, int64_t num_blocks, const int32_t* block_table, int32_t max_blocks_per_seq,
+               const int32_t* context_lens, int32_t max_context_len, const void* w_uk, const void* w_uv,
+               void* out, void* workspace, size_t workspace_bytes, const mla_decode_opts_t* opts, void* stream) {
+    DecodeLayout L;
+    if (int rc = decode_layout(dims, batch, q_len, max_context_len, opts, &L)) return rc;
+    if (!q_nope || !q_pe || !pool || !block_table || !context_lens || !w_uk || !w_uv || !out || !workspace)
+        return MLA_ERR_INVALID_ARG;
+    if (num_blocks < 1 || max_blocks_per_seq < 1) return MLA_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(max_blocks_per_seq) * dims->block_size < max_context_len) return MLA_ERR_INVALID_ARG;
+    if (!aligned(workspace, kAlign) || !aligned(pool, 16)) return MLA_ERR_INVALID_ARG;
+    if (workspace_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+    if (int rc = device_ok()) return rc;
+
+    cudaStream_t st = as_stream(stream);
+    char* ws = static_cast<char*>(workspace);
+    PlanHeader* hdr = reinterpret_cast<PlanHeader*>(ws + L.hdr);
+    int32_t* tile_prefix = reinterpret_cast<int32_t*>(ws + L.tile_prefix);
+    int32_t* part_offsets = reinterpret_cast<int32_t*>(ws + L.part_offsets);
+    uint16_t* q = reinterpret_cast<uint16_t*>(ws + L.q);
+    float* o_part = reinterpret_cast<float*>(ws + L.o_part);
+    float* lse_part = reinterpret_cast<float*>(ws + L.lse_part);
+    const int32_t G = batch * q_len;
+    const int H = dims->num_heads, dc = dims->kv_lora_rank, dr = dims->rope_dim;
+
+    plan_kernel<<<1, 1024, 0, st>>>(context_lens, batch, q_len, L.tile, L.workers, hdr, tile_prefix, part_offsets);
+    if (int rc = launch_status()) return rc;
+
+    const size_t absorb_smem = sizeof(float) * kAbsorbGroups * dims->qk_nope_dim;
+    if (int rc = ensure_smem(absorb_q_kernel, absorb_smem)) return rc;
+    absorb_q_kernel<<<dim3(H, (G + kAbsorbGroups - 1) / kAbsorbGroups), kAbsorbThreads, absorb_smem, st>>>(
+        static_cast<const uint16_t*>(q_nope), static_cast<const uint16_t*>(q_pe),
+        static_cast<const uint16_t*>(w_uk), q, G, H, dims->qk_nope_dim, dc, dr);
+    if (int rc = launch_status()) return rc;
+
+    GenericDecodeParams P;
+    P.q = q;
+    P.pool = static_cast<const uint16_t*>(pool);
+    P.block_table = block_table;
+    P.context_lens = context_lens;
+    P.hdr = hdr;
+    P.tile_prefix = tile_prefix;
+    P.part_offsets = part_offsets;
+    P.o_part = o_part;
+    P.lse_part = lse_part;
+    P.num_blocks = num_blocks;
+    P.batch = batch;
+    P.max_blocks_per_seq = max_blocks_per_seq;
+    P.block_size = dims->block_size;
+    P.q_len = q_len;
+    P.H = H;
+    P.dc = dc;
+    P.dr = dr;
+    P.scale = dims->softmax_scale;
+    const size_t gsmem = generic_decode_smem(dc, dr);
+    if (int rc = ensure_smem(generic_decode_kernel, gsmem)) return rc;
+    if (opts && opts->event_attn_begin) cudaEventRecord(static_cast<cudaEvent_t>(opts->event_attn_begin), st);
+    generic_decode_kernel<<<dim3(L.workers, (H + kGenHeads - 1) / kGenHeads), kGenThreads, gsmem, st>>>(P);
+    if (int rc = launch_status()) return rc;
+    if (opts && opts->event_attn_end) cudaEventRecord(static_cast<cudaEvent_t>(opts->event_attn_end), st);
+
+    const size_t uv_smem = sizeof(float) * kUvGroups * dc;
+    if (int rc = ensure_smem(combine_uv_kernel, uv_smem)) return rc;
+    combine_uv_kernel<<<dim3(H, (G + kUvGroups - 1) / kUvGroups), kUvThreads, uv_smem, st>>>(
+        o_part, lse_part, part_offsets, static_cast<const uint16_t*>(w_uv), G, H, dc, dims->v_head_dim,
+        static_cast<uint16_t*>(out));
+    return launch_status();
+}
+
+int mla_combine(const mla_dims_t* dims, const float* o_part, const float* lse_part, const int32_t* part_offsets,
+                int32_t n_groups, float* o_lat, float* lse_out, void* stream) {
+    if (int rc = check_dims(dims)) return rc;
+    if (!o_part || !lse_part || !part_offsets || !o_lat || n_groups < 1) return MLA_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(n_groups) * dims->num_heads >= (int64_t(1) << 31)) return MLA_ERR_UNSUPPORTED_DIMS;
+    if (int rc = device_ok()) return rc;
+    combine_kernel<<<n_groups * dims->num_heads, 128, 0, as_stream(stream)>>>(
+        o_part, lse_part, part_offsets, n_groups, dims->num_heads, dims->kv_lora_rank, o_lat, lse_out);
+    return launch_status();
+}
+
+int mla_debug_resolve_slots(const mla_dims_t* dims, const int32_t* block_table, int32_t num_seqs,
+                            int32_t max_blocks_per_seq, int64_t num_blocks, const int32_t* seq_ids,
+                            const int32_t* positions, int32_t n, int64_t* rows, void* stream) {
+    if (int rc = check_dims(dims)) return rc;
+    if (!block_table || !seq_ids || !positions || !rows || n < 1 || num_seqs < 1 || max_blocks_per_seq < 1)
+        return MLA_ERR_INVALID_ARG;
+    if (int rc = device_ok()) return rc;
+    resolve_slots_kernel<<<(n + 255) / 256, 256, 0, as_stream(stream)>>>(
+        block_table, num_seqs, max_blocks_per_seq, num_blocks, dims->block_size, seq_ids, positions, n, rows);
+    return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,112 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+symbol, and rejects bad arguments before touching a device. No kernel is
+launched here; on a machine without a GPU a fully valid call must return
+MLA_ERR_NO_DEVICE rather than crash."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mla_latent_kv_29_b200 import inputs as I
+from mla_latent_kv_29_b200 import lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def so():
+    if not os.path.exists(L.LIB_PATH):
+        from mla_latent_kv_29_b200 import build
+
+        build.build()
+    return L.load()
+
+
+def declared_symbols():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            txt = open(os.path.join(inc, f)).read()
+            names |= set(re.findall(r"MLA_API\s+[\w\s\*]+?\b(mla_\w+)\s*\(", txt))
+    return names
+
+
+def test_every_declared_symbol_is_exported(so):
+    names = declared_symbols()
+    assert {"mla_append_kv", "mla_decode", "mla_combine"} <= names
+    for n in names:
+        assert hasattr(so, n), n
+    assert set(L.EXPORTED) == names
+
+
+def test_error_strings_and_version(so):
+    for code in L.STATUS_NAMES:
+        assert L.error_string(code)
+    assert L.error_string(12345) == "unknown status"
+    assert so.mla_version() >= 100
+
+
+def _dims(**kw):
+    d = dict(num_heads=128, kv_lora_rank=512, rope_dim=64, qk_nope_dim=128, v_head_dim=128, block_size=64,
+             softmax_scale=192 ** -0.5)
+    d.update(kw)
+    return L.CDims(**d)
+
+
+def _decode(so, dims, ws_bytes=1 << 30, null_q=False, batch=2, q_len=1, max_len=1000, opts=None):
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first or no device
+    return so.mla_decode(ctypes.byref(dims), None if null_q else fake, fake, batch, q_len, fake, 100, fake, 16,
+                         fake, max_len, fake, fake, fake, ctypes.c_void_p(1 << 20), ws_bytes,
+                         ctypes.byref(opts) if opts else None, None)
+
+
+def test_workspace_size_v3(so):
+    n = so.mla_decode_workspace_size(ctypes.byref(_dims()), 64, 1, 8192, None)
+    assert n > 64 * 128 * 576 * 2  # at least the absorbed queries
+    assert n % 256 == 0
+    assert so.mla_decode_workspace_size(ctypes.byref(_dims(num_heads=0)), 64, 1, 8192, None) == 0
+    assert so.mla_decode_workspace_size(ctypes.byref(_dims()), 4, 8, 4, None) == 0  # max_len < q_len
+    assert so.mla_append_workspace_size(ctypes.byref(_dims()), 64, 7168) >= 64 * 576 * 4
+
+
+def test_decode_validation(so):
+    assert _decode(so, _dims(), null_q=True) == -1
+    assert _decode(so, _dims(kv_lora_rank=4096)) == -2
+    assert _decode(so, _dims(rope_dim=3)) == -1 or _decode(so, _dims(rope_dim=3)) == -2
+    assert _decode(so, _dims(softmax_scale=float("nan"))) == -1
+    assert _decode(so, _dims(), ws_bytes=16) == -3
+    assert _decode(so, _dims(), batch=0) == -1
+    assert _decode(so, _dims(), max_len=2000) == -1  # 16 pages of 64 do not cover 2000 tokens
+
+
+def test_combine_and_append_validation(so):
+    d = _dims()
+    assert so.mla_combine(ctypes.byref(d), None, None, None, 4, None, None, None) == -1
+    fake = ctypes.c_void_p(1 << 20)
+    assert so.mla_append_kv(ctypes.byref(d), fake, 0, 7168, fake, None, 1e-6, 1e4, fake, fake, fake, 16, 1, fake,
+                            10, fake, 1 << 30, None) == -1
+    assert so.mla_append_kv(ctypes.byref(d), fake, 64, 7168, fake, None, 1e-6, 1e4, fake, fake, fake, 16, 1, fake,
+                            10, fake, 16, None) == -3
+
+
+def test_valid_call_without_gpu_reports_no_device(so):
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _decode(so, _dims()) == -7
+    assert so.mla_combine(ctypes.byref(_dims()), ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 20),
+                          ctypes.c_void_p(1 << 20), 4, ctypes.c_void_p(1 << 20), None, None) == -7
+
+
+def test_python_binding_has_no_cpu_path():
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    w = I.WORKLOADS["tiny_b1_l128"]
+    q = torch.zeros(1, 1, 16, 32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        L.decode(w.dims, w.softmax_scale, q, q, q, q, q, 128, q, q)

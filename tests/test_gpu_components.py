@@ -1,0 +1,128 @@
+"""GPU parity of the non-decode entry points through the C ABI: the split-KV
+combine, the page resolver (bit-exact) and the fused cache append."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from mla_latent_kv_29_b200 import inputs as I
+from oracle import mla_oracle as O
+
+from _data import build, oracle_append_pool, to_device, tolerance_ok
+
+pytestmark = pytest.mark.gpu
+
+
+def _lib():
+    from mla_latent_kv_29_b200 import lib
+
+    return lib
+
+
+# ------------------------------------------------------------------ combine
+@pytest.mark.parametrize("dims", [I.V3, I.TINY])
+def test_combine_matches_oracle_merge(dims):
+    L = _lib()
+    g = torch.Generator().manual_seed(4242)
+    counts = [1, 3, 0, 7, 2, 64, 65, 1]  # 0: a group with no parts; 65: more than one merge chunk
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    n, H, dc = int(offs[-1]), dims.num_heads, dims.kv_lora_rank
+    o = torch.randn(n, H, dc, generator=g)
+    lse = torch.randn(n, H, generator=g) * 4
+    lse[offs[1]:offs[2]][1] = -math.inf          # an empty split
+    lse[offs[4]:offs[5]] = -math.inf             # a group whose parts are all empty
+    dev = "cuda"
+    lse_out = torch.empty(len(counts), H, device=dev)
+    got = L.combine(dims, o.to(dev), lse.to(dev), torch.from_numpy(offs).to(dev), lse_out=lse_out)
+    torch.cuda.synchronize()
+    got, lse_got = got.cpu().numpy(), lse_out.cpu().numpy()
+    for gi in range(len(counts)):
+        a, b = offs[gi], offs[gi + 1]
+        if a == b:
+            np.testing.assert_array_equal(got[gi], 0.0)
+            assert np.all(lse_got[gi] == -np.inf)
+            continue
+        ref, ref_lse = O.merge_partials(o[a:b].numpy(), lse[a:b].numpy())
+        ok, err, bound = tolerance_ok(got[gi], ref)
+        assert ok, (gi, err, bound)
+        finite = np.isfinite(ref_lse)
+        np.testing.assert_array_equal(np.isfinite(lse_got[gi]), finite)
+        np.testing.assert_allclose(lse_got[gi][finite], ref_lse[finite], rtol=1e-5, atol=1e-5)
+
+
+# ---------------------------------------------------------------- resolver
+def test_resolve_slots_bit_exact():
+    L = _lib()
+    w = I.WORKLOADS["v3_b64_l1k_8k"]
+    lengths = I.context_lengths(w)
+    table, nblk = I.block_table(w, lengths)
+    g = torch.Generator().manual_seed(9)
+    n = 20000
+    seq = torch.randint(0, w.batch, (n,), generator=g, dtype=torch.int32)
+    pos = (torch.rand(n, generator=g) * lengths[seq.long()].float()).to(torch.int32)
+    # out-of-range probes: sequence, negative position, position past the table row
+    seq = torch.cat([seq, torch.tensor([-1, 64, 0, 0], dtype=torch.int32)])
+    pos = torch.cat([pos, torch.tensor([0, 0, -3, table.shape[1] * 64], dtype=torch.int32)])
+    rows = L.resolve_slots(w.dims, table.cuda(), nblk, seq.cuda(), pos.cuda()).cpu()
+    tab = table.numpy()
+    ref = [O.resolve_slot(tab, int(b), int(t), 64) for b, t in zip(seq[:n].tolist(), pos[:n].tolist())]
+    assert rows[:n].tolist() == ref
+    assert rows[n:].tolist() == [-1, -1, -1, -1]
+
+
+# ------------------------------------------------------------------ append
+def _append_case(n_seqs, per_seq, hidden, seed):
+    w = I.scaled(I.WORKLOADS["v3_b16_sq4_l16k_append"], batch=n_seqs, q_len=per_seq, length=300,
+                 name=f"append_{seed}", seed=seed, append_hidden=hidden)
+    return w
+
+
+@pytest.mark.parametrize("n_seqs,per_seq,hidden", [(3, 1, 256), (5, 4, 7168), (16, 4, 7168), (2, 40, 512)])
+def test_append_matches_oracle_and_touches_only_its_rows(n_seqs, per_seq, hidden):
+    L = _lib()
+    w = _append_case(n_seqs, per_seq, hidden, 31 + n_seqs)
+    data = build(w, fill=float("nan"))
+    ref_pool = oracle_append_pool(w, data)
+    dd = to_device(data)
+    before = dd["pool"].clone()
+    ap = dd["append"]
+    L.append_kv(w.dims, ap["x"], ap["w_kva"], ap["seq_ids"], ap["positions"], dd["table"], dd["pool"])
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    after = dd["pool"].cpu()
+    d = w.dims
+    flat_a, flat_b = after.view(-1, d.row_width), before.cpu().view(-1, d.row_width)
+    tab = data["table"].numpy()
+    slots = [O.resolve_slot(tab, int(b), int(p), d.block_size)
+             for b, p in zip(data["append"]["seq_ids"].tolist(), data["append"]["positions"].tolist())]
+    mask = torch.ones(flat_a.shape[0], dtype=torch.bool)
+    mask[slots] = False
+    # every other row is untouched, bit for bit (NaN sentinels included)
+    assert torch.equal(flat_a[mask].view(torch.int16), flat_b[mask].view(torch.int16))
+    # the written rows match the oracle's fp64 rows
+    ref_rows = O.append_rows(data["append"]["x"], data["append"]["w_kva"], data["append"]["positions"].numpy(),
+                             d.kv_lora_rank)
+    got = flat_a[slots].float().numpy()
+    ok, err, bound = tolerance_ok(got, ref_rows)
+    assert ok, (err, bound)
+    # elementwise: one bf16 rounding plus fp32 accumulation error
+    assert np.all(np.abs(got - ref_rows) <= 2.0 ** -8 * np.abs(ref_rows) + 2e-3)
+    # and the oracle's own bf16 storage of those rows differs by at most one bf16 step
+    ref_bf16 = ref_pool.view(-1, d.row_width)[slots].float().numpy()
+    assert np.all(np.abs(got - ref_bf16) <= 2.0 ** -7 * np.abs(ref_bf16) + 1e-3)
+
+
+def test_append_bad_slot_is_skipped_and_reported():
+    L = _lib()
+    w = _append_case(2, 2, 128, 77)
+    data = build(w, fill=0.0)
+    data["append"]["seq_ids"][1] = 5  # no such sequence
+    dd = to_device(data)
+    before = dd["pool"].clone()
+    ap = dd["append"]
+    L.device_error()
+    L.append_kv(w.dims, ap["x"], ap["w_kva"], ap["seq_ids"], ap["positions"], dd["table"], dd["pool"])
+    assert L.device_error() == -5
+    changed = (dd["pool"] != before).any(-1).view(-1).sum().item()
+    assert changed == 3  # the three valid tokens were written

@@ -1,0 +1,151 @@
+"""GPU parity of mla_decode against the fp64 oracle, through the C ABI.
+
+Tolerance (the stated bar for bf16 inputs with fp32 accumulation):
+max|err| <= 2e-2 * max|ref| + 1e-3 over each compared output tensor.
+Small cases compare every output; full-size workloads compare every head of
+a seeded sample of sequences (the oracle decompresses K and V explicitly,
+which costs H * L * d_c * (d_n + d_v) multiply-adds per sequence).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from mla_latent_kv_29_b200 import inputs as I
+from oracle import mla_oracle as O
+
+from _data import build, oracle_append_pool, to_device, tolerance_ok
+
+pytestmark = pytest.mark.gpu
+
+KERNELS = {"generic": 2}
+
+
+def _lib():
+    from mla_latent_kv_29_b200 import lib
+
+    return lib
+
+
+def run_decode(w, dd, kernel=0, num_workers=0, pool=None):
+    L = _lib()
+    out = L.decode(w.dims, w.softmax_scale, dd["q_nope"], dd["q_pe"], dd["pool"] if pool is None else pool,
+                   dd["table"], dd["lengths"], int(dd["lengths"].max()), dd["w_uk"], dd["w_uv"],
+                   kernel=kernel, num_workers=num_workers)
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    return out.float().cpu().numpy()
+
+
+def oracle_out(w, data, batch_ids=None, pool=None):
+    return O.decode_paged(data["q_nope"], data["q_pe"], data["pool"] if pool is None else pool,
+                          data["table"].numpy(), data["lengths"], data["w_uk"], data["w_uv"], w.dims,
+                          w.softmax_scale, batch_ids=batch_ids)
+
+
+def check(got, ref, ids=None):
+    if ids is not None:
+        got, ref = got[ids], ref[ids]
+    assert np.all(np.isfinite(got))
+    ok, err, bound = tolerance_ok(got, ref)
+    assert ok, f"max|err| {err:.3e} > {bound:.3e}"
+    return err
+
+
+def small_v3(name, batch, q_len, lengths, paged=True, spare=0):
+    w = I.scaled(I.WORKLOADS["v3_b64_l1k_8k"], batch=batch, q_len=q_len, name=name, paged=paged,
+                 spare_blocks=spare)
+    return w, torch.tensor(lengths, dtype=torch.int32)
+
+
+@pytest.mark.parametrize("kernel", list(KERNELS))
+def test_tiny_config(kernel):
+    w = I.WORKLOADS["tiny_b1_l128"]
+    data = build(w)
+    got = run_decode(w, to_device(data), kernel=KERNELS[kernel])
+    check(got, oracle_out(w, data))
+
+
+@pytest.mark.parametrize("kernel", list(KERNELS))
+@pytest.mark.parametrize("case", [
+    ("ragged_sq1", 3, 1, [1, 65, 300]),
+    ("ragged_sq4", 2, 4, [4, 130]),
+    ("tiles_exact", 2, 1, [128, 256]),
+    ("one_page_tail", 4, 2, [63, 64, 65, 129]),
+])
+@pytest.mark.parametrize("workers", [0, 1, 5, 1000])
+def test_v3_small_cases(kernel, case, workers):
+    name, B, sq, lens = case
+    w, lengths = small_v3(name, B, sq, lens)
+    data = build(w, lengths=lengths)
+    got = run_decode(w, to_device(data), kernel=KERNELS[kernel], num_workers=workers)
+    check(got, oracle_out(w, data))
+
+
+@pytest.mark.parametrize("kernel", list(KERNELS))
+def test_nan_in_unused_rows_and_blocks(kernel):
+    w, lengths = small_v3("nan_fill", 3, 2, [70, 5, 200], spare=3)
+    data = build(w, fill=float("nan"), lengths=lengths)
+    got = run_decode(w, to_device(data), kernel=KERNELS[kernel], num_workers=7)
+    check(got, oracle_out(w, data))
+
+
+@pytest.mark.parametrize("kernel", list(KERNELS))
+def test_paged_and_contiguous_layouts_agree_bitwise(kernel):
+    lens = [300, 77]
+    wp, lengths = small_v3("layout", 2, 1, lens, paged=True)
+    wc = I.scaled(wp, name="layout", paged=False)
+    dp = build(wp, lengths=lengths)
+    dc = build(wc, lengths=lengths)
+    assert not torch.equal(dp["table"], dc["table"])
+    a = run_decode(wp, to_device(dp), kernel=KERNELS[kernel], num_workers=3)
+    b = run_decode(wc, to_device(dc), kernel=KERNELS[kernel], num_workers=3)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_bad_block_id_sets_device_fault():
+    L = _lib()
+    w, lengths = small_v3("bad_block", 2, 1, [100, 100])
+    data = build(w, lengths=lengths)
+    data["table"][1, 1] = 10_000  # outside the pool
+    dd = to_device(data)
+    L.device_error()  # clear
+    out = L.decode(w.dims, w.softmax_scale, dd["q_nope"], dd["q_pe"], dd["pool"], dd["table"], dd["lengths"],
+                   100, dd["w_uk"], dd["w_uv"], kernel=2)
+    assert L.device_error() == -5
+    got = out.float().cpu().numpy()
+    ref = oracle_out(w, data, batch_ids=[0])
+    check(got, ref, ids=[0])  # the healthy sequence is unaffected
+    assert L.device_error() == 0  # cleared by the read
+
+
+# ---------------------------------------------------------------- full size
+def _sample(w, k):
+    g = torch.Generator().manual_seed(w.seed + 77)
+    return sorted(torch.randperm(w.batch, generator=g)[:k].tolist())
+
+
+@pytest.mark.parametrize("name,k", [("v3_b1_l4096", 1), ("v3_b64_l1k_8k", 3), ("v3_b8_l32k", 1)])
+def test_full_size_workloads(name, k):
+    w = I.WORKLOADS[name]
+    data = build(w)
+    dd = to_device(data)
+    ids = _sample(w, k)
+    ref = oracle_out(w, data, batch_ids=ids)
+    got = run_decode(w, dd)
+    check(got, ref, ids=ids)
+    assert np.all(np.isfinite(got))
+
+
+def test_full_size_sq4_with_append():
+    L = _lib()
+    w = I.WORKLOADS["v3_b16_sq4_l16k_append"]
+    data = build(w, fill=float("nan"))
+    dd = to_device(data)
+    ap = dd["append"]
+    L.append_kv(w.dims, ap["x"], ap["w_kva"], ap["seq_ids"], ap["positions"], dd["table"], dd["pool"])
+    got = run_decode(w, dd)
+    ids = _sample(w, 2)
+    ref = oracle_out(w, data, batch_ids=ids, pool=oracle_append_pool(w, data))
+    check(got, ref, ids=ids)
