@@ -91,8 +91,15 @@ def c_dims(d: Dims, softmax_scale: float) -> CDims:
                  float(softmax_scale))
 
 
+def _event_handle(ev) -> Optional[int]:
+    # torch creates the CUDA event on its first record(); make sure the handle exists
+    if ev.cuda_event == 0:
+        ev.record()
+    return ev.cuda_event
+
+
 def c_opts(kernel: int = KERNEL_AUTO, num_workers: int = 0, events=None) -> CDecodeOpts:
-    b, e = (None, None) if events is None else (events[0].cuda_event, events[1].cuda_event)
+    b, e = (None, None) if events is None else (_event_handle(events[0]), _event_handle(events[1]))
     return CDecodeOpts(int(kernel), int(num_workers), b, e)
 
 
