@@ -54,7 +54,9 @@ typedef enum mla_status {
     MLA_ERR_CUDA = -4,                /* a CUDA runtime call or launch failed */
     MLA_ERR_DEVICE_FAULT = -5,        /* device error word: bad block id / slot / position */
     MLA_ERR_DEVICE_TIMEOUT = -6,      /* device error word: a bounded wait expired */
-    MLA_ERR_NO_DEVICE = -7            /* no sm_100 device is current */
+    MLA_ERR_NO_DEVICE = -7,           /* no sm_100 device is current */
+    MLA_ERR_SCRATCH_LIMIT = -8        /* mla_decode_no_alloc: the problem needs more
+                                         scratch than MLA_NO_ALLOC_SCRATCH_BYTES */
 } mla_status_t;
 
 /* Per-layer sizes. DeepSeek-V3: {128, 512, 64, 128, 128, 64, 1/sqrt(192)}
@@ -159,6 +161,44 @@ MLA_API int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q
 
 MLA_API size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t batch, int32_t q_len,
                                  int32_t max_context_len, const mla_decode_opts_t* opts);
+
+/* ------------------------------------------------------------------ */
+/* mla_decode for callers that cannot allocate device memory. The paper
+ * has no counterpart: this is a deployment convenience of this library.
+ *
+ * Some callers cannot call cudaMalloc (or any allocator): a plugin whose
+ * host process owns all device memory through its own pooled allocator and
+ * forbids raw allocations, a latency-critical path that cannot afford the
+ * device-wide synchronisation cudaMalloc/cudaFree may cause, or plain C code
+ * with no memory manager at all. They still pass every input and output
+ * buffer; only the decode scratch (split-KV schedule, absorbed queries and
+ * partial results, the same bytes mla_decode_workspace_size() reports) comes
+ * from a fixed buffer compiled into the library: a static device array of
+ * MLA_NO_ALLOC_SCRATCH_BYTES, which every GPU that loads the library holds
+ * until the process exits.
+ *
+ * Arguments and results are those of mla_decode without the workspace.
+ * Returns MLA_ERR_SCRATCH_LIMIT, before enqueuing anything, when the
+ * problem needs more scratch than the buffer holds (for DeepSeek-V3 dims
+ * the default schedule fits batch * q_len up to 64).
+ *
+ * Set-up: the first call on each device looks up the buffer's device
+ * address (cudaGetSymbolAddress, with that device current) and caches it;
+ * make that first call before any stream capture on that device.
+ * Sharing: every call on a device uses the same buffer and leaves its
+ * contents behind. Nothing in it needs to start at zero (each call writes
+ * every scratch byte it later reads), but calls whose work overlaps on the
+ * GPU (different streams, no ordering between them) race on the buffer:
+ * order them on one stream or with events. */
+#define MLA_NO_ALLOC_SCRATCH_BYTES (48u * 1024u * 1024u)
+
+MLA_API int mla_decode_no_alloc(const mla_dims_t* dims, const void* q_nope, const void* q_pe,
+                                int32_t batch, int32_t q_len,
+                                const void* pool, int64_t num_blocks,
+                                const int32_t* block_table, int32_t max_blocks_per_seq,
+                                const int32_t* context_lens, int32_t max_context_len,
+                                const void* w_uk, const void* w_uv, void* out,
+                                const mla_decode_opts_t* opts, void* stream);
 
 /* ------------------------------------------------------------------ */
 /* Log-sum-exp combine of split-KV partials (the merge the split decode

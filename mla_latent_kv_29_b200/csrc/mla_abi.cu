@@ -4,6 +4,7 @@
 // is to synchronise and read the device status word).
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "mla_b200.h"
 #include "common.cuh"
@@ -154,6 +155,7 @@ const char* mla_error_string(int s) {
         case MLA_ERR_DEVICE_FAULT: return "device fault: block id, slot or position out of range";
         case MLA_ERR_DEVICE_TIMEOUT: return "device timeout: a bounded wait expired";
         case MLA_ERR_NO_DEVICE: return "no sm_100 CUDA device is current";
+        case MLA_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the fixed no-allocation buffer";
         default: return "unknown status";
     }
 }
@@ -320,3 +322,58 @@ int mla_debug_resolve_slots(const mla_dims_t* dims, const int32_t* block_table, 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without allocation: the scratch comes from a buffer compiled into
+// the library instead of a caller-provided workspace. It exists for callers
+// that cannot allocate device memory themselves (see mla_b200.h). Host code
+// must not pass `g_no_alloc_scratch` itself to a kernel: on the host that
+// name is only a stand-in for the symbol. The device address is looked up
+// with cudaGetSymbolAddress once per device, with that device current.
+namespace mla {
+namespace {
+
+static __device__ __align__(256) unsigned char g_no_alloc_scratch[MLA_NO_ALLOC_SCRATCH_BYTES];
+
+std::mutex g_no_alloc_mutex;
+void* g_no_alloc_ptr[64] = {nullptr};
+
+int no_alloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return MLA_ERR_NO_DEVICE; }
+    if (dev < 0 || dev >= 64) return MLA_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lock(g_no_alloc_mutex);
+    if (!g_no_alloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_no_alloc_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return MLA_ERR_CUDA;
+        }
+        g_no_alloc_ptr[dev] = p;
+    }
+    *out = g_no_alloc_ptr[dev];
+    return MLA_OK;
+}
+
+}  // namespace
+}  // namespace mla
+
+extern "C" int mla_decode_no_alloc(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int32_t batch,
+                                   int32_t q_len, const void* pool, int64_t num_blocks, const int32_t* block_table,
+                                   int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                   int32_t max_context_len, const void* w_uk, const void* w_uv, void* out,
+                                   const mla_decode_opts_t* opts, void* stream) {
+    const size_t need = mla_decode_workspace_size(dims, batch, q_len, max_context_len, opts);
+    if (need == 0) {  // same validation verdict as mla_decode
+        DecodeLayout L;
+        const int rc = decode_layout(dims, batch, q_len, max_context_len, opts, &L);
+        return rc ? rc : MLA_ERR_INVALID_ARG;
+    }
+    if (need > MLA_NO_ALLOC_SCRATCH_BYTES) return MLA_ERR_SCRATCH_LIMIT;
+    if (int rc = device_ok()) return rc;
+    void* scratch = nullptr;
+    if (int rc = no_alloc_scratch(&scratch)) return rc;
+    return mla_decode(dims, q_nope, q_pe, batch, q_len, pool, num_blocks, block_table, max_blocks_per_seq,
+                      context_lens, max_context_len, w_uk, w_uv, out, scratch, MLA_NO_ALLOC_SCRATCH_BYTES, opts,
+                      stream);
+}

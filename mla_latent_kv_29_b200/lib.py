@@ -23,13 +23,14 @@ MLA_OK = 0
 STATUS_NAMES = {
     0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED_DIMS",
     -3: "MLA_ERR_WORKSPACE_TOO_SMALL", -4: "MLA_ERR_CUDA", -5: "MLA_ERR_DEVICE_FAULT",
-    -6: "MLA_ERR_DEVICE_TIMEOUT", -7: "MLA_ERR_NO_DEVICE",
+    -6: "MLA_ERR_DEVICE_TIMEOUT", -7: "MLA_ERR_NO_DEVICE", -8: "MLA_ERR_SCRATCH_LIMIT",
 }
+NO_ALLOC_SCRATCH_BYTES = 48 * 1024 * 1024  # MLA_NO_ALLOC_SCRATCH_BYTES
 KERNEL_AUTO, KERNEL_SM100, KERNEL_GENERIC = 0, 1, 2
 
 EXPORTED = ("mla_append_kv", "mla_append_workspace_size", "mla_decode", "mla_decode_workspace_size",
             "mla_combine", "mla_debug_resolve_slots", "mla_get_device_error", "mla_error_string",
-            "mla_version")
+            "mla_version", "mla_decode_no_alloc")
 
 
 class MLAError(RuntimeError):
@@ -73,6 +74,7 @@ def load():
         "mla_get_device_error": (_I32, [ctypes.POINTER(ctypes.c_int), _P]),
         "mla_error_string": (ctypes.c_char_p, [_I32]),
         "mla_version": (_I32, []),
+        "mla_decode_no_alloc": (_I32, [D, _P, _P, _I32, _I32, _P, _I64, _P, _I32, _P, _I32, _P, _P, _P, O, _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -186,6 +188,26 @@ def decode(dims: Dims, softmax_scale: float, q_nope, q_pe, pool, block_table, co
         _ptr(out, torch.bfloat16, "out"), _ptr(workspace, None, "workspace"),
         workspace.numel() * workspace.element_size(), ctypes.byref(o), _stream(stream))
     _check(st, "mla_decode")
+    return out
+
+
+def decode_no_alloc(dims: Dims, softmax_scale: float, q_nope, q_pe, pool, block_table, context_lens,
+                    max_context_len: int, w_uk, w_uv, out=None, kernel: int = KERNEL_AUTO, num_workers: int = 0,
+                    stream=None):
+    """mla_decode with the library's built-in scratch buffer (no workspace argument)."""
+    lib = load()
+    cd = c_dims(dims, softmax_scale)
+    o = c_opts(kernel, num_workers)
+    B, Sq = q_nope.shape[0], q_nope.shape[1]
+    if out is None:
+        out = torch.empty(B, Sq, dims.num_heads, dims.v_head_dim, dtype=torch.bfloat16, device=q_nope.device)
+    st = lib.mla_decode_no_alloc(
+        ctypes.byref(cd), _ptr(q_nope, torch.bfloat16, "q_nope"), _ptr(q_pe, torch.bfloat16, "q_pe"), B, Sq,
+        _ptr(pool, torch.bfloat16, "pool"), pool.shape[0], _ptr(block_table, torch.int32, "block_table"),
+        block_table.shape[1], _ptr(context_lens, torch.int32, "context_lens"), int(max_context_len),
+        _ptr(w_uk, torch.bfloat16, "w_uk"), _ptr(w_uv, torch.bfloat16, "w_uv"),
+        _ptr(out, torch.bfloat16, "out"), ctypes.byref(o), _stream(stream))
+    _check(st, "mla_decode_no_alloc")
     return out
 
 
