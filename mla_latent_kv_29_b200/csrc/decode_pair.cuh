@@ -1,0 +1,476 @@
+// Split-KV absorbed MLA attention on the sm_100a tensor cores (DeepSeek-V3
+// dims: 128 heads, latent 512, RoPE 64).
+//
+// Per new token g and split segment [tok_begin, tok_end) of its visible
+// tokens: S = scale * [q_lat ; q_pe] . [c ; k_pe]^T over all 128 heads at once
+// (the absorbed score of "一次讲透MHA、GQA、MQA、MLA", section "MLA的实现"; all
+// heads share the latent tile, so it is a dense [128 x 576] . [576 x tokens]
+// contraction), online softmax, O += P . c (the [128 x tokens] .
+// [tokens x 512] value contraction), then the normalised partial (O / l,
+// lse) of the segment.
+//
+// Work split. One worker is a cluster of two CTAs (a pair). Tensor-core MMAs
+// are issued by the pair's leader with cta_group::2 and M = 128 heads: CTA r
+// holds heads 64r..64r+63 of every operand A (queries, softmax weights) and
+// of every accumulator, folded over all 128 TMEM lanes (columns [0, N/2) of
+// the result in lanes 0-63, [N/2, N) in lanes 64-127), and supplies half of
+// every operand B:
+//   S MMA  (M 128, N 128 tokens, K 576): CTA r supplies the 64 tokens of its
+//          page of the 128-token tile (all 576 values per token);
+//   PV MMA (M 128, N 256 latent columns, K 128 tokens), twice per tile:
+//          CTA r supplies latent columns 256r + 128n .. +127 for all tokens.
+// The tile's latent values therefore reach each CTA twice (once as keys,
+// once as values), so shared-memory fills are ~1.9x the HBM bytes, while
+// HBM reads stay ~1x because the second read of a page hits L2.
+//
+// Warp roles per CTA (256 threads): warp 0 streams TMA boxes into a ring of
+// 8 KB stages; warp 1 allocates tensor memory (both CTAs) and, in the
+// leader, issues MMAs; warps 4-7 (thread t = TMEM lane t) run the softmax,
+// rescale O when the running max grows by more than 2^8, write P to shared
+// memory and, at the end of a segment, normalise O and write the partial.
+// Every mbarrier wait is bounded (see ptx::mbar_wait): on expiry the kernel
+// records MLA_ERR_DEVICE_TIMEOUT and every role drains to the common exit.
+#pragma once
+
+#include "common.cuh"
+#include "plan.cuh"
+#include "sm100.cuh"
+
+namespace mla {
+namespace pair {
+
+constexpr int kH = 128, kDc = 512, kDr = 64, kD = kDc + kDr;
+constexpr int kTile = 128;       // tokens per pair iteration
+constexpr int kBox = 8192;       // one [64 rows x 64 bf16] 128B-swizzled box = one ring stage
+constexpr int kQBoxes = kD / 64; // 9
+constexpr int kStages = 12;
+constexpr int kThreads = 256;
+constexpr int kTmemCols = 512;
+constexpr int kTmS = 0;          // two S buffers of 64 columns
+constexpr int kTmO = 128;        // O: 256 columns
+
+constexpr int kOffQ = 0;
+constexpr int kOffRing = kOffQ + kQBoxes * kBox;
+constexpr int kOffP = kOffRing + kStages * kBox;
+constexpr int kOffBar = kOffP + 2 * kBox;
+
+enum Bar {
+    B_QFULL = 0, B_QEMPTY, B_SFULL0, B_SFULL1, B_SEMPTY0, B_SEMPTY1, B_PFULL, B_PVDONE, B_OEMPTY, B_PATCH, B_XCHG,
+    B_KVFULL0, B_KVEMPTY0 = B_KVFULL0 + kStages, B_COUNT = B_KVEMPTY0 + kStages
+};
+constexpr int kOffRed = kOffBar + 8 * 64;          // exchange buffer [2][128] floats
+constexpr int kOffMisc = kOffRed + 2 * 128 * 4;    // abort flag, TMEM base
+constexpr int kSmemBytes = kOffMisc + 64 + 1024;   // + slack to align the base to 1 KB
+static_assert(B_COUNT <= 64, "barrier area");
+
+struct Params {
+    const PlanHeader* hdr;
+    const int32_t* tile_prefix;
+    const int32_t* part_offsets;
+    const int32_t* context_lens;
+    const int32_t* block_table;
+    float* o_part;  // [n_parts, 128, 512]
+    float* lse_part;  // [n_parts, 128]
+    int64_t num_blocks;
+    int32_t batch, max_blocks_per_seq, block_size, q_len;
+    float scale_log2;  // softmax_scale * log2(e)
+};
+
+struct Ctx {
+    uint8_t* smem;
+    uint32_t sbase;
+    uint32_t rank;
+    uint32_t pair;
+    uint32_t tmem;
+    volatile int* abort;
+    __device__ uint32_t bar(int i) const { return sbase + kOffBar + 8 * i; }
+    __device__ uint32_t leader_bar(int i) const { return ptx::mapa(bar(i), 0); }
+};
+
+__device__ __forceinline__ int tiles_of(const Segment& s) { return (s.tok_end - s.tok_begin + kTile - 1) / kTile; }
+
+// ------------------------------------------------------------------ producer
+__device__ __forceinline__ bool ring_slot(const Ctx& c, uint32_t& stage, uint32_t& phase, uint32_t& slot_full) {
+    if (!ptx::mbar_wait(c.bar(B_KVEMPTY0 + stage), phase ^ 1, c.abort)) return false;
+    slot_full = c.leader_bar(B_KVFULL0 + stage);
+    return true;
+}
+
+__device__ __forceinline__ void ring_next(uint32_t& stage, uint32_t& phase) {
+    if (++stage == kStages) { stage = 0; phase ^= 1; }
+}
+
+__device__ void producer(const Params& P, const CUtensorMap* tm_q, const CUtensorMap* tm_kv64,
+                         const CUtensorMap* tm_kv32, const Ctx& c) {
+    const uint32_t lane = ptx::lane_id();
+    uint32_t stage = 0, phase = 0, patch_phase = 0;
+    int seg_i = 0;
+    SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    Segment seg;
+    while (it.next(seg)) {
+        const int32_t g = seg.group, b = g / P.q_len;
+        if (seg_i > 0 && !ptx::mbar_wait(c.bar(B_QEMPTY), (seg_i - 1) & 1, c.abort)) return;
+        if (lane == 0) {
+            const uint32_t full = c.leader_bar(B_QFULL);
+            ptx::mbar_arrive_expect_tx_cluster(full, kQBoxes * kBox);
+            for (int k = 0; k < kQBoxes; ++k)
+                ptx::tma_load_2d_pair(c.sbase + kOffQ + k * kBox, tm_q, 64 * k, g * kH + 64 * c.rank, full);
+        }
+        __syncwarp();
+        const int n_tiles = tiles_of(seg);
+        for (int j = 0; j <= n_tiles; ++j) {
+            if (j < n_tiles) {  // key boxes of tile j: this CTA's 64-token page, all 576 values
+                const int32_t t0 = seg.tok_begin + j * kTile;
+                int32_t th = t0 + 64 * static_cast<int32_t>(c.rank);
+                if (th >= seg.tok_end) th = t0;  // no visible token in this half: any valid page (masked)
+                int64_t row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks,
+                                          P.block_size, b, th);
+                if (row < 0) {
+                    if (lane == 0) record_status(MLA_ERR_DEVICE_FAULT);
+                    row = 0;
+                }
+                for (int k = 0; k < kQBoxes; ++k) {
+                    uint32_t full;
+                    if (!ring_slot(c, stage, phase, full)) return;
+                    if (lane == 0) {
+                        ptx::mbar_arrive_expect_tx_cluster(full, kBox);
+                        ptx::tma_load_2d_pair(c.sbase + kOffRing + stage * kBox, tm_kv64, 64 * k,
+                                              static_cast<int32_t>(row), full);
+                    }
+                    __syncwarp();
+                    ring_next(stage, phase);
+                }
+            }
+            if (j >= 1) {  // value boxes of tile j-1: 32 tokens x this CTA's 128 latent columns per stage
+                const int32_t tv = seg.tok_begin + (j - 1) * kTile;
+                for (int q = 0; q < 4; ++q) {
+                    const int32_t tq = tv + 32 * q;
+                    const int nv = max(0, min(32, seg.tok_end - tq));
+                    int64_t row = -1;
+                    if (nv > 0) {
+                        row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks, P.block_size,
+                                          b, tq);
+                        if (row < 0 && lane == 0) record_status(MLA_ERR_DEVICE_FAULT);
+                    }
+                    for (int n = 0; n < 2; ++n) {
+                        uint32_t full;
+                        if (!ring_slot(c, stage, phase, full)) return;
+                        const uint32_t dst = c.sbase + kOffRing + stage * kBox;
+                        const int32_t x0 = 256 * static_cast<int32_t>(c.rank) + 128 * n;
+                        if (row >= 0 && nv == 32) {
+                            if (lane == 0) {
+                                ptx::mbar_arrive_expect_tx_cluster(full, kBox);
+                                ptx::tma_load_2d_pair(dst, tm_kv32, x0, static_cast<int32_t>(row), full);
+                                ptx::tma_load_2d_pair(dst + kBox / 2, tm_kv32, x0 + 64, static_cast<int32_t>(row), full);
+                            }
+                        } else {
+                            // Tail of the visible range: rows past it may hold anything (even NaN),
+                            // and 0 * NaN would poison O, so they are zeroed before the MMA reads them.
+                            int keep = 0;
+                            if (row >= 0) {
+                                if (lane == 0) {
+                                    ptx::mbar_arrive_expect_tx_local(c.bar(B_PATCH), kBox);
+                                    ptx::tma_load_2d(dst, tm_kv32, x0, static_cast<int32_t>(row), c.bar(B_PATCH));
+                                    ptx::tma_load_2d(dst + kBox / 2, tm_kv32, x0 + 64, static_cast<int32_t>(row),
+                                                     c.bar(B_PATCH));
+                                }
+                                if (!ptx::mbar_wait(c.bar(B_PATCH), patch_phase, c.abort)) return;
+                                patch_phase ^= 1;
+                                keep = nv;
+                            }
+                            uint4* p = reinterpret_cast<uint4*>(c.smem + kOffRing + stage * kBox);
+                            for (int i = lane; i < kBox / 16; i += 32) {
+                                const int r = (i & 255) >> 3;  // token row within its 4 KB box
+                                if (r >= keep) p[i] = make_uint4(0u, 0u, 0u, 0u);
+                            }
+                            ptx::fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) ptx::mbar_arrive_cluster(full);
+                        }
+                        __syncwarp();
+                        ring_next(stage, phase);
+                    }
+                }
+            }
+        }
+        ++seg_i;
+    }
+}
+
+// ------------------------------------------------------------------- MMA
+__device__ void mma_issuer(const Params& P, const Ctx& c) {
+    constexpr uint32_t kIdS = ptx::idesc_bf16(128, 128, false, false);
+    constexpr uint32_t kIdPV = ptx::idesc_bf16(128, 256, false, true);
+    const uint32_t lane = ptx::lane_id();
+    uint32_t stage = 0, phase = 0, tile_cnt = 0, pv_cnt = 0;
+    int seg_i = 0;
+    SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    Segment seg;
+    while (it.next(seg)) {
+        if (!ptx::mbar_wait(c.bar(B_QFULL), seg_i & 1, c.abort)) return;
+        ptx::tc_fence_after();
+        const int n_tiles = tiles_of(seg);
+        for (int j = 0; j <= n_tiles; ++j) {
+            if (j < n_tiles) {  // S = Q K^T for tile j into S buffer sb
+                const uint32_t sb = tile_cnt & 1;
+                if (!ptx::mbar_wait(c.bar(B_SEMPTY0 + sb), ((tile_cnt >> 1) & 1) ^ 1, c.abort)) return;
+                ptx::tc_fence_after();
+                for (int k = 0; k < kQBoxes; ++k) {
+                    if (!ptx::mbar_wait(c.bar(B_KVFULL0 + stage), phase, c.abort)) return;
+                    ptx::tc_fence_after();
+                    if (lane == 0) {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t a = ptx::smem_desc_sw128(c.sbase + kOffQ + k * kBox + 32 * kk, 16, 1024);
+                            const uint64_t bd =
+                                ptx::smem_desc_sw128(c.sbase + kOffRing + stage * kBox + 32 * kk, 16, 1024);
+                            ptx::mma_bf16_pair(c.tmem + kTmS + 64 * sb, a, bd, kIdS, (k | kk) != 0);
+                        }
+                        ptx::mma_commit_pair(c.bar(B_KVEMPTY0 + stage), 0x3);
+                    }
+                    __syncwarp();
+                    ring_next(stage, phase);
+                }
+                if (lane == 0) {
+                    ptx::mma_commit_pair(c.bar(B_SFULL0 + sb), 0x3);
+                    if (j == n_tiles - 1) ptx::mma_commit_pair(c.bar(B_QEMPTY), 0x3);
+                }
+                __syncwarp();
+                ++tile_cnt;
+            }
+            if (j >= 1) {  // O += P V for tile j-1
+                const bool first = (j == 1);
+                if (!ptx::mbar_wait(c.bar(B_PFULL), pv_cnt & 1, c.abort)) return;
+                if (first && !ptx::mbar_wait(c.bar(B_OEMPTY), (seg_i & 1) ^ 1, c.abort)) return;
+                ptx::tc_fence_after();
+                for (int q = 0; q < 4; ++q) {
+                    for (int n = 0; n < 2; ++n) {
+                        if (!ptx::mbar_wait(c.bar(B_KVFULL0 + stage), phase, c.abort)) return;
+                        ptx::tc_fence_after();
+                        if (lane == 0) {
+#pragma unroll
+                            for (int kk = 0; kk < 2; ++kk) {
+                                const uint32_t pa = c.sbase + kOffP + (q >> 1) * kBox + 64 * (q & 1) + 32 * kk;
+                                const uint64_t a = ptx::smem_desc_sw128(pa, 16, 1024);
+                                const uint64_t bd =
+                                    ptx::smem_desc_sw128(c.sbase + kOffRing + stage * kBox + 2048 * kk, kBox / 2, 1024);
+                                ptx::mma_bf16_pair(c.tmem + kTmO + 128 * n, a, bd, kIdPV, !(first && q == 0 && kk == 0));
+                            }
+                            ptx::mma_commit_pair(c.bar(B_KVEMPTY0 + stage), 0x3);
+                        }
+                        __syncwarp();
+                        ring_next(stage, phase);
+                    }
+                }
+                if (lane == 0) ptx::mma_commit_pair(c.bar(B_PVDONE), 0x3);
+                __syncwarp();
+                ++pv_cnt;
+            }
+        }
+        ++seg_i;
+    }
+}
+
+// --------------------------------------------------------------- softmax
+struct Exchanger {  // swaps one float between thread t and thread t ^ 64 of the softmax warps
+    float* red;
+    uint32_t bar;
+    uint32_t n = 0;
+    __device__ bool swap(float v, float& partner, int t, volatile int* abort) {
+        float* buf = red + (n & 1) * 128;
+        buf[t] = v;
+        __syncwarp();
+        if (ptx::lane_id() == 0) ptx::mbar_arrive_local(bar);
+        if (!ptx::mbar_wait(bar, n & 1, abort)) return false;
+        partner = buf[t ^ 64];
+        ++n;
+        return true;
+    }
+};
+
+__device__ void softmax(const Params& P, const Ctx& c) {
+    const int t = static_cast<int>(threadIdx.x) - 128;  // TMEM lane
+    const uint32_t lane = ptx::lane_id();
+    const int half = t >> 6, hrow = t & 63;
+    const int head = 64 * static_cast<int>(c.rank) + hrow;
+    const uint32_t tl = c.tmem + (static_cast<uint32_t>(t & ~31) << 16);  // this warp's lane quadrant
+    const uint32_t sempty[2] = {c.leader_bar(B_SEMPTY0), c.leader_bar(B_SEMPTY1)};
+    const uint32_t pfull = c.leader_bar(B_PFULL), oempty = c.leader_bar(B_OEMPTY);
+    uint8_t* prow = c.smem + kOffP + half * kBox + hrow * 128;
+    Exchanger xc{reinterpret_cast<float*>(c.smem + kOffRed), c.bar(B_XCHG)};
+    uint32_t tile_cnt = 0, pv_wait = 0;
+    SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    Segment seg;
+    while (it.next(seg)) {
+        float m_run = -INFINITY, l_run = 0.f;
+        const int n_tiles = tiles_of(seg);
+        for (int j = 0; j < n_tiles; ++j) {
+            const uint32_t sb = tile_cnt & 1;
+            if (!ptx::mbar_wait(c.bar(B_SFULL0 + sb), (tile_cnt >> 1) & 1, c.abort)) return;
+            ptx::tc_fence_after();
+            float s[64];
+            {
+                float (&s0)[32] = *reinterpret_cast<float(*)[32]>(&s[0]);
+                float (&s1)[32] = *reinterpret_cast<float(*)[32]>(&s[32]);
+                ptx::tmem_ld32(tl + kTmS + 64 * sb, s0);
+                ptx::tmem_ld32(tl + kTmS + 64 * sb + 32, s1);
+                ptx::tmem_wait_ld();
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_cluster(sempty[sb]);
+            ++tile_cnt;
+
+            const int32_t tok0 = seg.tok_begin + j * kTile + 64 * half;
+            const int nvalid = max(0, min(64, seg.tok_end - tok0));
+            float mloc = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                s[i] = i < nvalid ? s[i] * P.scale_log2 : -INFINITY;
+                mloc = fmaxf(mloc, s[i]);
+            }
+            float mpart;
+            if (!xc.swap(mloc, mpart, t, c.abort)) return;
+            const float m_tile = fmaxf(mloc, mpart);
+            const float m_new = fmaxf(m_run, m_tile);
+            const bool rescale = m_new > m_run + 8.f;  // keep a stale max unless it grows by > 2^8
+            const float m_use = rescale ? m_new : m_run;
+            const float alpha = rescale ? exp2f(m_run - m_new) : 1.f;
+            float psum = 0.f;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                s[i] = exp2f(s[i] - m_use);  // exp2(-inf) = 0 for masked tokens
+                psum += s[i];
+            }
+            l_run = l_run * alpha + psum;
+            if (j > 0) {  // PV of the previous tile must be done before P and O are touched
+                if (!ptx::mbar_wait(c.bar(B_PVDONE), pv_wait & 1, c.abort)) return;
+                ++pv_wait;
+                ptx::tc_fence_after();
+                if (rescale) {
+#pragma unroll 1
+                    for (int cc = 0; cc < 8; ++cc) {
+                        float o[32];
+                        ptx::tmem_ld32(tl + kTmO + 32 * cc, o);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                        ptx::tmem_st32(tl + kTmO + 32 * cc, o);
+                    }
+                    ptx::tmem_wait_st();
+                }
+            }
+            // P row (bf16) into the K-major 128B-swizzled A operand of the PV MMA
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) {
+                uint4 u;
+                u.x = pack_bf16x2(s[8 * c8 + 0], s[8 * c8 + 1]);
+                u.y = pack_bf16x2(s[8 * c8 + 2], s[8 * c8 + 3]);
+                u.z = pack_bf16x2(s[8 * c8 + 4], s[8 * c8 + 5]);
+                u.w = pack_bf16x2(s[8 * c8 + 6], s[8 * c8 + 7]);
+                *reinterpret_cast<uint4*>(prow + ((c8 ^ (hrow & 7)) << 4)) = u;
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_cluster(pfull);
+            m_run = m_use;
+        }
+        // segment epilogue: normalise O and write the partial
+        if (!ptx::mbar_wait(c.bar(B_PVDONE), pv_wait & 1, c.abort)) return;
+        ++pv_wait;
+        ptx::tc_fence_after();
+        float lpart;
+        if (!xc.swap(l_run, lpart, t, c.abort)) return;
+        const float l_tot = l_run + lpart;
+        const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+        float* dst = P.o_part + (static_cast<int64_t>(seg.slot) * kH + head) * kDc + 256 * half;
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+            float o[32];
+            ptx::tmem_ld32(tl + kTmO + 32 * cc, o);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4*>(dst + 32 * cc + i) =
+                    make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+        }
+        if (half == 0)
+            P.lse_part[static_cast<int64_t>(seg.slot) * kH + head] =
+                l_tot > 0.f ? (m_run + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(oempty);
+    }
+}
+
+// ------------------------------------------------------------------ kernel
+// grid: 2 * workers CTAs (clusters of 2); block 256; dynamic smem kSmemBytes.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    pair_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv64,
+                       const __grid_constant__ CUtensorMap tm_kv32, const Params P) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw = ptx::smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    const int warp = threadIdx.x >> 5;
+    Ctx c;
+    c.smem = smem;
+    c.sbase = ptx::smem_u32(smem);
+    c.rank = ptx::cluster_ctarank();
+    c.pair = ptx::cluster_id_x();
+    c.abort = reinterpret_cast<volatile int*>(smem + kOffMisc);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc + 16);
+
+    if (threadIdx.x == 0) {
+        *c.abort = 0;
+        ptx::mbar_init(c.bar(B_QFULL), 2);
+        ptx::mbar_init(c.bar(B_QEMPTY), 1);
+        ptx::mbar_init(c.bar(B_SFULL0), 1);
+        ptx::mbar_init(c.bar(B_SFULL1), 1);
+        ptx::mbar_init(c.bar(B_SEMPTY0), 8);
+        ptx::mbar_init(c.bar(B_SEMPTY1), 8);
+        ptx::mbar_init(c.bar(B_PFULL), 8);
+        ptx::mbar_init(c.bar(B_PVDONE), 1);
+        ptx::mbar_init(c.bar(B_OEMPTY), 8);
+        ptx::mbar_init(c.bar(B_PATCH), 1);
+        ptx::mbar_init(c.bar(B_XCHG), 4);
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(c.bar(B_KVFULL0 + s), 2);
+            ptx::mbar_init(c.bar(B_KVEMPTY0 + s), 1);
+        }
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && ptx::lane_id() == 0) {
+        ptx::prefetch_tmap(&tm_q);
+        ptx::prefetch_tmap(&tm_kv64);
+        ptx::prefetch_tmap(&tm_kv32);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), kTmemCols);
+        ptx::tmem_relinquish_pair();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync();  // the peer's barriers exist before anyone arrives on them
+    ptx::tc_fence_after();
+    c.tmem = *tmem_slot;
+
+    if (warp == 0) {
+        producer(P, &tm_q, &tm_kv64, &tm_kv32, c);
+    } else if (warp == 1) {
+        if (c.rank == 0) mma_issuer(P, c);
+    } else if (warp >= 4) {
+        softmax(P, c);
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync();  // no MMA or remote arrive targets this CTA any more
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc_pair(c.tmem, kTmemCols);
+    }
+}
+
+}  // namespace pair
+}  // namespace mla

@@ -13,6 +13,9 @@
 #include "combine.cuh"
 #include "decode_generic.cuh"
 #include "append.cuh"
+#include "decode_pair.cuh"
+
+#include <cudaTypedefs.h>
 
 namespace mla {
 namespace {
@@ -71,18 +74,58 @@ struct DecodeLayout {
     int32_t workers, max_parts, kernel, tile;
 };
 
+constexpr int kKernelPair = 1, kKernelGeneric = 2;
+
+// The tensor-core pair kernel is specialised to DeepSeek-V3 dims and needs
+// every 64-token half tile inside one page.
+bool pair_kernel_fits(const mla_dims_t* d) {
+    return d->num_heads == pair::kH && d->kv_lora_rank == pair::kDc && d->rope_dim == pair::kDr &&
+           d->block_size % 64 == 0;
+}
+
 int pick_kernel(const mla_dims_t* d, const mla_decode_opts_t* o) {
-    (void)d;
     const int k = o ? o->kernel : 0;
-    if (k == 0 || k == 2) return 2;
+    if (k == 0) return pair_kernel_fits(d) ? kKernelPair : kKernelGeneric;
+    if (k == kKernelPair) return pair_kernel_fits(d) ? kKernelPair : -1;
+    if (k == kKernelGeneric) return kKernelGeneric;
     return -1;
 }
 
 int default_workers(const mla_dims_t* d, int kernel) {
-    (void)kernel;
+    if (kernel == kKernelPair) return num_sms() / 2;  // one cluster of two CTAs per SM pair
     const int hb = (d->num_heads + kGenHeads - 1) / kGenHeads;
     const int target = 4 * num_sms();
     return target / hb > 0 ? target / hb : 1;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// 2-D bf16 tensor map over rows of `cols` values (row stride `cols` * 2 bytes),
+// box = box_rows x 64 values, 128-byte swizzle.
+int encode_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return MLA_ERR_CUDA;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
 int decode_layout(const mla_dims_t* d, int32_t batch, int32_t q_len, int32_t max_len,
@@ -93,7 +136,7 @@ int decode_layout(const mla_dims_t* d, int32_t batch, int32_t q_len, int32_t max
     const int kernel = pick_kernel(d, o);
     if (kernel < 0) return MLA_ERR_UNSUPPORTED_DIMS;
     L->kernel = kernel;
-    L->tile = kGenTokens;
+    L->tile = kernel == kKernelPair ? pair::kTile : kGenTokens;
     const int64_t G = static_cast<int64_t>(batch) * q_len;
     const int64_t tiles_per_group = (max_len + L->tile - 1) / L->tile;
     if (G * tiles_per_group >= (int64_t(1) << 31) || G * d->num_heads >= (int64_t(1) << 31))
@@ -264,6 +307,32 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         static_cast<const uint16_t*>(w_uk), q, G, H, dims->qk_nope_dim, dc, dr);
     if (int rc = launch_status()) return rc;
 
+    if (L.kernel == kKernelPair) {
+        CUtensorMap tm_q, tm_kv64, tm_kv32;
+        const uint64_t pool_rows = static_cast<uint64_t>(num_blocks) * dims->block_size;
+        if (int rc = encode_rows(&tm_q, q, pair::kD, static_cast<uint64_t>(G) * H, 64)) return rc;
+        if (int rc = encode_rows(&tm_kv64, pool, pair::kD, pool_rows, 64)) return rc;
+        if (int rc = encode_rows(&tm_kv32, pool, pair::kD, pool_rows, 32)) return rc;
+        pair::Params PP;
+        PP.hdr = hdr;
+        PP.tile_prefix = tile_prefix;
+        PP.part_offsets = part_offsets;
+        PP.context_lens = context_lens;
+        PP.block_table = block_table;
+        PP.o_part = o_part;
+        PP.lse_part = lse_part;
+        PP.num_blocks = num_blocks;
+        PP.batch = batch;
+        PP.max_blocks_per_seq = max_blocks_per_seq;
+        PP.block_size = dims->block_size;
+        PP.q_len = q_len;
+        PP.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
+        if (int rc = ensure_smem(pair::pair_decode_kernel, pair::kSmemBytes)) return rc;
+        if (opts && opts->event_attn_begin) cudaEventRecord(static_cast<cudaEvent_t>(opts->event_attn_begin), st);
+        pair::pair_decode_kernel<<<2 * L.workers, pair::kThreads, pair::kSmemBytes, st>>>(tm_q, tm_kv64, tm_kv32, PP);
+        if (int rc = launch_status()) return rc;
+        if (opts && opts->event_attn_end) cudaEventRecord(static_cast<cudaEvent_t>(opts->event_attn_end), st);
+    } else {
     GenericDecodeParams P;
     P.q = q;
     P.pool = static_cast<const uint16_t*>(pool);
@@ -289,6 +358,7 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     generic_decode_kernel<<<dim3(L.workers, (H + kGenHeads - 1) / kGenHeads), kGenThreads, gsmem, st>>>(P);
     if (int rc = launch_status()) return rc;
     if (opts && opts->event_attn_end) cudaEventRecord(static_cast<cudaEvent_t>(opts->event_attn_end), st);
+    }
 
     const size_t uv_smem = sizeof(float) * kUvGroups * dc;
     if (int rc = ensure_smem(combine_uv_kernel, uv_smem)) return rc;

@@ -19,7 +19,7 @@ from _data import build, oracle_append_pool, to_device, tolerance_ok
 
 pytestmark = pytest.mark.gpu
 
-KERNELS = {"generic": 2}
+KERNELS = {"generic": 2, "pair": 1}
 
 
 def _lib():
@@ -59,12 +59,23 @@ def small_v3(name, batch, q_len, lengths, paged=True, spare=0):
     return w, torch.tensor(lengths, dtype=torch.int32)
 
 
-@pytest.mark.parametrize("kernel", list(KERNELS))
+@pytest.mark.parametrize("kernel", ["auto", "generic"])
 def test_tiny_config(kernel):
     w = I.WORKLOADS["tiny_b1_l128"]
     data = build(w)
-    got = run_decode(w, to_device(data), kernel=KERNELS[kernel])
+    got = run_decode(w, to_device(data), kernel=KERNELS.get(kernel, 0))
     check(got, oracle_out(w, data))
+
+
+def test_pair_kernel_rejects_other_dims():
+    L = _lib()
+    w = I.WORKLOADS["tiny_b1_l128"]
+    assert L.decode_workspace_size(w.dims, w.softmax_scale, 1, 1, 128, kernel=1) == 0
+    data = to_device(build(w))
+    with pytest.raises(L.MLAError) as e:
+        L.decode(w.dims, w.softmax_scale, data["q_nope"], data["q_pe"], data["pool"], data["table"],
+                 data["lengths"], 128, data["w_uk"], data["w_uv"], kernel=1)
+    assert e.value.status == -2
 
 
 @pytest.mark.parametrize("kernel", list(KERNELS))
