@@ -43,7 +43,8 @@ constexpr int kH = 128, kDc = 512, kDr = 64, kD = kDc + kDr;
 constexpr int kTile = 128;       // tokens per pair iteration
 constexpr int kBox = 8192;       // one [64 rows x 64 bf16] 128B-swizzled box = one ring stage
 constexpr int kQBoxes = kD / 64; // 9
-constexpr int kStages = 12;
+constexpr int kStages = 16;
+constexpr int kPrefetchTiles = 3;  // pages are pulled into L2 this many tiles ahead
 constexpr int kThreads = 256;
 constexpr int kTmemCols = 512;
 constexpr int kTmS = 0;          // two S buffers of 64 columns
@@ -69,6 +70,7 @@ struct Params {
     const int32_t* part_offsets;
     const int32_t* context_lens;
     const int32_t* block_table;
+    const uint16_t* pool;  // [num_blocks * block_size, 576]
     float* o_part;  // [n_parts, 128, 512]
     float* lse_part;  // [n_parts, 128]
     int64_t num_blocks;
@@ -118,7 +120,17 @@ __device__ void producer(const Params& P, const CUtensorMap* tm_q, const CUtenso
         }
         __syncwarp();
         const int n_tiles = tiles_of(seg);
+        // Pull this CTA's page of tile jj into L2 so that the ring's TMA loads see L2, not HBM, latency.
+        auto prefetch_tile = [&](int jj) {
+            const int32_t t = seg.tok_begin + jj * kTile + 64 * static_cast<int32_t>(c.rank);
+            if (jj >= n_tiles || t >= seg.tok_end || lane != 0) return;
+            const int64_t row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks,
+                                            P.block_size, b, t);
+            if (row >= 0) ptx::prefetch_l2(P.pool + row * kD, 64 * kD * 2);
+        };
+        for (int jj = 0; jj < kPrefetchTiles; ++jj) prefetch_tile(jj);
         for (int j = 0; j <= n_tiles; ++j) {
+            prefetch_tile(j + kPrefetchTiles);
             if (j < n_tiles) {  // key boxes of tile j: this CTA's 64-token page, all 576 values
                 const int32_t t0 = seg.tok_begin + j * kTile;
                 int32_t th = t0 + 64 * static_cast<int32_t>(c.rank);
@@ -195,6 +207,15 @@ __device__ void producer(const Params& P, const CUtensorMap* tm_q, const CUtenso
         }
         ++seg_i;
     }
+    // Tail: wait until the MMA has released every stage this CTA filled and
+    // the last query block, so that no asynchronous arrival (a multicast
+    // tcgen05.commit) can reach this CTA's shared memory after it exits --
+    // it would land in the barriers of whatever CTA runs here next.
+    for (int i = 0; i < kStages; ++i) {
+        if (!ptx::mbar_wait(c.bar(B_KVEMPTY0 + stage), phase ^ 1, c.abort)) return;
+        ring_next(stage, phase);
+    }
+    if (seg_i > 0) ptx::mbar_wait(c.bar(B_QEMPTY), (seg_i - 1) & 1, c.abort);
 }
 
 // ------------------------------------------------------------------- MMA
