@@ -23,9 +23,12 @@
 // once as values), so shared-memory fills are ~1.9x the HBM bytes, while
 // HBM reads stay ~1x because the second read of a page hits L2.
 //
-// Warp roles per CTA (256 threads): warp 0 streams TMA boxes into a ring of
-// 8 KB stages; warp 1 allocates tensor memory (both CTAs) and, in the
-// leader, issues MMAs; warps 4-7 (thread t = TMEM lane t) run the softmax,
+// Warp roles per CTA (256 threads): one thread of warp 0 streams the queries
+// and the key stages (three 64-column boxes of the CTA's page, 24 KB) into a
+// one-tile key ring; one thread of warp 2 streams the value stages (32
+// tokens x 256 columns, 16 KB) into a one-tile value ring; warp 1 allocates
+// tensor memory (both CTAs) and one of its threads, in the leader, issues the
+// MMAs; warps 4-7 (thread t = TMEM lane t) run the softmax,
 // rescale O when the running max grows by more than 2^8, write P to shared
 // memory and, at the end of a segment, normalise O and write the partial.
 // Every mbarrier wait is bounded (see ptx::mbar_wait): on expiry the kernel
@@ -41,9 +44,14 @@ namespace pair {
 
 constexpr int kH = 128, kDc = 512, kDr = 64, kD = kDc + kDr;
 constexpr int kTile = 128;       // tokens per pair iteration
-constexpr int kBox = 8192;       // one [64 rows x 64 bf16] 128B-swizzled box = one ring stage
+constexpr int kBox = 8192;       // one [64 rows x 64 bf16] 128B-swizzled box
 constexpr int kQBoxes = kD / 64; // 9
-constexpr int kStages = 16;
+constexpr int kKStage = 3 * kBox;    // key stage: three 64-column boxes of a page (24 KB)
+constexpr int kKPerTile = kQBoxes / 3;  // 3 key stages per tile
+constexpr int kKStages = 3;          // key ring: one tile
+constexpr int kVStage = 2 * kBox;    // value stage: 32 tokens x 256 latent columns (4 x 4 KB)
+constexpr int kVPerTile = 4;         // 4 value stages per tile
+constexpr int kVStages = 4;          // value ring: one tile
 constexpr int kPrefetchTiles = 3;  // pages are pulled into L2 this many tiles ahead
 constexpr int kThreads = 256;
 constexpr int kTmemCols = 512;
@@ -51,13 +59,15 @@ constexpr int kTmS = 0;          // two S buffers of 64 columns
 constexpr int kTmO = 128;        // O: 256 columns
 
 constexpr int kOffQ = 0;
-constexpr int kOffRing = kOffQ + kQBoxes * kBox;
-constexpr int kOffP = kOffRing + kStages * kBox;
+constexpr int kOffK = kOffQ + kQBoxes * kBox;
+constexpr int kOffV = kOffK + kKStages * kKStage;
+constexpr int kOffP = kOffV + kVStages * kVStage;
 constexpr int kOffBar = kOffP + 2 * kBox;
 
 enum Bar {
     B_QFULL = 0, B_QEMPTY, B_SFULL0, B_SFULL1, B_SEMPTY0, B_SEMPTY1, B_PFULL, B_PVDONE, B_OEMPTY, B_PATCH, B_XCHG,
-    B_KVFULL0, B_KVEMPTY0 = B_KVFULL0 + kStages, B_COUNT = B_KVEMPTY0 + kStages
+    B_KFULL0, B_KEMPTY0 = B_KFULL0 + kKStages, B_VFULL0 = B_KEMPTY0 + kKStages, B_VEMPTY0 = B_VFULL0 + kVStages,
+    B_COUNT = B_VEMPTY0 + kVStages
 };
 constexpr int kOffRed = kOffBar + 8 * 64;          // exchange buffer [2][128] floats
 constexpr int kOffMisc = kOffRed + 2 * 128 * 4;    // abort flag, TMEM base
@@ -92,138 +102,142 @@ struct Ctx {
 __device__ __forceinline__ int tiles_of(const Segment& s) { return (s.tok_end - s.tok_begin + kTile - 1) / kTile; }
 
 // ------------------------------------------------------------------ producer
-__device__ __forceinline__ bool ring_slot(const Ctx& c, uint32_t& stage, uint32_t& phase, uint32_t& slot_full) {
-    if (!ptx::mbar_wait(c.bar(B_KVEMPTY0 + stage), phase ^ 1, c.abort)) return false;
-    slot_full = c.leader_bar(B_KVFULL0 + stage);
-    return true;
-}
-
+template <int N>
 __device__ __forceinline__ void ring_next(uint32_t& stage, uint32_t& phase) {
-    if (++stage == kStages) { stage = 0; phase ^= 1; }
+    if (++stage == N) { stage = 0; phase ^= 1; }
 }
 
-__device__ void producer(const Params& P, const CUtensorMap* tm_q, const CUtensorMap* tm_kv64,
-                         const CUtensorMap* tm_kv32, const Ctx& c) {
-    const uint32_t lane = ptx::lane_id();
-    uint32_t stage = 0, phase = 0, patch_phase = 0;
+// Queries and key stages; one thread (lane 0 of warp 0).
+__device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUtensorMap* tm_kv64, const Ctx& c) {
+    uint32_t stage = 0, phase = 0;
     int seg_i = 0;
     SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
     Segment seg;
     while (it.next(seg)) {
         const int32_t g = seg.group, b = g / P.q_len;
         if (seg_i > 0 && !ptx::mbar_wait(c.bar(B_QEMPTY), (seg_i - 1) & 1, c.abort)) return;
-        if (lane == 0) {
+        {
             const uint32_t full = c.leader_bar(B_QFULL);
             ptx::mbar_arrive_expect_tx_cluster(full, kQBoxes * kBox);
             for (int k = 0; k < kQBoxes; ++k)
                 ptx::tma_load_2d_pair(c.sbase + kOffQ + k * kBox, tm_q, 64 * k, g * kH + 64 * c.rank, full);
         }
-        __syncwarp();
         const int n_tiles = tiles_of(seg);
-        // Pull this CTA's page of tile jj into L2 so that the ring's TMA loads see L2, not HBM, latency.
+        // Pull this CTA's page of tile jj into L2 so that the TMA loads see L2, not HBM, latency.
         auto prefetch_tile = [&](int jj) {
             const int32_t t = seg.tok_begin + jj * kTile + 64 * static_cast<int32_t>(c.rank);
-            if (jj >= n_tiles || t >= seg.tok_end || lane != 0) return;
+            if (jj >= n_tiles || t >= seg.tok_end) return;
             const int64_t row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks,
                                             P.block_size, b, t);
             if (row >= 0) ptx::prefetch_l2(P.pool + row * kD, 64 * kD * 2);
         };
         for (int jj = 0; jj < kPrefetchTiles; ++jj) prefetch_tile(jj);
-        for (int j = 0; j <= n_tiles; ++j) {
+        for (int j = 0; j < n_tiles; ++j) {
             prefetch_tile(j + kPrefetchTiles);
-            if (j < n_tiles) {  // key boxes of tile j: this CTA's 64-token page, all 576 values
-                const int32_t t0 = seg.tok_begin + j * kTile;
-                int32_t th = t0 + 64 * static_cast<int32_t>(c.rank);
-                if (th >= seg.tok_end) th = t0;  // no visible token in this half: any valid page (masked)
-                int64_t row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks,
-                                          P.block_size, b, th);
-                if (row < 0) {
-                    if (lane == 0) record_status(MLA_ERR_DEVICE_FAULT);
-                    row = 0;
-                }
-                for (int k = 0; k < kQBoxes; ++k) {
-                    uint32_t full;
-                    if (!ring_slot(c, stage, phase, full)) return;
-                    if (lane == 0) {
-                        ptx::mbar_arrive_expect_tx_cluster(full, kBox);
-                        ptx::tma_load_2d_pair(c.sbase + kOffRing + stage * kBox, tm_kv64, 64 * k,
-                                              static_cast<int32_t>(row), full);
-                    }
-                    __syncwarp();
-                    ring_next(stage, phase);
-                }
+            // this CTA's 64-token page of tile j, all 576 values
+            const int32_t t0 = seg.tok_begin + j * kTile;
+            int32_t th = t0 + 64 * static_cast<int32_t>(c.rank);
+            if (th >= seg.tok_end) th = t0;  // no visible token in this half: any valid page (masked)
+            int64_t row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks, P.block_size,
+                                      b, th);
+            if (row < 0) {
+                record_status(MLA_ERR_DEVICE_FAULT);
+                row = 0;
             }
-            if (j >= 1) {  // value boxes of tile j-1: 32 tokens x this CTA's 128 latent columns per stage
-                const int32_t tv = seg.tok_begin + (j - 1) * kTile;
-                for (int q = 0; q < 4; ++q) {
-                    const int32_t tq = tv + 32 * q;
-                    const int nv = max(0, min(32, seg.tok_end - tq));
-                    int64_t row = -1;
-                    if (nv > 0) {
-                        row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks, P.block_size,
-                                          b, tq);
-                        if (row < 0 && lane == 0) record_status(MLA_ERR_DEVICE_FAULT);
-                    }
-                    for (int n = 0; n < 2; ++n) {
-                        uint32_t full;
-                        if (!ring_slot(c, stage, phase, full)) return;
-                        const uint32_t dst = c.sbase + kOffRing + stage * kBox;
-                        const int32_t x0 = 256 * static_cast<int32_t>(c.rank) + 128 * n;
-                        if (row >= 0 && nv == 32) {
-                            if (lane == 0) {
-                                ptx::mbar_arrive_expect_tx_cluster(full, kBox);
-                                ptx::tma_load_2d_pair(dst, tm_kv32, x0, static_cast<int32_t>(row), full);
-                                ptx::tma_load_2d_pair(dst + kBox / 2, tm_kv32, x0 + 64, static_cast<int32_t>(row), full);
-                            }
-                        } else {
-                            // Tail of the visible range: rows past it may hold anything (even NaN),
-                            // and 0 * NaN would poison O, so they are zeroed before the MMA reads them.
-                            int keep = 0;
-                            if (row >= 0) {
-                                if (lane == 0) {
-                                    ptx::mbar_arrive_expect_tx_local(c.bar(B_PATCH), kBox);
-                                    ptx::tma_load_2d(dst, tm_kv32, x0, static_cast<int32_t>(row), c.bar(B_PATCH));
-                                    ptx::tma_load_2d(dst + kBox / 2, tm_kv32, x0 + 64, static_cast<int32_t>(row),
-                                                     c.bar(B_PATCH));
-                                }
-                                if (!ptx::mbar_wait(c.bar(B_PATCH), patch_phase, c.abort)) return;
-                                patch_phase ^= 1;
-                                keep = nv;
-                            }
-                            uint4* p = reinterpret_cast<uint4*>(c.smem + kOffRing + stage * kBox);
-                            for (int i = lane; i < kBox / 16; i += 32) {
-                                const int r = (i & 255) >> 3;  // token row within its 4 KB box
-                                if (r >= keep) p[i] = make_uint4(0u, 0u, 0u, 0u);
-                            }
-                            ptx::fence_proxy_async_smem();
-                            __syncwarp();
-                            if (lane == 0) ptx::mbar_arrive_cluster(full);
-                        }
-                        __syncwarp();
-                        ring_next(stage, phase);
-                    }
-                }
+            for (int ks = 0; ks < kKPerTile; ++ks) {
+                if (!ptx::mbar_wait(c.bar(B_KEMPTY0 + stage), phase ^ 1, c.abort)) return;
+                const uint32_t full = c.leader_bar(B_KFULL0 + stage);
+                ptx::mbar_arrive_expect_tx_cluster(full, kKStage);
+                for (int bx = 0; bx < 3; ++bx)
+                    ptx::tma_load_2d_pair(c.sbase + kOffK + stage * kKStage + bx * kBox, tm_kv64, 64 * (3 * ks + bx),
+                                          static_cast<int32_t>(row), full);
+                ring_next<kKStages>(stage, phase);
             }
         }
         ++seg_i;
     }
-    // Tail: wait until the MMA has released every stage this CTA filled and
-    // the last query block, so that no asynchronous arrival (a multicast
-    // tcgen05.commit) can reach this CTA's shared memory after it exits --
-    // it would land in the barriers of whatever CTA runs here next.
-    for (int i = 0; i < kStages; ++i) {
-        if (!ptx::mbar_wait(c.bar(B_KVEMPTY0 + stage), phase ^ 1, c.abort)) return;
-        ring_next(stage, phase);
+    // Tail: wait until the MMA has released every key stage and the last query
+    // block, so that no asynchronous arrival (a multicast tcgen05.commit) can
+    // reach this CTA's shared memory after it exits -- it would land in the
+    // barriers of whatever CTA runs here next.
+    for (int i = 0; i < kKStages; ++i) {
+        if (!ptx::mbar_wait(c.bar(B_KEMPTY0 + stage), phase ^ 1, c.abort)) return;
+        ring_next<kKStages>(stage, phase);
     }
     if (seg_i > 0) ptx::mbar_wait(c.bar(B_QEMPTY), (seg_i - 1) & 1, c.abort);
 }
 
+// Value stages; one thread (lane 0 of warp 2). Stage q of a tile holds tokens
+// 32q..32q+31 and this CTA's latent columns 256r..256r+255 as four 4 KB boxes:
+// box (n, h) = columns 256r + 128n + 64h at offset (2n + h) * 4 KB.
+__device__ void value_producer(const Params& P, const CUtensorMap* tm_kv32, const Ctx& c) {
+    uint32_t stage = 0, phase = 0, patch_phase = 0;
+    SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    Segment seg;
+    while (it.next(seg)) {
+        const int32_t b = seg.group / P.q_len;
+        const int n_tiles = tiles_of(seg);
+        for (int j = 0; j < n_tiles; ++j) {
+            const int32_t tv = seg.tok_begin + j * kTile;
+            for (int q = 0; q < kVPerTile; ++q) {
+                const int32_t tq = tv + 32 * q;
+                const int nv = max(0, min(32, seg.tok_end - tq));
+                int64_t row = -1;
+                if (nv > 0) {
+                    row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks, P.block_size, b, tq);
+                    if (row < 0) record_status(MLA_ERR_DEVICE_FAULT);
+                }
+                if (!ptx::mbar_wait(c.bar(B_VEMPTY0 + stage), phase ^ 1, c.abort)) return;
+                const uint32_t full = c.leader_bar(B_VFULL0 + stage);
+                const uint32_t dst = c.sbase + kOffV + stage * kVStage;
+                const int32_t x0 = 256 * static_cast<int32_t>(c.rank);
+                if (row >= 0 && nv == 32) {
+                    ptx::mbar_arrive_expect_tx_cluster(full, kVStage);
+                    for (int bx = 0; bx < 4; ++bx)
+                        ptx::tma_load_2d_pair(dst + bx * (kBox / 2), tm_kv32, x0 + 64 * bx, static_cast<int32_t>(row),
+                                              full);
+                } else {
+                    // Tail of the visible range: rows past it may hold anything (even NaN),
+                    // and 0 * NaN would poison O, so they are zeroed before the MMA reads them.
+                    int keep = 0;
+                    if (row >= 0) {
+                        ptx::mbar_arrive_expect_tx_local(c.bar(B_PATCH), kVStage);
+                        for (int bx = 0; bx < 4; ++bx)
+                            ptx::tma_load_2d(dst + bx * (kBox / 2), tm_kv32, x0 + 64 * bx, static_cast<int32_t>(row),
+                                             c.bar(B_PATCH));
+                        if (!ptx::mbar_wait(c.bar(B_PATCH), patch_phase, c.abort)) return;
+                        patch_phase ^= 1;
+                        keep = nv;
+                    }
+                    uint4* p = reinterpret_cast<uint4*>(c.smem + kOffV + stage * kVStage);
+                    for (int i = 0; i < kVStage / 16; ++i) {
+                        const int r = (i & 255) >> 3;  // token row within its 4 KB box
+                        if (r >= keep) p[i] = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    ptx::fence_proxy_async_smem();
+                    ptx::mbar_arrive_cluster(full);
+                }
+                ring_next<kVStages>(stage, phase);
+            }
+        }
+    }
+    for (int i = 0; i < kVStages; ++i) {  // tail, as for the key ring
+        if (!ptx::mbar_wait(c.bar(B_VEMPTY0 + stage), phase ^ 1, c.abort)) return;
+        ring_next<kVStages>(stage, phase);
+    }
+}
+
 // ------------------------------------------------------------------- MMA
 __device__ void mma_issuer(const Params& P, const Ctx& c) {
+    // runs in one thread (lane 0 of warp 1 of the leader CTA)
     constexpr uint32_t kIdS = ptx::idesc_bf16(128, 128, false, false);
     constexpr uint32_t kIdPV = ptx::idesc_bf16(128, 256, false, true);
-    const uint32_t lane = ptx::lane_id();
-    uint32_t stage = 0, phase = 0, tile_cnt = 0, pv_cnt = 0;
+    // Base descriptors; operand offsets are added in 16-byte units to the start-address field.
+    const uint64_t dq = ptx::smem_desc_sw128(c.sbase + kOffQ, 16, 1024);
+    const uint64_t dk = ptx::smem_desc_sw128(c.sbase + kOffK, 16, 1024);
+    const uint64_t dp = ptx::smem_desc_sw128(c.sbase + kOffP, 16, 1024);
+    const uint64_t dv = ptx::smem_desc_sw128(c.sbase + kOffV, kBox / 2, 1024);
+    uint32_t kst = 0, kph = 0, vst = 0, vph = 0, tile_cnt = 0, pv_cnt = 0;
     int seg_i = 0;
     SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
     Segment seg;
@@ -234,57 +248,48 @@ __device__ void mma_issuer(const Params& P, const Ctx& c) {
         for (int j = 0; j <= n_tiles; ++j) {
             if (j < n_tiles) {  // S = Q K^T for tile j into S buffer sb
                 const uint32_t sb = tile_cnt & 1;
+                const uint32_t d_s = c.tmem + kTmS + 64 * sb;
                 if (!ptx::mbar_wait(c.bar(B_SEMPTY0 + sb), ((tile_cnt >> 1) & 1) ^ 1, c.abort)) return;
-                ptx::tc_fence_after();
-                for (int k = 0; k < kQBoxes; ++k) {
-                    if (!ptx::mbar_wait(c.bar(B_KVFULL0 + stage), phase, c.abort)) return;
+                for (int ks = 0; ks < kKPerTile; ++ks) {
+                    if (!ptx::mbar_wait(c.bar(B_KFULL0 + kst), kph, c.abort)) return;
                     ptx::tc_fence_after();
-                    if (lane == 0) {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t a = ptx::smem_desc_sw128(c.sbase + kOffQ + k * kBox + 32 * kk, 16, 1024);
-                            const uint64_t bd =
-                                ptx::smem_desc_sw128(c.sbase + kOffRing + stage * kBox + 32 * kk, 16, 1024);
-                            ptx::mma_bf16_pair(c.tmem + kTmS + 64 * sb, a, bd, kIdS, (k | kk) != 0);
-                        }
-                        ptx::mma_commit_pair(c.bar(B_KVEMPTY0 + stage), 0x3);
+                    for (int bx = 0; bx < 3; ++bx) {
+                        const int k = 3 * ks + bx;
+                        const uint64_t a0 = dq + static_cast<uint64_t>((k * kBox) >> 4);
+                        const uint64_t b0 = dk + static_cast<uint64_t>((kst * kKStage + bx * kBox) >> 4);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            ptx::mma_bf16_pair(d_s, a0 + 2 * kk, b0 + 2 * kk, kIdS, (k | kk) != 0);
                     }
-                    __syncwarp();
-                    ring_next(stage, phase);
+                    ptx::mma_commit_pair(c.bar(B_KEMPTY0 + kst), 0x3);
+                    ring_next<kKStages>(kst, kph);
                 }
-                if (lane == 0) {
-                    ptx::mma_commit_pair(c.bar(B_SFULL0 + sb), 0x3);
-                    if (j == n_tiles - 1) ptx::mma_commit_pair(c.bar(B_QEMPTY), 0x3);
-                }
-                __syncwarp();
+                ptx::mma_commit_pair(c.bar(B_SFULL0 + sb), 0x3);
+                if (j == n_tiles - 1) ptx::mma_commit_pair(c.bar(B_QEMPTY), 0x3);
                 ++tile_cnt;
             }
             if (j >= 1) {  // O += P V for tile j-1
                 const bool first = (j == 1);
                 if (!ptx::mbar_wait(c.bar(B_PFULL), pv_cnt & 1, c.abort)) return;
                 if (first && !ptx::mbar_wait(c.bar(B_OEMPTY), (seg_i & 1) ^ 1, c.abort)) return;
-                ptx::tc_fence_after();
-                for (int q = 0; q < 4; ++q) {
-                    for (int n = 0; n < 2; ++n) {
-                        if (!ptx::mbar_wait(c.bar(B_KVFULL0 + stage), phase, c.abort)) return;
-                        ptx::tc_fence_after();
-                        if (lane == 0) {
+                for (int q = 0; q < kVPerTile; ++q) {
+                    if (!ptx::mbar_wait(c.bar(B_VFULL0 + vst), vph, c.abort)) return;
+                    ptx::tc_fence_after();
+                    // A: P tokens 32q + 16kk .. +15 (box q/2, byte 64 (q&1) + 32 kk of each 128-byte row)
+                    const uint64_t a0 = dp + static_cast<uint64_t>(((q >> 1) * kBox + 64 * (q & 1)) >> 4);
+                    const uint64_t b0 = dv + static_cast<uint64_t>((vst * kVStage) >> 4);
 #pragma unroll
-                            for (int kk = 0; kk < 2; ++kk) {
-                                const uint32_t pa = c.sbase + kOffP + (q >> 1) * kBox + 64 * (q & 1) + 32 * kk;
-                                const uint64_t a = ptx::smem_desc_sw128(pa, 16, 1024);
-                                const uint64_t bd =
-                                    ptx::smem_desc_sw128(c.sbase + kOffRing + stage * kBox + 2048 * kk, kBox / 2, 1024);
-                                ptx::mma_bf16_pair(c.tmem + kTmO + 128 * n, a, bd, kIdPV, !(first && q == 0 && kk == 0));
-                            }
-                            ptx::mma_commit_pair(c.bar(B_KVEMPTY0 + stage), 0x3);
-                        }
-                        __syncwarp();
-                        ring_next(stage, phase);
-                    }
+                    for (int n = 0; n < 2; ++n)
+#pragma unroll
+                        for (int kk = 0; kk < 2; ++kk)
+                            ptx::mma_bf16_pair(c.tmem + kTmO + 128 * n, a0 + 2 * kk,
+                                               b0 + static_cast<uint64_t>((n * kBox + 2048 * kk) >> 4), kIdPV,
+                                               !(first && q == 0 && kk == 0));
+                    ptx::mma_commit_pair(c.bar(B_VEMPTY0 + vst), 0x3);
+                    ring_next<kVStages>(vst, vph);
                 }
-                if (lane == 0) ptx::mma_commit_pair(c.bar(B_PVDONE), 0x3);
-                __syncwarp();
+                ptx::mma_commit_pair(c.bar(B_PVDONE), 0x3);
                 ++pv_cnt;
             }
         }
@@ -315,7 +320,8 @@ __device__ void softmax(const Params& P, const Ctx& c) {
     const int half = t >> 6, hrow = t & 63;
     const int head = 64 * static_cast<int>(c.rank) + hrow;
     const uint32_t tl = c.tmem + (static_cast<uint32_t>(t & ~31) << 16);  // this warp's lane quadrant
-    const uint32_t sempty[2] = {c.leader_bar(B_SEMPTY0), c.leader_bar(B_SEMPTY1)};
+    const uint32_t sempty0 = c.leader_bar(B_SEMPTY0), sempty1 = c.leader_bar(B_SEMPTY1);
+    const float scale_log2 = P.scale_log2;
     const uint32_t pfull = c.leader_bar(B_PFULL), oempty = c.leader_bar(B_OEMPTY);
     uint8_t* prow = c.smem + kOffP + half * kBox + hrow * 128;
     Exchanger xc{reinterpret_cast<float*>(c.smem + kOffRed), c.bar(B_XCHG)};
@@ -339,31 +345,36 @@ __device__ void softmax(const Params& P, const Ctx& c) {
             }
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive_cluster(sempty[sb]);
+            if (lane == 0) ptx::mbar_arrive_cluster(sb ? sempty1 : sempty0);
             ++tile_cnt;
 
             const int32_t tok0 = seg.tok_begin + j * kTile + 64 * half;
             const int nvalid = max(0, min(64, seg.tok_end - tok0));
-            float mloc = -INFINITY;
+            if (nvalid < 64) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                s[i] = i < nvalid ? s[i] * P.scale_log2 : -INFINITY;
-                mloc = fmaxf(mloc, s[i]);
+                for (int i = 0; i < 64; ++i)
+                    if (i >= nvalid) s[i] = -INFINITY;
             }
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], s[i]);
+            // the scale is positive, so the max of the raw scores gives the max of the scaled ones
+            const float mloc = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale_log2;
             float mpart;
             if (!xc.swap(mloc, mpart, t, c.abort)) return;
             const float m_tile = fmaxf(mloc, mpart);
             const float m_new = fmaxf(m_run, m_tile);
             const bool rescale = m_new > m_run + 8.f;  // keep a stale max unless it grows by > 2^8
             const float m_use = rescale ? m_new : m_run;
-            const float alpha = rescale ? exp2f(m_run - m_new) : 1.f;
-            float psum = 0.f;
+            const float alpha = rescale ? ptx::ex2(m_run - m_new) : 1.f;
+            const float neg_m = -m_use;
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
-                s[i] = exp2f(s[i] - m_use);  // exp2(-inf) = 0 for masked tokens
-                psum += s[i];
+                s[i] = ptx::ex2(fmaf(s[i], scale_log2, neg_m));  // 2^-inf = 0 for masked tokens
+                ps[i & 3] += s[i];
             }
-            l_run = l_run * alpha + psum;
+            l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
             if (j > 0) {  // PV of the previous tile must be done before P and O are touched
                 if (!ptx::mbar_wait(c.bar(B_PVDONE), pv_wait & 1, c.abort)) return;
                 ++pv_wait;
@@ -385,10 +396,10 @@ __device__ void softmax(const Params& P, const Ctx& c) {
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8) {
                 uint4 u;
-                u.x = pack_bf16x2(s[8 * c8 + 0], s[8 * c8 + 1]);
-                u.y = pack_bf16x2(s[8 * c8 + 2], s[8 * c8 + 3]);
-                u.z = pack_bf16x2(s[8 * c8 + 4], s[8 * c8 + 5]);
-                u.w = pack_bf16x2(s[8 * c8 + 6], s[8 * c8 + 7]);
+                u.x = ptx::bf16x2(s[8 * c8 + 0], s[8 * c8 + 1]);
+                u.y = ptx::bf16x2(s[8 * c8 + 2], s[8 * c8 + 3]);
+                u.z = ptx::bf16x2(s[8 * c8 + 4], s[8 * c8 + 5]);
+                u.w = ptx::bf16x2(s[8 * c8 + 6], s[8 * c8 + 7]);
                 *reinterpret_cast<uint4*>(prow + ((c8 ^ (hrow & 7)) << 4)) = u;
             }
             ptx::fence_proxy_async_smem();
@@ -455,9 +466,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ptx::mbar_init(c.bar(B_OEMPTY), 8);
         ptx::mbar_init(c.bar(B_PATCH), 1);
         ptx::mbar_init(c.bar(B_XCHG), 4);
-        for (int s = 0; s < kStages; ++s) {
-            ptx::mbar_init(c.bar(B_KVFULL0 + s), 2);
-            ptx::mbar_init(c.bar(B_KVEMPTY0 + s), 1);
+        for (int s = 0; s < kKStages; ++s) {
+            ptx::mbar_init(c.bar(B_KFULL0 + s), 2);
+            ptx::mbar_init(c.bar(B_KEMPTY0 + s), 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
+            ptx::mbar_init(c.bar(B_VFULL0 + s), 2);
+            ptx::mbar_init(c.bar(B_VEMPTY0 + s), 1);
         }
         ptx::fence_mbar_init();
     }
@@ -477,9 +492,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     c.tmem = *tmem_slot;
 
     if (warp == 0) {
-        producer(P, &tm_q, &tm_kv64, &tm_kv32, c);
+        if (ptx::lane_id() == 0) key_producer(P, &tm_q, &tm_kv64, c);
+    } else if (warp == 2) {
+        if (ptx::lane_id() == 0) value_producer(P, &tm_kv32, c);
     } else if (warp == 1) {
-        if (c.rank == 0) mma_issuer(P, c);
+        if (c.rank == 0 && ptx::lane_id() == 0) mma_issuer(P, c);
     } else if (warp >= 4) {
         softmax(P, c);
     }
