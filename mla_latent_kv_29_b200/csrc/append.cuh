@@ -120,11 +120,15 @@ __global__ void __launch_bounds__(256) append_epilogue_kernel(AppendEpiloguePara
     // rotate-half RoPE: pair (i, i + dr/2) rotated by pos * base^(-2i/dr)
     const int half = P.dr / 2;
     for (int i = threadIdx.x; i < half; i += blockDim.x) {
-        const double inv_freq = pow(P.rope_base, -2.0 * i / static_cast<double>(P.dr));
-        double sn, cs;
-        sincos(static_cast<double>(pos) * inv_freq, &sn, &cs);
+        // angle = pos * base^(-2i/dr), formed in double; reduced to [-pi, pi] with a
+        // two-term 2*pi so the float sine/cosine stay on their short-argument path
+        const double inv_freq = exp2(-2.0 * i / static_cast<double>(P.dr) * log2(P.rope_base));
+        const double angle = static_cast<double>(pos) * inv_freq;
+        const double k = rint(angle * 0.15915494309189535);  // 1 / (2 pi)
+        const double reduced = fma(-k, 2.4492935982947064e-16, fma(-k, 6.283185307179586, angle));
+        float s, c;
+        sincosf(static_cast<float>(reduced), &s, &c);
         const float x1 = kv[P.dc + i], x2 = kv[P.dc + i + half];
-        const float c = static_cast<float>(cs), s = static_cast<float>(sn);
         dst[P.dc + i] = f32_to_bf16(x1 * c - x2 * s);
         dst[P.dc + i + half] = f32_to_bf16(x2 * c + x1 * s);
     }

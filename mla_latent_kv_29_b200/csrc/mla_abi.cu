@@ -14,6 +14,7 @@
 #include "decode_generic.cuh"
 #include "append.cuh"
 #include "decode_pair.cuh"
+#include "gemm_small.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -168,15 +169,35 @@ int ensure_smem(K kernel, size_t bytes) {
     return MLA_OK;
 }
 
-// ---- append workspace ------------------------------------------------
-int append_splits(int32_t n_tokens, int32_t hidden, int32_t N) {
-    const int64_t tiles = static_cast<int64_t>((N + kApTileN - 1) / kApTileN) * ((n_tokens + kApTileT - 1) / kApTileT);
+// ---- tensor-core GEMM eligibility ------------------------------------
+// absorb: d_n multiple of 16 (<= 256), d_c multiple of 128; up-projection:
+// d_v multiple of 64 and the [64 + d_v, d_c + 8] bf16 tiles within 227 KB.
+bool tc_gemm_dims_ok(const mla_dims_t* d) {
+    return d->qk_nope_dim % 16 == 0 && d->qk_nope_dim <= 256 && d->kv_lora_rank % 128 == 0 &&
+           d->v_head_dim % 64 == 0 && uv_tc_smem(d->kv_lora_rank, d->v_head_dim) <= 227 * 1024 && d->kv_lora_rank <= 512;
+}
+
+// ---- append split-K plan ----------------------------------------------
+struct AppendPlan {
+    bool tc;
+    int splits, k_per_split;
+};
+
+AppendPlan append_plan(int32_t n_tokens, int32_t hidden, int32_t N) {
+    AppendPlan a;
+    a.tc = (N % kApTc == 0) && (hidden % kApTc == 0);
+    const int tile_n = a.tc ? kApTc : kApTileN, tile_t = a.tc ? kApTc : kApTileT, tile_k = a.tc ? kApTc : kApTileK;
+    const int64_t tiles = static_cast<int64_t>((N + tile_n - 1) / tile_n) * ((n_tokens + tile_t - 1) / tile_t);
     const int64_t target = 2 * num_sms();
+    const int64_t chunks = (hidden + tile_k - 1) / tile_k;
     int64_t s = tiles >= target ? 1 : (target + tiles - 1) / tiles;
-    const int64_t max_s = (hidden + kApTileK - 1) / kApTileK;
-    if (s > max_s) s = max_s;
+    if (s > chunks) s = chunks;
     if (s > 64) s = 64;
-    return static_cast<int>(s < 1 ? 1 : s);
+    if (s < 1) s = 1;
+    const int64_t per = (chunks + s - 1) / s;  // K chunks per split
+    a.k_per_split = static_cast<int>(per * tile_k);
+    a.splits = static_cast<int>((chunks + per - 1) / per);
+    return a;
 }
 
 }  // namespace
@@ -217,8 +238,8 @@ int mla_get_device_error(int* device_status, void* stream) {
 size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t n_tokens, int32_t hidden) {
     if (check_dims(dims) || n_tokens < 1 || hidden < 1) return 0;
     const int N = dims->kv_lora_rank + dims->rope_dim;
-    const int s = append_splits(n_tokens, hidden, N);
-    return align_up(sizeof(float) * static_cast<size_t>(s) * n_tokens * N);
+    const AppendPlan a = append_plan(n_tokens, hidden, N);
+    return align_up(sizeof(float) * static_cast<size_t>(a.splits) * n_tokens * N);
 }
 
 int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t hidden, const void* w_kva,
@@ -235,14 +256,21 @@ int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32
     if (workspace_bytes < mla_append_workspace_size(dims, n_tokens, hidden)) return MLA_ERR_WORKSPACE_TOO_SMALL;
     if (int rc = device_ok()) return rc;
     const int N = dims->kv_lora_rank + dims->rope_dim;
-    const int splits = append_splits(n_tokens, hidden, N);
-    int k_per_split = (hidden + splits - 1) / splits;
-    k_per_split = (k_per_split + kApTileK - 1) / kApTileK * kApTileK;
+    const AppendPlan ap = append_plan(n_tokens, hidden, N);
+    const int splits = ap.splits;
     float* part = static_cast<float*>(workspace);
     cudaStream_t st = as_stream(stream);
-    dim3 g1((N + kApTileN - 1) / kApTileN, (n_tokens + kApTileT - 1) / kApTileT, splits);
-    append_gemm_kernel<<<g1, 256, 0, st>>>(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w_kva),
-                                           part, n_tokens, hidden, N, k_per_split);
+    if (ap.tc) {
+        if (!aligned(x, 16) || !aligned(w_kva, 16)) return MLA_ERR_INVALID_ARG;
+        dim3 g1(N / kApTc, (n_tokens + kApTc - 1) / kApTc, splits);
+        append_gemm_tc_kernel<<<g1, 128, 0, st>>>(static_cast<const uint16_t*>(x),
+                                                  static_cast<const uint16_t*>(w_kva), part, n_tokens, hidden, N,
+                                                  ap.k_per_split);
+    } else {
+        dim3 g1((N + kApTileN - 1) / kApTileN, (n_tokens + kApTileT - 1) / kApTileT, splits);
+        append_gemm_kernel<<<g1, 256, 0, st>>>(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w_kva),
+                                               part, n_tokens, hidden, N, ap.k_per_split);
+    }
     if (int rc = launch_status()) return rc;
     AppendEpilogueParams P;
     P.part = part;
@@ -300,11 +328,20 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     plan_kernel<<<1, 1024, 0, st>>>(context_lens, batch, q_len, L.tile, L.workers, hdr, tile_prefix, part_offsets);
     if (int rc = launch_status()) return rc;
 
-    const size_t absorb_smem = sizeof(float) * kAbsorbGroups * dims->qk_nope_dim;
-    if (int rc = ensure_smem(absorb_q_kernel, absorb_smem)) return rc;
-    absorb_q_kernel<<<dim3(H, (G + kAbsorbGroups - 1) / kAbsorbGroups), kAbsorbThreads, absorb_smem, st>>>(
-        static_cast<const uint16_t*>(q_nope), static_cast<const uint16_t*>(q_pe),
-        static_cast<const uint16_t*>(w_uk), q, G, H, dims->qk_nope_dim, dc, dr);
+    const bool tc = tc_gemm_dims_ok(dims) && aligned(q_nope, 16) && aligned(w_uk, 16) && aligned(w_uv, 16);
+    if (tc) {
+        const size_t smem = absorb_tc_smem(dims->qk_nope_dim);
+        if (int rc = ensure_smem(absorb_tc_kernel, smem)) return rc;
+        absorb_tc_kernel<<<dim3(H, dc / 128, (G + kTcRows - 1) / kTcRows), kTcThreads, smem, st>>>(
+            static_cast<const uint16_t*>(q_nope), static_cast<const uint16_t*>(q_pe),
+            static_cast<const uint16_t*>(w_uk), q, G, H, dims->qk_nope_dim, dc, dr);
+    } else {
+        const size_t absorb_smem = sizeof(float) * kAbsorbGroups * dims->qk_nope_dim;
+        if (int rc = ensure_smem(absorb_q_kernel, absorb_smem)) return rc;
+        absorb_q_kernel<<<dim3(H, (G + kAbsorbGroups - 1) / kAbsorbGroups), kAbsorbThreads, absorb_smem, st>>>(
+            static_cast<const uint16_t*>(q_nope), static_cast<const uint16_t*>(q_pe),
+            static_cast<const uint16_t*>(w_uk), q, G, H, dims->qk_nope_dim, dc, dr);
+    }
     if (int rc = launch_status()) return rc;
 
     if (L.kernel == kKernelPair) {
@@ -361,11 +398,22 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     if (opts && opts->event_attn_end) cudaEventRecord(static_cast<cudaEvent_t>(opts->event_attn_end), st);
     }
 
-    const size_t uv_smem = sizeof(float) * kUvGroups * dc;
-    if (int rc = ensure_smem(combine_uv_kernel, uv_smem)) return rc;
-    combine_uv_kernel<<<dim3(H, (G + kUvGroups - 1) / kUvGroups), kUvThreads, uv_smem, st>>>(
-        o_part, lse_part, part_offsets, static_cast<const uint16_t*>(w_uv), G, H, dc, dims->v_head_dim,
-        static_cast<uint16_t*>(out));
+    if (tc) {
+        // the absorbed queries are dead once the attention kernel is done: o_lat (bf16) reuses them
+        uint16_t* o_lat = q;
+        merge_bf16_kernel<<<dim3(G, (H + 7) / 8), 256, 0, st>>>(o_part, lse_part, part_offsets, G, H, dc, o_lat);
+        if (int rc = launch_status()) return rc;
+        const size_t smem = uv_tc_smem(dc, dims->v_head_dim);
+        if (int rc = ensure_smem(uv_tc_kernel, smem)) return rc;
+        uv_tc_kernel<<<dim3(H, (G + kTcRows - 1) / kTcRows), kTcThreads, smem, st>>>(
+            o_lat, static_cast<const uint16_t*>(w_uv), G, H, dc, dims->v_head_dim, static_cast<uint16_t*>(out));
+    } else {
+        const size_t uv_smem = sizeof(float) * kUvGroups * dc;
+        if (int rc = ensure_smem(combine_uv_kernel, uv_smem)) return rc;
+        combine_uv_kernel<<<dim3(H, (G + kUvGroups - 1) / kUvGroups), kUvThreads, uv_smem, st>>>(
+            o_part, lse_part, part_offsets, static_cast<const uint16_t*>(w_uv), G, H, dc, dims->v_head_dim,
+            static_cast<uint16_t*>(out));
+    }
     return launch_status();
 }
 

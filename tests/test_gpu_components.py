@@ -126,3 +126,24 @@ def test_append_bad_slot_is_skipped_and_reported():
     assert L.device_error() == -5
     changed = (dd["pool"] != before).any(-1).view(-1).sum().item()
     assert changed == 3  # the three valid tokens were written
+
+
+def test_append_tiny_dims_uses_the_cuda_core_path():
+    """d_c + d_r = 80 is not a multiple of the tensor-core tile: exercises the CUDA-core GEMM."""
+    L = _lib()
+    w = I.scaled(I.WORKLOADS["tiny_b1_l128"], batch=2, q_len=3, length=128, name="append_tiny", seed=91,
+                 append_hidden=96, append_w_std=96 ** -0.5)
+    data = build(w, fill=float("nan"))
+    dd = to_device(data)
+    ap = dd["append"]
+    L.append_kv(w.dims, ap["x"], ap["w_kva"], ap["seq_ids"], ap["positions"], dd["table"], dd["pool"])
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    d = w.dims
+    tab = data["table"].numpy()
+    slots = [O.resolve_slot(tab, int(b), int(p), d.block_size)
+             for b, p in zip(data["append"]["seq_ids"].tolist(), data["append"]["positions"].tolist())]
+    got = dd["pool"].view(-1, d.row_width)[torch.tensor(slots, device="cuda")].float().cpu().numpy()
+    ref = O.append_rows(data["append"]["x"], data["append"]["w_kva"], data["append"]["positions"].numpy(),
+                        d.kv_lora_rank)
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 2e-3)
