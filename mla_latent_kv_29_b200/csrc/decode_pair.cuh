@@ -52,7 +52,6 @@ constexpr int kKStages = 3;          // key ring: one tile
 constexpr int kVStage = 2 * kBox;    // value stage: 32 tokens x 256 latent columns (4 x 4 KB)
 constexpr int kVPerTile = 4;         // 4 value stages per tile
 constexpr int kVStages = 4;          // value ring: one tile
-constexpr int kPrefetchTiles = 3;  // pages are pulled into L2 this many tiles ahead
 constexpr int kThreads = 256;
 constexpr int kTmemCols = 512;
 constexpr int kTmS = 0;          // two S buffers of 64 columns
@@ -80,7 +79,6 @@ struct Params {
     const int32_t* part_offsets;
     const int32_t* context_lens;
     const int32_t* block_table;
-    const uint16_t* pool;  // [num_blocks * block_size, 576]
     float* o_part;  // [n_parts, 128, 512]
     float* lse_part;  // [n_parts, 128]
     int64_t num_blocks;
@@ -123,17 +121,7 @@ __device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUt
                 ptx::tma_load_2d_pair(c.sbase + kOffQ + k * kBox, tm_q, 64 * k, g * kH + 64 * c.rank, full);
         }
         const int n_tiles = tiles_of(seg);
-        // Pull this CTA's page of tile jj into L2 so that the TMA loads see L2, not HBM, latency.
-        auto prefetch_tile = [&](int jj) {
-            const int32_t t = seg.tok_begin + jj * kTile + 64 * static_cast<int32_t>(c.rank);
-            if (jj >= n_tiles || t >= seg.tok_end) return;
-            const int64_t row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks,
-                                            P.block_size, b, t);
-            if (row >= 0) ptx::prefetch_l2(P.pool + row * kD, 64 * kD * 2);
-        };
-        for (int jj = 0; jj < kPrefetchTiles; ++jj) prefetch_tile(jj);
         for (int j = 0; j < n_tiles; ++j) {
-            prefetch_tile(j + kPrefetchTiles);
             // this CTA's 64-token page of tile j, all 576 values
             const int32_t t0 = seg.tok_begin + j * kTile;
             int32_t th = t0 + 64 * static_cast<int32_t>(c.rank);

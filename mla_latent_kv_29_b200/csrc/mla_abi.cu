@@ -356,7 +356,6 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         PP.part_offsets = part_offsets;
         PP.context_lens = context_lens;
         PP.block_table = block_table;
-        PP.pool = static_cast<const uint16_t*>(pool);
         PP.o_part = o_part;
         PP.lse_part = lse_part;
         PP.num_blocks = num_blocks;

@@ -131,12 +131,6 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
         : "memory");
 }
 
-// Starts pulling `bytes` (a multiple of 16) of global memory into L2.
-__device__ __forceinline__ void prefetch_l2(const void* gptr, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(gptr)), "r"(bytes)
-                 : "memory");
-}
-
 // 2-D tile load signalled on a barrier of this CTA.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, int32_t x, int32_t y, uint32_t bar) {
     asm volatile(
