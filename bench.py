@@ -303,7 +303,17 @@ def make_step(w, st, kernel):
     return step
 
 
-LAUNCHES_PER_STEP = 2 + 4  # append: GEMM + epilogue; decode: plan, absorb, attention, combine+W_UV
+def count_library_launches(step, device):
+    """Kernels of this library (names in the mla:: namespace) launched by one
+    untimed step, as seen by the CUDA activity profiler."""
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        step()
+        torch.cuda.synchronize(device)
+    names = [e.name for e in prof.events() if "CUDA" in str(e.device_type) and e.name.startswith("mla::")]
+    return len(names), sorted(set(n.split("(")[0] for n in names))
 
 
 def run_ours(args, w):
@@ -323,6 +333,7 @@ def run_ours(args, w):
         step()
     torch.cuda.synchronize(device)
     assert lib.device_error() == 0, "device fault during warm-up"
+    launches_per_step, kernel_names = count_library_launches(step, device)
 
     sampler = ClockSampler(device.index)
     soak_end = time.time() + args.soak
@@ -332,19 +343,32 @@ def run_ours(args, w):
         torch.cuda.synchronize(device)
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    ea = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ea = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    ea[0].record()
+    ea[1].record()  # the handles exist before any capture
+    graph = None
+    if args.graph:
+        # the step's launches are replayed from one CUDA graph (no host launch gaps)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step(events=ea)
+        graph.replay()
+        torch.cuda.synchronize(device)
+    run = graph.replay if graph is not None else (lambda: step(events=ea))
+    attn_ms = []
     barrier(device)
     torch.cuda.synchronize(device)
     for k in range(K):
         flush.zero_()  # evicts L2 (126 MB) between timed steps
         ev[k][0].record()
-        step(events=ea[k])
+        run()
         ev[k][1].record()
+        ev[k][1].synchronize()
+        attn_ms.append(ea[0].elapsed_time(ea[1]))
     torch.cuda.synchronize(device)
     barrier(device)
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    attn_ms = [a.elapsed_time(b) for a, b in ea]
     assert lib.device_error() == 0, "device fault during the timed steps"
 
     # end to end through the public API with host buffers (pinned)
@@ -356,6 +380,12 @@ def run_ours(args, w):
     h_out = torch.empty(st["out"].shape, dtype=torch.bfloat16).pin_memory()
     d_x, d_qn, d_qp = torch.empty_like(st["x_new"]), torch.empty_like(st["q_nope"]), torch.empty_like(st["q_pe"])
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    e2e_graph = None
+    if args.graph:
+        e2e_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(e2e_graph):
+            step(x_new=d_x, q_nope=d_qn, q_pe=d_qp)
+        torch.cuda.synchronize(device)
     barrier(device)
     torch.cuda.synchronize(device)
     for k in range(K):
@@ -366,7 +396,10 @@ def run_ours(args, w):
         d_qp.copy_(h_qp, non_blocking=True)
         st["new_seq"].copy_(h_seq, non_blocking=True)
         st["new_pos"].copy_(h_pos, non_blocking=True)
-        step(x_new=d_x, q_nope=d_qn, q_pe=d_qp)
+        if e2e_graph is not None:
+            e2e_graph.replay()
+        else:
+            step(x_new=d_x, q_nope=d_qn, q_pe=d_qp)
         h_out.copy_(st["out"], non_blocking=True)
         e2e_ev[k][1].record()
     torch.cuda.synchronize(device)
@@ -393,7 +426,8 @@ def run_ours(args, w):
                    "context": f"U[{w.length_range[0]},{w.length_range[1]}]", "cached_tokens_per_gpu": tot["T"],
                    "heads": w.dims.num_heads, "latent": w.dims.kv_lora_rank, "rope": w.dims.rope_dim,
                    "page": w.dims.block_size, "paged": "shuffled", "l2": "flushed (256 MB write) before each step",
-                   "step": "append of the batch's new tokens + absorbed decode"},
+                   "step": "append of the batch's new tokens + absorbed decode",
+                   "launch": "CUDA graph replay" if args.graph else "direct launches"},
         "roofline": roof,
         "attn_us": round(t_attn * 1e3, 2),
         "attn_hbm_gbs": round(attn_gbs, 1), "attn_tflops": round(attn_tfs, 2),
@@ -405,7 +439,8 @@ def run_ours(args, w):
                 "h2d_bytes_per_step": (h_x.numel() + h_qn.numel() + h_qp.numel()) * 2
                                       + (h_seq.numel() + h_pos.numel()) * 4,
                 "d2h_bytes_per_step": h_out.numel() * 2},
-        "gpu_launches": LAUNCHES_PER_STEP * K,
+        "gpu_launches": launches_per_step * K,
+        "kernels": kernel_names,
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -455,6 +490,8 @@ def main(argv=None):
     ap.add_argument("--soak", type=float, default=1.5, help="seconds of untimed steps while clocks are sampled")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
+                    help="replay each step from a captured CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -82,7 +82,10 @@ typedef struct mla_decode_opts {
                             balanced schedule targets (>= 1) */
     void* event_attn_begin; /* NULL or a cudaEvent_t recorded on `stream` right
                                before the split-KV attention kernel */
-    void* event_attn_end;   /* NULL or a cudaEvent_t recorded right after it */
+    void* event_attn_end;   /* NULL or a cudaEvent_t recorded right after it.
+                               Under stream capture both are captured as
+                               external event-record nodes, so a graph
+                               replay records them again. */
 } mla_decode_opts_t;
 
 /* Paged latent cache ("pool"), [MLA-arch] 3.2 kept as one row per token:

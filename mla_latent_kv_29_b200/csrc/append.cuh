@@ -86,10 +86,18 @@ __global__ void __launch_bounds__(256) append_epilogue_kernel(AppendEpiloguePara
     __shared__ float red[32];
     const int t = blockIdx.x;
     const int N = P.dc + P.dr;
+    const int64_t split_stride = static_cast<int64_t>(P.T) * N;
     for (int n = threadIdx.x; n < N; n += blockDim.x) {
-        float s = 0.f;
-        for (int k = 0; k < P.splits; ++k) s += P.part[(static_cast<int64_t>(k) * P.T + t) * N + n];
-        kv[n] = s;
+        // independent loads of all splits first, then the sum
+        const float* src = P.part + static_cast<int64_t>(t) * N + n;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        int k = 0;
+        for (; k + 8 <= P.splits; k += 8) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc[u] += __ldg(src + (k + u) * split_stride);
+        }
+        for (; k < P.splits; ++k) acc[0] += __ldg(src + k * split_stride);
+        kv[n] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
     }
     __syncthreads();
     // RMSNorm over the latent part

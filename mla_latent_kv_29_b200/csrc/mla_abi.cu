@@ -300,6 +300,18 @@ size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t batch, int32_t 
     return L.total;
 }
 
+// Timing hook: inside a stream capture the event becomes an external
+// event-record node of the graph, so that it is recorded on every replay.
+static void record_hook(void* ev, cudaStream_t st) {
+    if (!ev) return;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(st, &cs);
+    if (cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev), st, cudaEventRecordExternal);
+    else
+        cudaEventRecord(static_cast<cudaEvent_t>(ev), st);
+}
+
 int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int32_t batch, int32_t q_len,
                const void* pool, int64_t num_blocks, const int32_t* block_table, int32_t max_blocks_per_seq,
                const int32_t* context_lens, int32_t max_context_len, const void* w_uk, const void* w_uv,
@@ -365,10 +377,10 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         PP.q_len = q_len;
         PP.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
         if (int rc = ensure_smem(pair::pair_decode_kernel, pair::kSmemBytes)) return rc;
-        if (opts && opts->event_attn_begin) cudaEventRecord(static_cast<cudaEvent_t>(opts->event_attn_begin), st);
+        record_hook(opts ? opts->event_attn_begin : nullptr, st);
         pair::pair_decode_kernel<<<2 * L.workers, pair::kThreads, pair::kSmemBytes, st>>>(tm_q, tm_kv64, tm_kv32, PP);
         if (int rc = launch_status()) return rc;
-        if (opts && opts->event_attn_end) cudaEventRecord(static_cast<cudaEvent_t>(opts->event_attn_end), st);
+        record_hook(opts ? opts->event_attn_end : nullptr, st);
     } else {
     GenericDecodeParams P;
     P.q = q;
@@ -391,10 +403,10 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     P.scale = dims->softmax_scale;
     const size_t gsmem = generic_decode_smem(dc, dr);
     if (int rc = ensure_smem(generic_decode_kernel, gsmem)) return rc;
-    if (opts && opts->event_attn_begin) cudaEventRecord(static_cast<cudaEvent_t>(opts->event_attn_begin), st);
+    record_hook(opts ? opts->event_attn_begin : nullptr, st);
     generic_decode_kernel<<<dim3(L.workers, (H + kGenHeads - 1) / kGenHeads), kGenThreads, gsmem, st>>>(P);
     if (int rc = launch_status()) return rc;
-    if (opts && opts->event_attn_end) cudaEventRecord(static_cast<cudaEvent_t>(opts->event_attn_end), st);
+    record_hook(opts ? opts->event_attn_end : nullptr, st);
     }
 
     if (tc) {
