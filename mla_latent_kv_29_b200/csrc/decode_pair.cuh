@@ -23,12 +23,15 @@
 // once as values), so shared-memory fills are ~1.9x the HBM bytes, while
 // HBM reads stay ~1x because the second read of a page hits L2.
 //
-// Warp roles per CTA (256 threads): one thread of warp 0 streams the queries
-// and the key stages (three 64-column boxes of the CTA's page, 24 KB) into a
-// one-tile key ring; one thread of warp 2 streams the value stages (32
-// tokens x 256 columns, 16 KB) into a one-tile value ring; warp 1 allocates
-// tensor memory (both CTAs) and one of its threads, in the leader, issues the
-// MMAs; warps 4-7 (thread t = TMEM lane t) run the softmax,
+// Warp roles per CTA (288 threads): one thread of warp 0 streams the queries
+// and the key stages (three 64-column blocks of the CTA's page, 24 KB, one
+// TMA operation each) into a one-tile key ring; one thread of warp 2 streams
+// the value stages (32 tokens x 256 columns, 16 KB) into a one-tile value
+// ring; warp 1 allocates tensor memory (both CTAs). In the leader, three
+// threads issue the MMAs: lane 0 of warp 1 the score MMAs of even tiles,
+// lane 0 of warp 3 those of odd tiles, lane 0 of warp 8 the value MMAs (one
+// thread cannot issue tcgen05.mma fast enough for the M 128 x N 128 score
+// instructions). Warps 4-7 (thread t = TMEM lane t) run the softmax,
 // rescale O when the running max grows by more than 2^8, write P to shared
 // memory and, at the end of a segment, normalise O and write the partial.
 // Every mbarrier wait is bounded (see ptx::mbar_wait): on expiry the kernel
@@ -52,7 +55,12 @@ constexpr int kKStages = 3;          // key ring: one tile
 constexpr int kVStage = 2 * kBox;    // value stage: 32 tokens x 256 latent columns (4 x 4 KB)
 constexpr int kVPerTile = 4;         // 4 value stages per tile
 constexpr int kVStages = 4;          // value ring: one tile
-constexpr int kThreads = 256;
+// Pages are pulled into L2 this many tiles ahead of their TMA loads (0: off).
+#ifndef MLA_PAIR_PREFETCH_TILES
+#define MLA_PAIR_PREFETCH_TILES 0
+#endif
+constexpr int kPrefetchTiles = MLA_PAIR_PREFETCH_TILES;
+constexpr int kThreads = 288;  // 9 warps; the softmax warps 4-7 own TMEM lanes 0-127
 constexpr int kTmemCols = 512;
 constexpr int kTmS = 0;          // two S buffers of 64 columns
 constexpr int kTmO = 128;        // O: 256 columns
@@ -65,13 +73,15 @@ constexpr int kOffBar = kOffP + 2 * kBox;
 
 enum Bar {
     B_QFULL = 0, B_QEMPTY, B_SFULL0, B_SFULL1, B_SEMPTY0, B_SEMPTY1, B_PFULL, B_PVDONE, B_OEMPTY, B_PATCH, B_XCHG,
-    B_KFULL0, B_KEMPTY0 = B_KFULL0 + kKStages, B_VFULL0 = B_KEMPTY0 + kKStages, B_VEMPTY0 = B_VFULL0 + kVStages,
+    // key-full barriers come in two sets, for even and odd tiles (one per score issuer)
+    B_KFULL0, B_KEMPTY0 = B_KFULL0 + 2 * kKStages, B_VFULL0 = B_KEMPTY0 + kKStages, B_VEMPTY0 = B_VFULL0 + kVStages,
     B_COUNT = B_VEMPTY0 + kVStages
 };
 constexpr int kOffRed = kOffBar + 8 * 64;          // exchange buffer [2][128] floats
 constexpr int kOffMisc = kOffRed + 2 * 128 * 4;    // abort flag, TMEM base
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;   // + slack to align the base to 1 KB
 static_assert(B_COUNT <= 64, "barrier area");
+static_assert(kKStages == kKPerTile, "the score issuers assume a key ring of exactly one tile");
 
 struct Params {
     const PlanHeader* hdr;
@@ -79,6 +89,7 @@ struct Params {
     const int32_t* part_offsets;
     const int32_t* context_lens;
     const int32_t* block_table;
+    const uint16_t* pool;  // [num_blocks * block_size, 576], for the L2 prefetch
     float* o_part;  // [n_parts, 128, 512]
     float* lse_part;  // [n_parts, 128]
     int64_t num_blocks;
@@ -105,10 +116,13 @@ __device__ __forceinline__ void ring_next(uint32_t& stage, uint32_t& phase) {
     if (++stage == N) { stage = 0; phase ^= 1; }
 }
 
-// Queries and key stages; one thread (lane 0 of warp 0).
-__device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUtensorMap* tm_kv64, const Ctx& c) {
+// Queries and key stages; one thread (lane 0 of warp 0). tm_q and tm_k are
+// 3-D maps {64 columns, rows, 9 column blocks} with boxes {64, 64, 9} and
+// {64, 64, 3}: one TMA operation fills the whole query block or key stage.
+__device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUtensorMap* tm_k, const Ctx& c) {
     uint32_t stage = 0, phase = 0;
     int seg_i = 0;
+    uint32_t ktile = 0;  // running tile count of this pair
     SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
     Segment seg;
     while (it.next(seg)) {
@@ -117,11 +131,21 @@ __device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUt
         {
             const uint32_t full = c.leader_bar(B_QFULL);
             ptx::mbar_arrive_expect_tx_cluster(full, kQBoxes * kBox);
-            for (int k = 0; k < kQBoxes; ++k)
-                ptx::tma_load_2d_pair(c.sbase + kOffQ + k * kBox, tm_q, 64 * k, g * kH + 64 * c.rank, full);
+            ptx::tma_load_3d_pair(c.sbase + kOffQ, tm_q, 0, g * kH + 64 * c.rank, 0, full);
         }
         const int n_tiles = tiles_of(seg);
+        // L2 prefetch of this CTA's page of tile jj (only pages that hold visible tokens)
+        auto prefetch_tile = [&](int jj) {
+            if (kPrefetchTiles <= 0 || jj >= n_tiles) return;
+            const int32_t t = seg.tok_begin + jj * kTile + 64 * static_cast<int32_t>(c.rank);
+            if (t >= seg.tok_end) return;
+            const int64_t row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks,
+                                            P.block_size, b, t);
+            if (row >= 0) ptx::prefetch_l2(P.pool + row * kD, 64 * kD * 2);
+        };
+        for (int jj = 1; jj <= kPrefetchTiles; ++jj) prefetch_tile(jj);
         for (int j = 0; j < n_tiles; ++j) {
+            if (j > 0) prefetch_tile(j + kPrefetchTiles);
             // this CTA's 64-token page of tile j, all 576 values
             const int32_t t0 = seg.tok_begin + j * kTile;
             int32_t th = t0 + 64 * static_cast<int32_t>(c.rank);
@@ -134,13 +158,13 @@ __device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUt
             }
             for (int ks = 0; ks < kKPerTile; ++ks) {
                 if (!ptx::mbar_wait(c.bar(B_KEMPTY0 + stage), phase ^ 1, c.abort)) return;
-                const uint32_t full = c.leader_bar(B_KFULL0 + stage);
+                const uint32_t full = c.leader_bar(B_KFULL0 + (ktile & 1) * kKStages + stage);
                 ptx::mbar_arrive_expect_tx_cluster(full, kKStage);
-                for (int bx = 0; bx < 3; ++bx)
-                    ptx::tma_load_2d_pair(c.sbase + kOffK + stage * kKStage + bx * kBox, tm_kv64, 64 * (3 * ks + bx),
-                                          static_cast<int32_t>(row), full);
+                ptx::tma_load_3d_pair(c.sbase + kOffK + stage * kKStage, tm_k, 0, static_cast<int32_t>(row), 3 * ks,
+                                      full);
                 ring_next<kKStages>(stage, phase);
             }
+            ++ktile;
         }
         ++seg_i;
     }
@@ -157,8 +181,10 @@ __device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUt
 
 // Value stages; one thread (lane 0 of warp 2). Stage q of a tile holds tokens
 // 32q..32q+31 and this CTA's latent columns 256r..256r+255 as four 4 KB boxes:
-// box (n, h) = columns 256r + 128n + 64h at offset (2n + h) * 4 KB.
-__device__ void value_producer(const Params& P, const CUtensorMap* tm_kv32, const Ctx& c) {
+// box (n, h) = columns 256r + 128n + 64h at offset (2n + h) * 4 KB. tm_v is a
+// 3-D map {64 columns, rows, 9 column blocks} with box {64, 32, 4}: one TMA
+// operation fills a stage.
+__device__ void value_producer(const Params& P, const CUtensorMap* tm_v, const Ctx& c) {
     uint32_t stage = 0, phase = 0, patch_phase = 0;
     SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
     Segment seg;
@@ -178,21 +204,17 @@ __device__ void value_producer(const Params& P, const CUtensorMap* tm_kv32, cons
                 if (!ptx::mbar_wait(c.bar(B_VEMPTY0 + stage), phase ^ 1, c.abort)) return;
                 const uint32_t full = c.leader_bar(B_VFULL0 + stage);
                 const uint32_t dst = c.sbase + kOffV + stage * kVStage;
-                const int32_t x0 = 256 * static_cast<int32_t>(c.rank);
+                const int32_t z0 = 4 * static_cast<int32_t>(c.rank);  // column block of latent column 256r
                 if (row >= 0 && nv == 32) {
                     ptx::mbar_arrive_expect_tx_cluster(full, kVStage);
-                    for (int bx = 0; bx < 4; ++bx)
-                        ptx::tma_load_2d_pair(dst + bx * (kBox / 2), tm_kv32, x0 + 64 * bx, static_cast<int32_t>(row),
-                                              full);
+                    ptx::tma_load_3d_pair(dst, tm_v, 0, static_cast<int32_t>(row), z0, full);
                 } else {
                     // Tail of the visible range: rows past it may hold anything (even NaN),
                     // and 0 * NaN would poison O, so they are zeroed before the MMA reads them.
                     int keep = 0;
                     if (row >= 0) {
                         ptx::mbar_arrive_expect_tx_local(c.bar(B_PATCH), kVStage);
-                        for (int bx = 0; bx < 4; ++bx)
-                            ptx::tma_load_2d(dst + bx * (kBox / 2), tm_kv32, x0 + 64 * bx, static_cast<int32_t>(row),
-                                             c.bar(B_PATCH));
+                        ptx::tma_load_3d(dst, tm_v, 0, static_cast<int32_t>(row), z0, c.bar(B_PATCH));
                         if (!ptx::mbar_wait(c.bar(B_PATCH), patch_phase, c.abort)) return;
                         patch_phase ^= 1;
                         keep = nv;
@@ -216,16 +238,38 @@ __device__ void value_producer(const Params& P, const CUtensorMap* tm_kv32, cons
 }
 
 // ------------------------------------------------------------------- MMA
-__device__ void mma_issuer(const Params& P, const Ctx& c) {
-    // runs in one thread (lane 0 of warp 1 of the leader CTA)
+// Three issuing threads in the leader CTA: two for the score MMAs (even and
+// odd tiles, one S buffer each) and one for the value MMAs. A single thread
+// issues at most about one tcgen05.mma every ~47 cycles, while an
+// M 128 x N 128 x K 16 pair instruction takes the tensor cores 32 cycles, and
+// the three streams are independent (different TMEM accumulators, operands
+// and barriers).
+struct Descs {
+    uint64_t dq, dk, dp, dv;
+    __device__ explicit Descs(const Ctx& c)
+        // base descriptors; operand offsets are added in 16-byte units to the start-address field
+        : dq(ptx::smem_desc_sw128(c.sbase + kOffQ, 16, 1024)),
+          dk(ptx::smem_desc_sw128(c.sbase + kOffK, 16, 1024)),
+          dp(ptx::smem_desc_sw128(c.sbase + kOffP, 16, 1024)),
+          dv(ptx::smem_desc_sw128(c.sbase + kOffV, kBox / 2, 1024)) {}
+};
+
+// S = Q K^T for the tiles of one parity (the pair's running tile count t,
+// t % 2 == parity) into S buffer `parity`; one thread per parity (lane 0 of
+// warp 1 and of warp 3 of the leader CTA). The key ring holds one tile; the
+// producer signals the fill of stage ks for tile t on the key-full barrier
+// of t's parity, so tile t = 2m + parity is phase m of that barrier. A
+// parity wait can only tell apart adjacent phases; here the barrier is never
+// two phases ahead of its waiter, since the fill for tile t + 2 needs this
+// thread's own MMAs of tile t to have released the stage (a single barrier
+// set for both threads would let the odd thread see phase -1 as complete).
+// Both threads commit QEMPTY once per segment (the barrier counts 2), after
+// waiting for the segment's query block, so that a thread without tiles in
+// a segment cannot arrive twice on one phase.
+__device__ void mma_s_issuer(const Params& P, const Ctx& c, uint32_t parity) {
     constexpr uint32_t kIdS = ptx::idesc_bf16(128, 128, false, false);
-    constexpr uint32_t kIdPV = ptx::idesc_bf16(128, 256, false, true);
-    // Base descriptors; operand offsets are added in 16-byte units to the start-address field.
-    const uint64_t dq = ptx::smem_desc_sw128(c.sbase + kOffQ, 16, 1024);
-    const uint64_t dk = ptx::smem_desc_sw128(c.sbase + kOffK, 16, 1024);
-    const uint64_t dp = ptx::smem_desc_sw128(c.sbase + kOffP, 16, 1024);
-    const uint64_t dv = ptx::smem_desc_sw128(c.sbase + kOffV, kBox / 2, 1024);
-    uint32_t kst = 0, kph = 0, vst = 0, vph = 0, tile_cnt = 0, pv_cnt = 0;
+    const Descs D(c);
+    uint32_t tile_cnt = 0;
     int seg_i = 0;
     SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
     Segment seg;
@@ -233,53 +277,65 @@ __device__ void mma_issuer(const Params& P, const Ctx& c) {
         if (!ptx::mbar_wait(c.bar(B_QFULL), seg_i & 1, c.abort)) return;
         ptx::tc_fence_after();
         const int n_tiles = tiles_of(seg);
-        for (int j = 0; j <= n_tiles; ++j) {
-            if (j < n_tiles) {  // S = Q K^T for tile j into S buffer sb
-                const uint32_t sb = tile_cnt & 1;
-                const uint32_t d_s = c.tmem + kTmS + 64 * sb;
-                if (!ptx::mbar_wait(c.bar(B_SEMPTY0 + sb), ((tile_cnt >> 1) & 1) ^ 1, c.abort)) return;
-                for (int ks = 0; ks < kKPerTile; ++ks) {
-                    if (!ptx::mbar_wait(c.bar(B_KFULL0 + kst), kph, c.abort)) return;
-                    ptx::tc_fence_after();
+        for (int j = 0; j < n_tiles; ++j, ++tile_cnt) {
+            if ((tile_cnt & 1) != parity) continue;
+            const uint32_t d_s = c.tmem + kTmS + 64 * parity;
+            const uint32_t kph = (tile_cnt >> 1) & 1;  // phase of this parity's key-full barriers
+            if (!ptx::mbar_wait(c.bar(B_SEMPTY0 + parity), ((tile_cnt >> 1) & 1) ^ 1, c.abort)) return;
+#pragma unroll 1
+            for (int ks = 0; ks < kKPerTile; ++ks) {
+                if (!ptx::mbar_wait(c.bar(B_KFULL0 + parity * kKStages + ks), kph, c.abort)) return;
+                ptx::tc_fence_after();
 #pragma unroll
-                    for (int bx = 0; bx < 3; ++bx) {
-                        const int k = 3 * ks + bx;
-                        const uint64_t a0 = dq + static_cast<uint64_t>((k * kBox) >> 4);
-                        const uint64_t b0 = dk + static_cast<uint64_t>((kst * kKStage + bx * kBox) >> 4);
+                for (int bx = 0; bx < 3; ++bx) {
+                    const int k = 3 * ks + bx;
+                    const uint64_t a0 = D.dq + static_cast<uint64_t>((k * kBox) >> 4);
+                    const uint64_t b0 = D.dk + static_cast<uint64_t>((ks * kKStage + bx * kBox) >> 4);
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            ptx::mma_bf16_pair(d_s, a0 + 2 * kk, b0 + 2 * kk, kIdS, (k | kk) != 0);
-                    }
-                    ptx::mma_commit_pair(c.bar(B_KEMPTY0 + kst), 0x3);
-                    ring_next<kKStages>(kst, kph);
+                    for (int kk = 0; kk < 4; ++kk)
+                        ptx::mma_bf16_pair(d_s, a0 + 2 * kk, b0 + 2 * kk, kIdS, (k | kk) != 0);
                 }
-                ptx::mma_commit_pair(c.bar(B_SFULL0 + sb), 0x3);
-                if (j == n_tiles - 1) ptx::mma_commit_pair(c.bar(B_QEMPTY), 0x3);
-                ++tile_cnt;
+                ptx::mma_commit_pair(c.bar(B_KEMPTY0 + ks), 0x3);
             }
-            if (j >= 1) {  // O += P V for tile j-1
-                const bool first = (j == 1);
-                if (!ptx::mbar_wait(c.bar(B_PFULL), pv_cnt & 1, c.abort)) return;
-                if (first && !ptx::mbar_wait(c.bar(B_OEMPTY), (seg_i & 1) ^ 1, c.abort)) return;
-                for (int q = 0; q < kVPerTile; ++q) {
-                    if (!ptx::mbar_wait(c.bar(B_VFULL0 + vst), vph, c.abort)) return;
-                    ptx::tc_fence_after();
-                    // A: P tokens 32q + 16kk .. +15 (box q/2, byte 64 (q&1) + 32 kk of each 128-byte row)
-                    const uint64_t a0 = dp + static_cast<uint64_t>(((q >> 1) * kBox + 64 * (q & 1)) >> 4);
-                    const uint64_t b0 = dv + static_cast<uint64_t>((vst * kVStage) >> 4);
+            ptx::mma_commit_pair(c.bar(B_SFULL0 + parity), 0x3);
+        }
+        ptx::mma_commit_pair(c.bar(B_QEMPTY), 0x3);
+        ++seg_i;
+    }
+}
+
+// O += P V for every tile; one thread (lane 0 of warp 8 of the leader CTA).
+__device__ void mma_pv_issuer(const Params& P, const Ctx& c) {
+    constexpr uint32_t kIdPV = ptx::idesc_bf16(128, 256, false, true);
+    const Descs D(c);
+    uint32_t vst = 0, vph = 0, pv_cnt = 0;
+    int seg_i = 0;
+    SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    Segment seg;
+    while (it.next(seg)) {
+        const int n_tiles = tiles_of(seg);
+        for (int j = 0; j < n_tiles; ++j) {
+            const bool first = (j == 0);
+            if (!ptx::mbar_wait(c.bar(B_PFULL), pv_cnt & 1, c.abort)) return;
+            if (first && !ptx::mbar_wait(c.bar(B_OEMPTY), (seg_i & 1) ^ 1, c.abort)) return;
+            for (int q = 0; q < kVPerTile; ++q) {
+                if (!ptx::mbar_wait(c.bar(B_VFULL0 + vst), vph, c.abort)) return;
+                ptx::tc_fence_after();
+                // A: P tokens 32q + 16kk .. +15 (box q/2, byte 64 (q&1) + 32 kk of each 128-byte row)
+                const uint64_t a0 = D.dp + static_cast<uint64_t>(((q >> 1) * kBox + 64 * (q & 1)) >> 4);
+                const uint64_t b0 = D.dv + static_cast<uint64_t>((vst * kVStage) >> 4);
 #pragma unroll
-                    for (int n = 0; n < 2; ++n)
+                for (int n = 0; n < 2; ++n)
 #pragma unroll
-                        for (int kk = 0; kk < 2; ++kk)
-                            ptx::mma_bf16_pair(c.tmem + kTmO + 128 * n, a0 + 2 * kk,
-                                               b0 + static_cast<uint64_t>((n * kBox + 2048 * kk) >> 4), kIdPV,
-                                               !(first && q == 0 && kk == 0));
-                    ptx::mma_commit_pair(c.bar(B_VEMPTY0 + vst), 0x3);
-                    ring_next<kVStages>(vst, vph);
-                }
-                ptx::mma_commit_pair(c.bar(B_PVDONE), 0x3);
-                ++pv_cnt;
+                    for (int kk = 0; kk < 2; ++kk)
+                        ptx::mma_bf16_pair(c.tmem + kTmO + 128 * n, a0 + 2 * kk,
+                                           b0 + static_cast<uint64_t>((n * kBox + 2048 * kk) >> 4), kIdPV,
+                                           !(first && q == 0 && kk == 0));
+                ptx::mma_commit_pair(c.bar(B_VEMPTY0 + vst), 0x3);
+                ring_next<kVStages>(vst, vph);
             }
+            ptx::mma_commit_pair(c.bar(B_PVDONE), 0x3);
+            ++pv_cnt;
         }
         ++seg_i;
     }
@@ -427,8 +483,8 @@ __device__ void softmax(const Params& P, const Ctx& c) {
 // ------------------------------------------------------------------ kernel
 // grid: 2 * workers CTAs (clusters of 2); block 256; dynamic smem kSmemBytes.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    pair_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv64,
-                       const __grid_constant__ CUtensorMap tm_kv32, const Params P) {
+    pair_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const Params P) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = ptx::smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -444,7 +500,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         *c.abort = 0;
         ptx::mbar_init(c.bar(B_QFULL), 2);
-        ptx::mbar_init(c.bar(B_QEMPTY), 1);
+        ptx::mbar_init(c.bar(B_QEMPTY), 2);
         ptx::mbar_init(c.bar(B_SFULL0), 1);
         ptx::mbar_init(c.bar(B_SFULL1), 1);
         ptx::mbar_init(c.bar(B_SEMPTY0), 8);
@@ -456,6 +512,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ptx::mbar_init(c.bar(B_XCHG), 4);
         for (int s = 0; s < kKStages; ++s) {
             ptx::mbar_init(c.bar(B_KFULL0 + s), 2);
+            ptx::mbar_init(c.bar(B_KFULL0 + kKStages + s), 2);
             ptx::mbar_init(c.bar(B_KEMPTY0 + s), 1);
         }
         for (int s = 0; s < kVStages; ++s) {
@@ -466,8 +523,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     if (warp == 0 && ptx::lane_id() == 0) {
         ptx::prefetch_tmap(&tm_q);
-        ptx::prefetch_tmap(&tm_kv64);
-        ptx::prefetch_tmap(&tm_kv32);
+        ptx::prefetch_tmap(&tm_k);
+        ptx::prefetch_tmap(&tm_v);
     }
     if (warp == 1) {
         ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), kTmemCols);
@@ -480,11 +537,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     c.tmem = *tmem_slot;
 
     if (warp == 0) {
-        if (ptx::lane_id() == 0) key_producer(P, &tm_q, &tm_kv64, c);
+        if (ptx::lane_id() == 0) key_producer(P, &tm_q, &tm_k, c);
     } else if (warp == 2) {
-        if (ptx::lane_id() == 0) value_producer(P, &tm_kv32, c);
-    } else if (warp == 1) {
-        if (c.rank == 0 && ptx::lane_id() == 0) mma_issuer(P, c);
+        if (ptx::lane_id() == 0) value_producer(P, &tm_v, c);
+    } else if (warp == 1 || warp == 3) {
+        if (c.rank == 0 && ptx::lane_id() == 0) mma_s_issuer(P, c, static_cast<uint32_t>(warp >> 1));
+    } else if (warp == 8) {
+        if (c.rank == 0 && ptx::lane_id() == 0) mma_pv_issuer(P, c);
     } else if (warp >= 4) {
         softmax(P, c);
     }

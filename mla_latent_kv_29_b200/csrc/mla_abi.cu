@@ -114,16 +114,20 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// 2-D bf16 tensor map over rows of `cols` values (row stride `cols` * 2 bytes),
-// box = box_rows x 64 values, 128-byte swizzle.
-int encode_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+// 3-D bf16 tensor map over rows of `cols` values seen as {64 columns, rows,
+// cols / 64 column blocks} (row stride cols * 2 bytes, block stride 128 bytes),
+// box = {64, box_rows, box_blocks}, 128-byte swizzle. A box lands in shared
+// memory as box_blocks consecutive [box_rows x 64] swizzled tiles, the same
+// bytes as box_blocks separate 2-D boxes of 64 columns.
+int encode_row_blocks(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows,
+                      uint32_t box_blocks) {
     auto fn = tensor_map_encoder();
     if (!fn) return MLA_ERR_CUDA;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+    cuuint64_t dims[3] = {64, rows, cols / 64};
+    cuuint64_t strides[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64, box_rows, box_blocks};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
@@ -357,17 +361,18 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     if (int rc = launch_status()) return rc;
 
     if (L.kernel == kKernelPair) {
-        CUtensorMap tm_q, tm_kv64, tm_kv32;
+        CUtensorMap tm_q, tm_k, tm_v;
         const uint64_t pool_rows = static_cast<uint64_t>(num_blocks) * dims->block_size;
-        if (int rc = encode_rows(&tm_q, q, pair::kD, static_cast<uint64_t>(G) * H, 64)) return rc;
-        if (int rc = encode_rows(&tm_kv64, pool, pair::kD, pool_rows, 64)) return rc;
-        if (int rc = encode_rows(&tm_kv32, pool, pair::kD, pool_rows, 32)) return rc;
+        if (int rc = encode_row_blocks(&tm_q, q, pair::kD, static_cast<uint64_t>(G) * H, 64, pair::kQBoxes)) return rc;
+        if (int rc = encode_row_blocks(&tm_k, pool, pair::kD, pool_rows, 64, 3)) return rc;
+        if (int rc = encode_row_blocks(&tm_v, pool, pair::kD, pool_rows, 32, 4)) return rc;
         pair::Params PP;
         PP.hdr = hdr;
         PP.tile_prefix = tile_prefix;
         PP.part_offsets = part_offsets;
         PP.context_lens = context_lens;
         PP.block_table = block_table;
+        PP.pool = static_cast<const uint16_t*>(pool);
         PP.o_part = o_part;
         PP.lse_part = lse_part;
         PP.num_blocks = num_blocks;
@@ -378,7 +383,7 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         PP.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
         if (int rc = ensure_smem(pair::pair_decode_kernel, pair::kSmemBytes)) return rc;
         record_hook(opts ? opts->event_attn_begin : nullptr, st);
-        pair::pair_decode_kernel<<<2 * L.workers, pair::kThreads, pair::kSmemBytes, st>>>(tm_q, tm_kv64, tm_kv32, PP);
+        pair::pair_decode_kernel<<<2 * L.workers, pair::kThreads, pair::kSmemBytes, st>>>(tm_q, tm_k, tm_v, PP);
         if (int rc = launch_status()) return rc;
         record_hook(opts ? opts->event_attn_end : nullptr, st);
     } else {
