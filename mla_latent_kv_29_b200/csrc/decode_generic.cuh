@@ -24,6 +24,7 @@ struct GenericDecodeParams {
     const int32_t* block_table;
     const int32_t* context_lens;
     const PlanHeader* hdr;
+    const int32_t* worker_group;
     const int32_t* tile_prefix;
     const int32_t* part_offsets;
     float* o_part;           // [n_parts, H, dc]
@@ -56,7 +57,7 @@ __global__ void __launch_bounds__(kGenThreads) generic_decode_kernel(GenericDeco
     const int cl = tid % 16;                  // column phase
     const int ncol = (P.dc + 15) / 16;
 
-    SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kGenTokens, blockIdx.x);
+    SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kGenTokens, blockIdx.x);
     Segment seg;
     while (it.next(seg)) {
         const int32_t g = seg.group;

@@ -25,15 +25,16 @@
 //
 // Warp roles per CTA (288 threads): one thread of warp 0 streams the queries
 // and the key stages (three 64-column blocks of the CTA's page, 24 KB, one
-// TMA operation each) into a one-tile key ring; one thread of warp 2 streams
-// the value stages (32 tokens x 256 columns, 16 KB) into a one-tile value
-// ring; warp 1 allocates tensor memory (both CTAs). In the leader, three
-// threads issue the MMAs: lane 0 of warp 1 the score MMAs of even tiles,
-// lane 0 of warp 3 those of odd tiles, lane 0 of warp 8 the value MMAs (one
-// thread cannot issue tcgen05.mma fast enough for the M 128 x N 128 score
-// instructions). Warps 4-7 (thread t = TMEM lane t) run the softmax,
-// rescale O when the running max grows by more than 2^8, write P to shared
-// memory and, at the end of a segment, normalise O and write the partial.
+// TMA operation each) into a one-tile key ring; warp 2 streams the value
+// stages (32 tokens x 256 columns, 16 KB) into a one-tile value ring (one
+// thread issues, the warp zeroes the tail rows of partial stages); warp 1
+// allocates tensor memory (both CTAs). In the leader, three threads issue
+// the MMAs: lane 0 of warp 1 the score MMAs of even tiles, lane 0 of warp 3
+// those of odd tiles, lane 0 of warp 8 the value MMAs (one thread cannot
+// issue tcgen05.mma fast enough for the M 128 x N 128 score instructions).
+// Warps 4-7 (thread t = TMEM lane t) run the softmax, rescale O when the
+// running max grows by more than 2^8, write P to shared memory and, at the
+// end of a segment, normalise O and write the partial.
 // Every mbarrier wait is bounded (see ptx::mbar_wait): on expiry the kernel
 // records MLA_ERR_DEVICE_TIMEOUT and every role drains to the common exit.
 #pragma once
@@ -85,6 +86,7 @@ static_assert(kKStages == kKPerTile, "the score issuers assume a key ring of exa
 
 struct Params {
     const PlanHeader* hdr;
+    const int32_t* worker_group;
     const int32_t* tile_prefix;
     const int32_t* part_offsets;
     const int32_t* context_lens;
@@ -123,7 +125,7 @@ __device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUt
     uint32_t stage = 0, phase = 0;
     int seg_i = 0;
     uint32_t ktile = 0;  // running tile count of this pair
-    SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
     Segment seg;
     while (it.next(seg)) {
         const int32_t g = seg.group, b = g / P.q_len;
@@ -179,14 +181,23 @@ __device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUt
     if (seg_i > 0) ptx::mbar_wait(c.bar(B_QEMPTY), (seg_i - 1) & 1, c.abort);
 }
 
-// Value stages; one thread (lane 0 of warp 2). Stage q of a tile holds tokens
-// 32q..32q+31 and this CTA's latent columns 256r..256r+255 as four 4 KB boxes:
-// box (n, h) = columns 256r + 128n + 64h at offset (2n + h) * 4 KB. tm_v is a
-// 3-D map {64 columns, rows, 9 column blocks} with box {64, 32, 4}: one TMA
-// operation fills a stage.
+// Value stages; warp 2 (lane 0 issues and waits, the whole warp zeroes the
+// tail rows of a partial stage). Stage q of a tile holds tokens 32q..32q+31
+// and this CTA's latent columns 256r..256r+255 as four 4 KB boxes: box (n, h)
+// = columns 256r + 128n + 64h at offset (2n + h) * 4 KB. tm_v is a 3-D map
+// {64 columns, rows, 9 column blocks} with box {64, 32, 4}: one TMA operation
+// fills a stage. Stages that hold no visible token are skipped here and by
+// the value-MMA issuer alike (their softmax weights are all zero).
 __device__ void value_producer(const Params& P, const CUtensorMap* tm_v, const Ctx& c) {
+    const uint32_t lane = ptx::lane_id();
     uint32_t stage = 0, phase = 0, patch_phase = 0;
-    SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    // a wait by lane 0, its outcome shared so that the warp stays converged
+    auto wait0 = [&](uint32_t bar, uint32_t parity) -> bool {
+        int ok = 1;
+        if (lane == 0) ok = ptx::mbar_wait(bar, parity, c.abort) ? 1 : 0;
+        return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    };
+    SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
     Segment seg;
     while (it.next(seg)) {
         const int32_t b = seg.group / P.q_len;
@@ -195,44 +206,48 @@ __device__ void value_producer(const Params& P, const CUtensorMap* tm_v, const C
             const int32_t tv = seg.tok_begin + j * kTile;
             for (int q = 0; q < kVPerTile; ++q) {
                 const int32_t tq = tv + 32 * q;
-                const int nv = max(0, min(32, seg.tok_end - tq));
-                int64_t row = -1;
-                if (nv > 0) {
-                    row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks, P.block_size, b, tq);
-                    if (row < 0) record_status(MLA_ERR_DEVICE_FAULT);
-                }
-                if (!ptx::mbar_wait(c.bar(B_VEMPTY0 + stage), phase ^ 1, c.abort)) return;
+                const int nv = min(32, seg.tok_end - tq);
+                if (nv <= 0) break;
+                const int64_t row =
+                    resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks, P.block_size, b, tq);
+                if (row < 0 && lane == 0) record_status(MLA_ERR_DEVICE_FAULT);
+                if (!wait0(c.bar(B_VEMPTY0 + stage), phase ^ 1)) return;
                 const uint32_t full = c.leader_bar(B_VFULL0 + stage);
                 const uint32_t dst = c.sbase + kOffV + stage * kVStage;
                 const int32_t z0 = 4 * static_cast<int32_t>(c.rank);  // column block of latent column 256r
                 if (row >= 0 && nv == 32) {
-                    ptx::mbar_arrive_expect_tx_cluster(full, kVStage);
-                    ptx::tma_load_3d_pair(dst, tm_v, 0, static_cast<int32_t>(row), z0, full);
+                    if (lane == 0) {
+                        ptx::mbar_arrive_expect_tx_cluster(full, kVStage);
+                        ptx::tma_load_3d_pair(dst, tm_v, 0, static_cast<int32_t>(row), z0, full);
+                    }
                 } else {
                     // Tail of the visible range: rows past it may hold anything (even NaN),
                     // and 0 * NaN would poison O, so they are zeroed before the MMA reads them.
                     int keep = 0;
                     if (row >= 0) {
-                        ptx::mbar_arrive_expect_tx_local(c.bar(B_PATCH), kVStage);
-                        ptx::tma_load_3d(dst, tm_v, 0, static_cast<int32_t>(row), z0, c.bar(B_PATCH));
-                        if (!ptx::mbar_wait(c.bar(B_PATCH), patch_phase, c.abort)) return;
+                        if (lane == 0) {
+                            ptx::mbar_arrive_expect_tx_local(c.bar(B_PATCH), kVStage);
+                            ptx::tma_load_3d(dst, tm_v, 0, static_cast<int32_t>(row), z0, c.bar(B_PATCH));
+                        }
+                        if (!wait0(c.bar(B_PATCH), patch_phase)) return;
                         patch_phase ^= 1;
                         keep = nv;
                     }
                     uint4* p = reinterpret_cast<uint4*>(c.smem + kOffV + stage * kVStage);
-                    for (int i = 0; i < kVStage / 16; ++i) {
+                    for (int i = static_cast<int>(lane); i < kVStage / 16; i += 32) {
                         const int r = (i & 255) >> 3;  // token row within its 4 KB box
                         if (r >= keep) p[i] = make_uint4(0u, 0u, 0u, 0u);
                     }
                     ptx::fence_proxy_async_smem();
-                    ptx::mbar_arrive_cluster(full);
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive_cluster(full);
                 }
                 ring_next<kVStages>(stage, phase);
             }
         }
     }
     for (int i = 0; i < kVStages; ++i) {  // tail, as for the key ring
-        if (!ptx::mbar_wait(c.bar(B_VEMPTY0 + stage), phase ^ 1, c.abort)) return;
+        if (!wait0(c.bar(B_VEMPTY0 + stage), phase ^ 1)) return;
         ring_next<kVStages>(stage, phase);
     }
 }
@@ -271,7 +286,7 @@ __device__ void mma_s_issuer(const Params& P, const Ctx& c, uint32_t parity) {
     const Descs D(c);
     uint32_t tile_cnt = 0;
     int seg_i = 0;
-    SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
     Segment seg;
     while (it.next(seg)) {
         if (!ptx::mbar_wait(c.bar(B_QFULL), seg_i & 1, c.abort)) return;
@@ -310,7 +325,7 @@ __device__ void mma_pv_issuer(const Params& P, const Ctx& c) {
     const Descs D(c);
     uint32_t vst = 0, vph = 0, pv_cnt = 0;
     int seg_i = 0;
-    SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
     Segment seg;
     while (it.next(seg)) {
         const int n_tiles = tiles_of(seg);
@@ -318,7 +333,9 @@ __device__ void mma_pv_issuer(const Params& P, const Ctx& c) {
             const bool first = (j == 0);
             if (!ptx::mbar_wait(c.bar(B_PFULL), pv_cnt & 1, c.abort)) return;
             if (first && !ptx::mbar_wait(c.bar(B_OEMPTY), (seg_i & 1) ^ 1, c.abort)) return;
+            const int32_t tv = seg.tok_begin + j * kTile;
             for (int q = 0; q < kVPerTile; ++q) {
+                if (seg.tok_end - (tv + 32 * q) <= 0) break;  // no visible token: skipped by the producer too
                 if (!ptx::mbar_wait(c.bar(B_VFULL0 + vst), vph, c.abort)) return;
                 ptx::tc_fence_after();
                 // A: P tokens 32q + 16kk .. +15 (box q/2, byte 64 (q&1) + 32 kk of each 128-byte row)
@@ -370,7 +387,7 @@ __device__ void softmax(const Params& P, const Ctx& c) {
     uint8_t* prow = c.smem + kOffP + half * kBox + hrow * 128;
     Exchanger xc{reinterpret_cast<float*>(c.smem + kOffRed), c.bar(B_XCHG)};
     uint32_t tile_cnt = 0, pv_wait = 0;
-    SegmentIter it(P.hdr, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
     Segment seg;
     while (it.next(seg)) {
         float m_run = -INFINITY, l_run = 0.f;
@@ -460,16 +477,32 @@ __device__ void softmax(const Params& P, const Ctx& c) {
         if (!xc.swap(l_run, lpart, t, c.abort)) return;
         const float l_tot = l_run + lpart;
         const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
-        float* dst = P.o_part + (static_cast<int64_t>(seg.slot) * kH + head) * kDc + 256 * half;
+        // O rows go out through the (now idle) P buffer: each thread writes its row's
+        // 32-column slice to shared memory (16-byte chunks XOR-swizzled by row), then
+        // the warp stores its 32 rows with 8 lanes per 128-byte row segment, so every
+        // global store instruction covers whole 128-byte lines.
+        float* const o_base = P.o_part + static_cast<int64_t>(seg.slot) * kH * kDc;
+        uint8_t* const stage_buf = c.smem + kOffP;
+        const int wrow0 = t & ~31;  // first row (thread) of this warp
 #pragma unroll 1
         for (int cc = 0; cc < 8; ++cc) {
             float o[32];
             ptx::tmem_ld32(tl + kTmO + 32 * cc, o);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4*>(dst + 32 * cc + i) =
-                    make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+            for (int k = 0; k < 8; ++k)
+                *reinterpret_cast<float4*>(stage_buf + t * 128 + ((k ^ (t & 7)) << 4)) =
+                    make_float4(o[4 * k] * inv, o[4 * k + 1] * inv, o[4 * k + 2] * inv, o[4 * k + 3] * inv);
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int r = wrow0 + 4 * k + static_cast<int>(lane >> 3), ch = static_cast<int>(lane & 7);
+                const float4 v = *reinterpret_cast<const float4*>(stage_buf + r * 128 + ((ch ^ (r & 7)) << 4));
+                const int r_head = 64 * static_cast<int>(c.rank) + (r & 63);
+                *reinterpret_cast<float4*>(o_base + static_cast<int64_t>(r_head) * kDc + 256 * (r >> 6) + 32 * cc +
+                                           4 * ch) = v;
+            }
+            __syncwarp();
         }
         if (half == 0)
             P.lse_part[static_cast<int64_t>(seg.slot) * kH + head] =
@@ -539,7 +572,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         if (ptx::lane_id() == 0) key_producer(P, &tm_q, &tm_k, c);
     } else if (warp == 2) {
-        if (ptx::lane_id() == 0) value_producer(P, &tm_v, c);
+        value_producer(P, &tm_v, c);
     } else if (warp == 1 || warp == 3) {
         if (c.rank == 0 && ptx::lane_id() == 0) mma_s_issuer(P, c, static_cast<uint32_t>(warp >> 1));
     } else if (warp == 8) {

@@ -71,7 +71,7 @@ int num_sms() {
 
 // ---- decode workspace ------------------------------------------------
 struct DecodeLayout {
-    size_t hdr, tile_prefix, part_offsets, q, o_part, lse_part, total;
+    size_t hdr, tile_prefix, part_offsets, worker_group, q, o_part, lse_part, total;
     int32_t workers, max_parts, kernel, tile;
 };
 
@@ -155,6 +155,7 @@ int decode_layout(const mla_dims_t* d, int32_t batch, int32_t q_len, int32_t max
     L->hdr = off; off = align_up(off + sizeof(PlanHeader));
     L->tile_prefix = off; off = align_up(off + sizeof(int32_t) * (G + 1));
     L->part_offsets = off; off = align_up(off + sizeof(int32_t) * (G + 1));
+    L->worker_group = off; off = align_up(off + sizeof(int32_t) * static_cast<size_t>(L->workers));
     L->q = off; off = align_up(off + sizeof(uint16_t) * G * d->num_heads * D);
     L->o_part = off; off = align_up(off + sizeof(float) * static_cast<size_t>(L->max_parts) * d->num_heads * d->kv_lora_rank);
     L->lse_part = off; off = align_up(off + sizeof(float) * static_cast<size_t>(L->max_parts) * d->num_heads);
@@ -335,13 +336,15 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     PlanHeader* hdr = reinterpret_cast<PlanHeader*>(ws + L.hdr);
     int32_t* tile_prefix = reinterpret_cast<int32_t*>(ws + L.tile_prefix);
     int32_t* part_offsets = reinterpret_cast<int32_t*>(ws + L.part_offsets);
+    int32_t* worker_group = reinterpret_cast<int32_t*>(ws + L.worker_group);
     uint16_t* q = reinterpret_cast<uint16_t*>(ws + L.q);
     float* o_part = reinterpret_cast<float*>(ws + L.o_part);
     float* lse_part = reinterpret_cast<float*>(ws + L.lse_part);
     const int32_t G = batch * q_len;
     const int H = dims->num_heads, dc = dims->kv_lora_rank, dr = dims->rope_dim;
 
-    plan_kernel<<<1, 1024, 0, st>>>(context_lens, batch, q_len, L.tile, L.workers, hdr, tile_prefix, part_offsets);
+    plan_kernel<<<1, 1024, 0, st>>>(context_lens, batch, q_len, L.tile, L.workers, hdr, tile_prefix, part_offsets,
+                                    worker_group);
     if (int rc = launch_status()) return rc;
 
     const bool tc = tc_gemm_dims_ok(dims) && aligned(q_nope, 16) && aligned(w_uk, 16) && aligned(w_uv, 16);
@@ -368,6 +371,7 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         if (int rc = encode_row_blocks(&tm_v, pool, pair::kD, pool_rows, 32, 4)) return rc;
         pair::Params PP;
         PP.hdr = hdr;
+        PP.worker_group = worker_group;
         PP.tile_prefix = tile_prefix;
         PP.part_offsets = part_offsets;
         PP.context_lens = context_lens;
@@ -393,6 +397,7 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     P.block_table = block_table;
     P.context_lens = context_lens;
     P.hdr = hdr;
+    P.worker_group = worker_group;
     P.tile_prefix = tile_prefix;
     P.part_offsets = part_offsets;
     P.o_part = o_part;

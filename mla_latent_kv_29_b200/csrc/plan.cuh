@@ -3,21 +3,28 @@
 //
 // A "group" is one new token of one sequence: g = b * q_len + s. Group g
 // sees vis(g) = L_b - q_len + s + 1 cached tokens (the causal rule for
-// several new tokens), i.e. ceil(vis / tile) tiles. All groups' tiles are
-// laid end to end (W tiles in total) and cut into P contiguous, non-empty
-// ranges, one per worker: worker p owns tiles [floor(W p / P),
-// floor(W (p+1) / P)). A worker emits one partial (o, lse) per group it
-// touches; group g's partials are the consecutive slots
-// part_offsets[g] .. part_offsets[g+1]-1, ordered by worker.
+// several new tokens), i.e. n_g = ceil(vis / tile) tiles. Every segment a
+// worker runs costs a fixed start-up (query load, pipeline fill, partial
+// write-out) on top of its tiles, so the schedule is cut in "units": each
+// group contributes kSegUnits units for that cost followed by one unit per
+// tile. Group g starts at unit V0(g) = tile_prefix[g] + kSegUnits * g; its
+// tile k sits at unit V0(g) + kSegUnits + k. The W' = V0(G) units are cut
+// into P contiguous ranges, worker p owning [floor(W' p / P), floor(W' (p+1) / P)).
+// A worker emits one partial (o, lse) per group whose tiles it touches;
+// group g's partials are the consecutive slots part_offsets[g] ..
+// part_offsets[g+1]-1, ordered by worker. worker_group[p] is the group whose
+// units hold the start of worker p's range.
 #pragma once
 
 #include "common.cuh"
 
 namespace mla {
 
+constexpr int32_t kSegUnits = 1;  // schedule units charged per segment (about one tile of time)
+
 struct PlanHeader {
-    int32_t total_tiles;  // W
-    int32_t workers;      // P (<= requested workers, <= W; 0 when W == 0)
+    int32_t total_units;  // W' (0 when no group has a visible token)
+    int32_t workers;      // P (<= requested workers, <= W'; 0 when W' == 0)
     int32_t n_groups;     // G
     int32_t n_parts;      // part_offsets[G]
 };
@@ -26,11 +33,14 @@ __host__ __device__ __forceinline__ int32_t worker_begin(int32_t p, int32_t W, i
     return static_cast<int32_t>((static_cast<int64_t>(W) * p) / P);
 }
 
-// The worker whose range holds tile t (largest p with worker_begin(p) <= t).
-__host__ __device__ __forceinline__ int32_t worker_of_tile(int32_t t, int32_t W, int32_t P) {
-    return static_cast<int32_t>(((static_cast<int64_t>(t) + 1) * P - 1) / W);
+// The worker whose range holds unit v (largest p with worker_begin(p) <= v).
+__host__ __device__ __forceinline__ int32_t worker_of_unit(int32_t v, int32_t W, int32_t P) {
+    return static_cast<int32_t>(((static_cast<int64_t>(v) + 1) * P - 1) / W);
 }
 
+__device__ __forceinline__ int32_t group_units_start(const int32_t* __restrict__ tile_prefix, int32_t g) {
+    return tile_prefix[g] + kSegUnits * g;
+}
 __device__ __forceinline__ int32_t group_tiles(const int32_t* __restrict__ context_lens, int32_t q_len,
                                                int32_t g, int32_t tile) {
     const int32_t b = g / q_len, s = g - b * q_len;
@@ -45,12 +55,12 @@ __device__ __forceinline__ int32_t group_visible(const int32_t* __restrict__ con
     return vis > 0 ? vis : 0;
 }
 
-// Largest g with tile_prefix[g] <= t (the non-empty group owning tile t).
-__device__ __forceinline__ int32_t group_of_tile(const int32_t* __restrict__ tile_prefix, int32_t G, int32_t t) {
+// Largest g in [0, G) with V0(g) <= v (the group whose units hold unit v).
+__device__ __forceinline__ int32_t group_of_unit(const int32_t* __restrict__ tile_prefix, int32_t G, int32_t v) {
     int32_t lo = 0, hi = G - 1;
     while (lo < hi) {
         const int32_t mid = (lo + hi + 1) >> 1;
-        if (tile_prefix[mid] <= t) lo = mid; else hi = mid - 1;
+        if (group_units_start(tile_prefix, mid) <= v) lo = mid; else hi = mid - 1;
     }
     return lo;
 }
@@ -83,12 +93,14 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
     return r;
 }
 
-// <<<1, 1024>>>. tile_prefix and part_offsets have G + 1 entries.
+// <<<1, 1024>>>. tile_prefix and part_offsets have G + 1 entries,
+// worker_group max_workers entries.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ context_lens, int32_t batch,
                                                     int32_t q_len, int32_t tile, int32_t max_workers,
                                                     PlanHeader* __restrict__ hdr,
                                                     int32_t* __restrict__ tile_prefix,
-                                                    int32_t* __restrict__ part_offsets) {
+                                                    int32_t* __restrict__ part_offsets,
+                                                    int32_t* __restrict__ worker_group) {
     __shared__ int32_t warp_tot[32];
     __shared__ int32_t chunk_total;
     const int32_t G = batch * q_len;
@@ -101,9 +113,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
         carry += chunk_total;
         __syncthreads();
     }
-    const int32_t W = carry;
+    const int32_t W = carry > 0 ? carry + kSegUnits * G : 0;
     const int32_t P = W > 0 ? min(max_workers, W) : 0;
-    if (threadIdx.x == 0) tile_prefix[G] = W;
+    if (threadIdx.x == 0) tile_prefix[G] = carry;
     __syncthreads();
     carry = 0;
     for (int32_t base = 0; base < G; base += 1024) {
@@ -111,16 +123,21 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
         int32_t n = 0;
         if (g < G) {
             const int32_t t0 = tile_prefix[g], t1 = tile_prefix[g + 1];
-            if (t1 > t0) n = worker_of_tile(t1 - 1, W, P) - worker_of_tile(t0, W, P) + 1;
+            if (t1 > t0) {
+                const int32_t v0 = t0 + kSegUnits * (g + 1);  // unit of the group's first tile
+                n = worker_of_unit(v0 + (t1 - t0) - 1, W, P) - worker_of_unit(v0, W, P) + 1;
+            }
         }
         const int32_t ex = block_exclusive_scan(n, warp_tot, &chunk_total);
         if (g < G) part_offsets[g] = carry + ex;
         carry += chunk_total;
         __syncthreads();
     }
+    for (int32_t p = threadIdx.x; p < P; p += 1024)
+        worker_group[p] = group_of_unit(tile_prefix, G, worker_begin(p, W, P));
     if (threadIdx.x == 0) {
         part_offsets[G] = carry;
-        hdr->total_tiles = W;
+        hdr->total_units = W;
         hdr->workers = P;
         hdr->n_groups = G;
         hdr->n_parts = carry;
@@ -141,34 +158,40 @@ struct SegmentIter {
     const int32_t* part_offsets;
     const int32_t* context_lens;
     int32_t G, q_len, tile, W, P, p;
-    int32_t t, t_end;
+    int32_t g, v, v_end;  // next group to look at; this worker's unit range [v, v_end)
 
-    __device__ SegmentIter(const PlanHeader* hdr, const int32_t* tp, const int32_t* po, const int32_t* cl,
-                           int32_t q_len_, int32_t tile_, int32_t worker)
+    __device__ SegmentIter(const PlanHeader* hdr, const int32_t* worker_group, const int32_t* tp, const int32_t* po,
+                           const int32_t* cl, int32_t q_len_, int32_t tile_, int32_t worker)
         : tile_prefix(tp), part_offsets(po), context_lens(cl), q_len(q_len_), tile(tile_), p(worker) {
         G = hdr->n_groups;
-        W = hdr->total_tiles;
+        W = hdr->total_units;
         P = hdr->workers;
         if (p < P) {
-            t = worker_begin(p, W, P);
-            t_end = worker_begin(p + 1, W, P);
+            v = worker_begin(p, W, P);
+            v_end = worker_begin(p + 1, W, P);
+            g = worker_group[p];
         } else {
-            t = t_end = 0;
+            v = v_end = 0;
+            g = G;
         }
     }
 
     __device__ bool next(Segment& s) {
-        if (t >= t_end) return false;
-        const int32_t g = group_of_tile(tile_prefix, G, t);
-        const int32_t g0 = tile_prefix[g], g1 = tile_prefix[g + 1];
-        const int32_t hi = min(t_end, g1);
-        const int32_t vis = group_visible(context_lens, q_len, g);
-        s.group = g;
-        s.tok_begin = (t - g0) * tile;
-        s.tok_end = min((hi - g0) * tile, vis);
-        s.slot = part_offsets[g] + (p - worker_of_tile(g0, W, P));
-        t = hi;
-        return true;
+        while (g < G) {
+            const int32_t t0 = tile_prefix[g], t1 = tile_prefix[g + 1];
+            const int32_t u = t0 + kSegUnits * (g + 1);  // unit of the group's first tile
+            if (u - kSegUnits >= v_end) break;
+            const int32_t k0 = max(0, v - u), k1 = min(t1 - t0, v_end - u);
+            const int32_t gg = g++;
+            if (k1 <= k0) continue;
+            s.group = gg;
+            s.tok_begin = k0 * tile;
+            s.tok_end = min(k1 * tile, group_visible(context_lens, q_len, gg));
+            s.slot = part_offsets[gg] + (p - worker_of_unit(u, W, P));
+            return true;
+        }
+        g = G;
+        return false;
     }
 };
 
