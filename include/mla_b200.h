@@ -150,9 +150,15 @@ MLA_API size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t n_token
  *   workspace >= mla_decode_workspace_size(...) bytes, 256-byte aligned,
  *           contents need not be initialised
  *   opts    NULL or kernel / split overrides
+ * Alignment: q_nope, w_uk, w_uv and out 16-byte aligned select the
+ * tensor-core GEMMs around the attention; the tcgen05 attention kernel
+ * (opts->kernel = 1, the default for DeepSeek-V3 dims) requires them and
+ * returns MLA_ERR_INVALID_ARG otherwise.
  * Rounding: q_lat is rounded to bf16 before the score product and the
- * softmax weights to bf16 before the value product; accumulation, partials
- * and the combine are fp32; out is rounded to bf16 once. */
+ * softmax weights to bf16 before the value product; accumulation and the
+ * combine are fp32; split partials are fp32 (CUDA-core kernel) or rounded
+ * to bf16 (tcgen05 kernel); o_lat is rounded to bf16 before the
+ * up-projection and out to bf16 once. */
 MLA_API int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe,
                int32_t batch, int32_t q_len,
                const void* pool, int64_t num_blocks,

@@ -24,17 +24,20 @@
 // HBM reads stay ~1x because the second read of a page hits L2.
 //
 // Warp roles per CTA (288 threads): one thread of warp 0 streams the queries
-// and the key stages (three 64-column blocks of the CTA's page, 24 KB, one
-// TMA operation each) into a one-tile key ring; warp 2 streams the value
-// stages (32 tokens x 256 columns, 16 KB) into a one-tile value ring (one
+// and the key stages (column blocks 0-2, 3-4, 5-6 and 7-8 of the CTA's page,
+// one TMA operation each) into a one-tile key ring; warp 2 streams the value
+// stages (32 tokens x 256 columns, 16 KB) into a three-stage value ring (one
 // thread issues, the warp zeroes the tail rows of partial stages); warp 1
 // allocates tensor memory (both CTAs). In the leader, three threads issue
-// the MMAs: lane 0 of warp 1 the score MMAs of even tiles, lane 0 of warp 3
-// those of odd tiles, lane 0 of warp 8 the value MMAs (one thread cannot
-// issue tcgen05.mma fast enough for the M 128 x N 128 score instructions).
+// the MMAs: lanes 0 of warps 1 and 3 the score MMAs of every tile (column
+// blocks 0-4 and 5-8, into two half-accumulators that the softmax adds),
+// lane 0 of warp 8 the value MMAs (one thread cannot issue tcgen05.mma fast
+// enough for the M 128 x N 128 score instructions).
 // Warps 4-7 (thread t = TMEM lane t) run the softmax, rescale O when the
-// running max grows by more than 2^8, write P to shared memory and, at the
-// end of a segment, normalise O and write the partial.
+// running max grows by more than 2^8, write P to shared memory (two buffers,
+// by tile parity, so that the P of tile j is written while the value MMAs of
+// tile j-1 still run) and, at the end of a segment, normalise O and write
+// the partial.
 // Every mbarrier wait is bounded (see ptx::mbar_wait): on expiry the kernel
 // records MLA_ERR_DEVICE_TIMEOUT and every role drains to the common exit.
 #pragma once
@@ -50,39 +53,41 @@ constexpr int kH = 128, kDc = 512, kDr = 64, kD = kDc + kDr;
 constexpr int kTile = 128;       // tokens per pair iteration
 constexpr int kBox = 8192;       // one [64 rows x 64 bf16] 128B-swizzled box
 constexpr int kQBoxes = kD / 64; // 9
-constexpr int kKStage = 3 * kBox;    // key stage: three 64-column boxes of a page (24 KB)
-constexpr int kKPerTile = kQBoxes / 3;  // 3 key stages per tile
-constexpr int kKStages = 3;          // key ring: one tile
+// Key ring: one tile = the CTA's page as 9 [64 x 64] boxes in column-block
+// order, filled as 4 stages (blocks 0-2, 3-4, 5-6, 7-8). The score MMAs of a
+// tile are split by column blocks between two issuing threads: "lo" takes
+// blocks 0-4 (stages 0, 1) into one accumulator, "hi" blocks 5-8 (stages 2,
+// 3) into another, and the softmax adds the two.
+constexpr int kKStages = 4;
+__host__ __device__ constexpr int kstage_first_block(int s) { return s == 0 ? 0 : 1 + 2 * s; }
+__host__ __device__ constexpr int kstage_blocks(int s) { return s == 0 ? 3 : 2; }
+constexpr int kKTile = kQBoxes * kBox;  // 72 KB
 constexpr int kVStage = 2 * kBox;    // value stage: 32 tokens x 256 latent columns (4 x 4 KB)
 constexpr int kVPerTile = 4;         // 4 value stages per tile
-constexpr int kVStages = 4;          // value ring: one tile
-// Pages are pulled into L2 this many tiles ahead of their TMA loads (0: off).
-#ifndef MLA_PAIR_PREFETCH_TILES
-#define MLA_PAIR_PREFETCH_TILES 0
-#endif
-constexpr int kPrefetchTiles = MLA_PAIR_PREFETCH_TILES;
+constexpr int kVStages = 3;          // value ring: three stages
 constexpr int kThreads = 288;  // 9 warps; the softmax warps 4-7 own TMEM lanes 0-127
 constexpr int kTmemCols = 512;
-constexpr int kTmS = 0;          // two S buffers of 64 columns
-constexpr int kTmO = 128;        // O: 256 columns
+constexpr int kTmS = 0;          // two S buffers (tile parity), each lo and hi halves of 64 columns
+constexpr int kTmO = 256;        // O: 256 columns (after the two S buffers of 128)
 
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQBoxes * kBox;
-constexpr int kOffV = kOffK + kKStages * kKStage;
+constexpr int kOffV = kOffK + kKTile;
 constexpr int kOffP = kOffV + kVStages * kVStage;
-constexpr int kOffBar = kOffP + 2 * kBox;
+constexpr int kOffBar = kOffP + 4 * kBox;  // two P buffers (tile parity) of 2 boxes
 
 enum Bar {
-    B_QFULL = 0, B_QEMPTY, B_SFULL0, B_SFULL1, B_SEMPTY0, B_SEMPTY1, B_PFULL, B_PVDONE, B_OEMPTY, B_PATCH, B_XCHG,
-    // key-full barriers come in two sets, for even and odd tiles (one per score issuer)
-    B_KFULL0, B_KEMPTY0 = B_KFULL0 + 2 * kKStages, B_VFULL0 = B_KEMPTY0 + kKStages, B_VEMPTY0 = B_VFULL0 + kVStages,
+    B_QFULL = 0, B_QEMPTY, B_SFULL0, B_SFULL1, B_SEMPTY0, B_SEMPTY1, B_PFULL0, B_PFULL1, B_PVDONE0, B_PVDONE1,
+    B_OEMPTY, B_PATCH, B_XCHG,
+    B_KFULL0, B_KEMPTY0 = B_KFULL0 + kKStages, B_VFULL0 = B_KEMPTY0 + kKStages, B_VEMPTY0 = B_VFULL0 + kVStages,
     B_COUNT = B_VEMPTY0 + kVStages
 };
 constexpr int kOffRed = kOffBar + 8 * 64;          // exchange buffer [2][128] floats
 constexpr int kOffMisc = kOffRed + 2 * 128 * 4;    // abort flag, TMEM base
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;   // + slack to align the base to 1 KB
 static_assert(B_COUNT <= 64, "barrier area");
-static_assert(kKStages == kKPerTile, "the score issuers assume a key ring of exactly one tile");
+static_assert(kTmS + 2 * 128 <= kTmO && kTmO + 256 <= kTmemCols, "tensor memory map: S buffers, then O");
+static_assert(kstage_first_block(kKStages - 1) + kstage_blocks(kKStages - 1) == kQBoxes, "key stages cover a page");
 
 struct Params {
     const PlanHeader* hdr;
@@ -91,8 +96,7 @@ struct Params {
     const int32_t* part_offsets;
     const int32_t* context_lens;
     const int32_t* block_table;
-    const uint16_t* pool;  // [num_blocks * block_size, 576], for the L2 prefetch
-    float* o_part;  // [n_parts, 128, 512]
+    uint16_t* o_part;  // [n_parts, 128, 512] bf16 (normalised partial outputs)
     float* lse_part;  // [n_parts, 128]
     int64_t num_blocks;
     int32_t batch, max_blocks_per_seq, block_size, q_len;
@@ -118,13 +122,14 @@ __device__ __forceinline__ void ring_next(uint32_t& stage, uint32_t& phase) {
     if (++stage == N) { stage = 0; phase ^= 1; }
 }
 
-// Queries and key stages; one thread (lane 0 of warp 0). tm_q and tm_k are
-// 3-D maps {64 columns, rows, 9 column blocks} with boxes {64, 64, 9} and
-// {64, 64, 3}: one TMA operation fills the whole query block or key stage.
-__device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUtensorMap* tm_k, const Ctx& c) {
-    uint32_t stage = 0, phase = 0;
+// Queries and key stages; one thread (lane 0 of warp 0). tm_q, tm_k3 and
+// tm_k2 are 3-D maps {64 columns, rows, 9 column blocks} with boxes
+// {64, 64, 9}, {64, 64, 3} and {64, 64, 2}: one TMA operation fills the whole
+// query block or a key stage.
+__device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUtensorMap* tm_k3,
+                             const CUtensorMap* tm_k2, const Ctx& c) {
+    uint32_t phase = 0;  // parity of the pair's running tile count
     int seg_i = 0;
-    uint32_t ktile = 0;  // running tile count of this pair
     SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
     Segment seg;
     while (it.next(seg)) {
@@ -136,18 +141,7 @@ __device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUt
             ptx::tma_load_3d_pair(c.sbase + kOffQ, tm_q, 0, g * kH + 64 * c.rank, 0, full);
         }
         const int n_tiles = tiles_of(seg);
-        // L2 prefetch of this CTA's page of tile jj (only pages that hold visible tokens)
-        auto prefetch_tile = [&](int jj) {
-            if (kPrefetchTiles <= 0 || jj >= n_tiles) return;
-            const int32_t t = seg.tok_begin + jj * kTile + 64 * static_cast<int32_t>(c.rank);
-            if (t >= seg.tok_end) return;
-            const int64_t row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks,
-                                            P.block_size, b, t);
-            if (row >= 0) ptx::prefetch_l2(P.pool + row * kD, 64 * kD * 2);
-        };
-        for (int jj = 1; jj <= kPrefetchTiles; ++jj) prefetch_tile(jj);
         for (int j = 0; j < n_tiles; ++j) {
-            if (j > 0) prefetch_tile(j + kPrefetchTiles);
             // this CTA's 64-token page of tile j, all 576 values
             const int32_t t0 = seg.tok_begin + j * kTile;
             int32_t th = t0 + 64 * static_cast<int32_t>(c.rank);
@@ -158,15 +152,15 @@ __device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUt
                 record_status(MLA_ERR_DEVICE_FAULT);
                 row = 0;
             }
-            for (int ks = 0; ks < kKPerTile; ++ks) {
-                if (!ptx::mbar_wait(c.bar(B_KEMPTY0 + stage), phase ^ 1, c.abort)) return;
-                const uint32_t full = c.leader_bar(B_KFULL0 + (ktile & 1) * kKStages + stage);
-                ptx::mbar_arrive_expect_tx_cluster(full, kKStage);
-                ptx::tma_load_3d_pair(c.sbase + kOffK + stage * kKStage, tm_k, 0, static_cast<int32_t>(row), 3 * ks,
-                                      full);
-                ring_next<kKStages>(stage, phase);
+            for (int ks = 0; ks < kKStages; ++ks) {
+                if (!ptx::mbar_wait(c.bar(B_KEMPTY0 + ks), phase ^ 1, c.abort)) return;
+                const uint32_t full = c.leader_bar(B_KFULL0 + ks);
+                const int blk = kstage_first_block(ks);
+                ptx::mbar_arrive_expect_tx_cluster(full, kstage_blocks(ks) * kBox);
+                ptx::tma_load_3d_pair(c.sbase + kOffK + blk * kBox, ks == 0 ? tm_k3 : tm_k2, 0,
+                                      static_cast<int32_t>(row), blk, full);
             }
-            ++ktile;
+            phase ^= 1;
         }
         ++seg_i;
     }
@@ -174,10 +168,8 @@ __device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUt
     // block, so that no asynchronous arrival (a multicast tcgen05.commit) can
     // reach this CTA's shared memory after it exits -- it would land in the
     // barriers of whatever CTA runs here next.
-    for (int i = 0; i < kKStages; ++i) {
-        if (!ptx::mbar_wait(c.bar(B_KEMPTY0 + stage), phase ^ 1, c.abort)) return;
-        ring_next<kKStages>(stage, phase);
-    }
+    for (int ks = 0; ks < kKStages; ++ks)
+        if (!ptx::mbar_wait(c.bar(B_KEMPTY0 + ks), phase ^ 1, c.abort)) return;
     if (seg_i > 0) ptx::mbar_wait(c.bar(B_QEMPTY), (seg_i - 1) & 1, c.abort);
 }
 
@@ -253,8 +245,9 @@ __device__ void value_producer(const Params& P, const CUtensorMap* tm_v, const C
 }
 
 // ------------------------------------------------------------------- MMA
-// Three issuing threads in the leader CTA: two for the score MMAs (even and
-// odd tiles, one S buffer each) and one for the value MMAs. A single thread
+// Three issuing threads in the leader CTA: two for the score MMAs (one per
+// half of the contraction, each with its own half-accumulator) and one for the
+// value MMAs. A single thread
 // issues at most about one tcgen05.mma every ~47 cycles, while an
 // M 128 x N 128 x K 16 pair instruction takes the tensor cores 32 cycles, and
 // the three streams are independent (different TMEM accumulators, operands
@@ -269,19 +262,14 @@ struct Descs {
           dv(ptx::smem_desc_sw128(c.sbase + kOffV, kBox / 2, 1024)) {}
 };
 
-// S = Q K^T for the tiles of one parity (the pair's running tile count t,
-// t % 2 == parity) into S buffer `parity`; one thread per parity (lane 0 of
-// warp 1 and of warp 3 of the leader CTA). The key ring holds one tile; the
-// producer signals the fill of stage ks for tile t on the key-full barrier
-// of t's parity, so tile t = 2m + parity is phase m of that barrier. A
-// parity wait can only tell apart adjacent phases; here the barrier is never
-// two phases ahead of its waiter, since the fill for tile t + 2 needs this
-// thread's own MMAs of tile t to have released the stage (a single barrier
-// set for both threads would let the odd thread see phase -1 as complete).
-// Both threads commit QEMPTY once per segment (the barrier counts 2), after
-// waiting for the segment's query block, so that a thread without tiles in
-// a segment cannot arrive twice on one phase.
-__device__ void mma_s_issuer(const Params& P, const Ctx& c, uint32_t parity) {
+// Partial scores S_half = Q[:, blocks] K[:, blocks]^T of every tile, into the
+// half-accumulator `half` of S buffer (tile & 1); one thread per half (lane 0
+// of warp 1: blocks 0-4, key stages 0-1; lane 0 of warp 3: blocks 5-8, key
+// stages 2-3), so that the two threads issue the 36 score instructions of a
+// tile concurrently. Each key stage is consumed by one thread only, once per
+// tile (phase = tile parity). Both threads commit QEMPTY once per segment (the
+// barrier counts 2) and SFULL once per tile (it counts 2).
+__device__ void mma_s_issuer(const Params& P, const Ctx& c, uint32_t half) {
     constexpr uint32_t kIdS = ptx::idesc_bf16(128, 128, false, false);
     const Descs D(c);
     uint32_t tile_cnt = 0;
@@ -293,26 +281,24 @@ __device__ void mma_s_issuer(const Params& P, const Ctx& c, uint32_t parity) {
         ptx::tc_fence_after();
         const int n_tiles = tiles_of(seg);
         for (int j = 0; j < n_tiles; ++j, ++tile_cnt) {
-            if ((tile_cnt & 1) != parity) continue;
-            const uint32_t d_s = c.tmem + kTmS + 64 * parity;
-            const uint32_t kph = (tile_cnt >> 1) & 1;  // phase of this parity's key-full barriers
-            if (!ptx::mbar_wait(c.bar(B_SEMPTY0 + parity), ((tile_cnt >> 1) & 1) ^ 1, c.abort)) return;
+            const uint32_t sb = tile_cnt & 1;
+            const uint32_t d_s = c.tmem + kTmS + 128 * sb + 64 * half;
+            if (!ptx::mbar_wait(c.bar(B_SEMPTY0 + sb), ((tile_cnt >> 1) & 1) ^ 1, c.abort)) return;
 #pragma unroll 1
-            for (int ks = 0; ks < kKPerTile; ++ks) {
-                if (!ptx::mbar_wait(c.bar(B_KFULL0 + parity * kKStages + ks), kph, c.abort)) return;
+            for (int ks = 2 * static_cast<int>(half); ks < 2 * static_cast<int>(half) + 2; ++ks) {
+                if (!ptx::mbar_wait(c.bar(B_KFULL0 + ks), tile_cnt & 1, c.abort)) return;
                 ptx::tc_fence_after();
-#pragma unroll
-                for (int bx = 0; bx < 3; ++bx) {
-                    const int k = 3 * ks + bx;
+                const int k_first = kstage_first_block(0 + 2 * static_cast<int>(half));
+                for (int k = kstage_first_block(ks); k < kstage_first_block(ks) + kstage_blocks(ks); ++k) {
                     const uint64_t a0 = D.dq + static_cast<uint64_t>((k * kBox) >> 4);
-                    const uint64_t b0 = D.dk + static_cast<uint64_t>((ks * kKStage + bx * kBox) >> 4);
+                    const uint64_t b0 = D.dk + static_cast<uint64_t>((k * kBox) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        ptx::mma_bf16_pair(d_s, a0 + 2 * kk, b0 + 2 * kk, kIdS, (k | kk) != 0);
+                        ptx::mma_bf16_pair(d_s, a0 + 2 * kk, b0 + 2 * kk, kIdS, (k != k_first) || (kk != 0));
                 }
                 ptx::mma_commit_pair(c.bar(B_KEMPTY0 + ks), 0x3);
             }
-            ptx::mma_commit_pair(c.bar(B_SFULL0 + parity), 0x3);
+            ptx::mma_commit_pair(c.bar(B_SFULL0 + sb), 0x3);
         }
         ptx::mma_commit_pair(c.bar(B_QEMPTY), 0x3);
         ++seg_i;
@@ -331,7 +317,8 @@ __device__ void mma_pv_issuer(const Params& P, const Ctx& c) {
         const int n_tiles = tiles_of(seg);
         for (int j = 0; j < n_tiles; ++j) {
             const bool first = (j == 0);
-            if (!ptx::mbar_wait(c.bar(B_PFULL), pv_cnt & 1, c.abort)) return;
+            const uint32_t pb = pv_cnt & 1;  // P buffer of this tile
+            if (!ptx::mbar_wait(c.bar(B_PFULL0 + pb), (pv_cnt >> 1) & 1, c.abort)) return;
             if (first && !ptx::mbar_wait(c.bar(B_OEMPTY), (seg_i & 1) ^ 1, c.abort)) return;
             const int32_t tv = seg.tok_begin + j * kTile;
             for (int q = 0; q < kVPerTile; ++q) {
@@ -339,7 +326,7 @@ __device__ void mma_pv_issuer(const Params& P, const Ctx& c) {
                 if (!ptx::mbar_wait(c.bar(B_VFULL0 + vst), vph, c.abort)) return;
                 ptx::tc_fence_after();
                 // A: P tokens 32q + 16kk .. +15 (box q/2, byte 64 (q&1) + 32 kk of each 128-byte row)
-                const uint64_t a0 = D.dp + static_cast<uint64_t>(((q >> 1) * kBox + 64 * (q & 1)) >> 4);
+                const uint64_t a0 = D.dp + static_cast<uint64_t>(((2 * pb + (q >> 1)) * kBox + 64 * (q & 1)) >> 4);
                 const uint64_t b0 = D.dv + static_cast<uint64_t>((vst * kVStage) >> 4);
 #pragma unroll
                 for (int n = 0; n < 2; ++n)
@@ -351,7 +338,7 @@ __device__ void mma_pv_issuer(const Params& P, const Ctx& c) {
                 ptx::mma_commit_pair(c.bar(B_VEMPTY0 + vst), 0x3);
                 ring_next<kVStages>(vst, vph);
             }
-            ptx::mma_commit_pair(c.bar(B_PVDONE), 0x3);
+            ptx::mma_commit_pair(c.bar(B_PVDONE0 + pb), 0x3);
             ++pv_cnt;
         }
         ++seg_i;
@@ -383,16 +370,28 @@ __device__ void softmax(const Params& P, const Ctx& c) {
     const uint32_t tl = c.tmem + (static_cast<uint32_t>(t & ~31) << 16);  // this warp's lane quadrant
     const uint32_t sempty0 = c.leader_bar(B_SEMPTY0), sempty1 = c.leader_bar(B_SEMPTY1);
     const float scale_log2 = P.scale_log2;
-    const uint32_t pfull = c.leader_bar(B_PFULL), oempty = c.leader_bar(B_OEMPTY);
-    uint8_t* prow = c.smem + kOffP + half * kBox + hrow * 128;
+    const uint32_t pfull0 = c.leader_bar(B_PFULL0), pfull1 = c.leader_bar(B_PFULL1);
+    const uint32_t oempty = c.leader_bar(B_OEMPTY);
     Exchanger xc{reinterpret_cast<float*>(c.smem + kOffRed), c.bar(B_XCHG)};
-    uint32_t tile_cnt = 0, pv_wait = 0;
+    uint32_t tile_cnt = 0;
+    // Value MMAs of the pair's tile k signal PVDONE[k & 1] (phase k >> 1). pv_done is the
+    // highest k known complete (a completion implies every earlier one). Each wait is at
+    // most one phase behind its barrier: tile k + 2's value MMAs need the P this thread
+    // writes after the wait.
+    int32_t pv_done = -1;
+    auto wait_pv = [&](int32_t k) -> bool {
+        if (k <= pv_done) return true;
+        if (!ptx::mbar_wait(c.bar(B_PVDONE0 + (k & 1)), (static_cast<uint32_t>(k) >> 1) & 1, c.abort)) return false;
+        pv_done = k;
+        return true;
+    };
     SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
     Segment seg;
     while (it.next(seg)) {
         float m_run = -INFINITY, l_run = 0.f;
         const int n_tiles = tiles_of(seg);
         for (int j = 0; j < n_tiles; ++j) {
+            const int32_t tc = static_cast<int32_t>(tile_cnt);
             const uint32_t sb = tile_cnt & 1;
             if (!ptx::mbar_wait(c.bar(B_SFULL0 + sb), (tile_cnt >> 1) & 1, c.abort)) return;
             ptx::tc_fence_after();
@@ -400,9 +399,17 @@ __device__ void softmax(const Params& P, const Ctx& c) {
             {
                 float (&s0)[32] = *reinterpret_cast<float(*)[32]>(&s[0]);
                 float (&s1)[32] = *reinterpret_cast<float(*)[32]>(&s[32]);
-                ptx::tmem_ld32(tl + kTmS + 64 * sb, s0);
-                ptx::tmem_ld32(tl + kTmS + 64 * sb + 32, s1);
+                ptx::tmem_ld32(tl + kTmS + 128 * sb, s0);
+                ptx::tmem_ld32(tl + kTmS + 128 * sb + 32, s1);
                 ptx::tmem_wait_ld();
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {  // + the hi half-accumulator
+                    float u[32];
+                    ptx::tmem_ld32(tl + kTmS + 128 * sb + 64 + 32 * h2, u);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) s[32 * h2 + i] += u[i];
+                }
             }
             ptx::tc_fence_before();
             __syncwarp();
@@ -436,23 +443,24 @@ __device__ void softmax(const Params& P, const Ctx& c) {
                 ps[i & 3] += s[i];
             }
             l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-            if (j > 0) {  // PV of the previous tile must be done before P and O are touched
-                if (!ptx::mbar_wait(c.bar(B_PVDONE), pv_wait & 1, c.abort)) return;
-                ++pv_wait;
+            if (j > 0 && rescale) {  // O is rescaled once the previous tile's value MMAs are done
+                if (!wait_pv(tc - 1)) return;
                 ptx::tc_fence_after();
-                if (rescale) {
 #pragma unroll 1
-                    for (int cc = 0; cc < 8; ++cc) {
-                        float o[32];
-                        ptx::tmem_ld32(tl + kTmO + 32 * cc, o);
-                        ptx::tmem_wait_ld();
+                for (int cc = 0; cc < 8; ++cc) {
+                    float o[32];
+                    ptx::tmem_ld32(tl + kTmO + 32 * cc, o);
+                    ptx::tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                        ptx::tmem_st32(tl + kTmO + 32 * cc, o);
-                    }
-                    ptx::tmem_wait_st();
+                    for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                    ptx::tmem_st32(tl + kTmO + 32 * cc, o);
                 }
+                ptx::tmem_wait_st();
             }
+            // this tile's P buffer was last read by the value MMAs of tile tc - 2
+            if (tc >= 2 && !wait_pv(tc - 2)) return;
+            ptx::tc_fence_after();
+            uint8_t* const prow = c.smem + kOffP + (2 * sb + half) * kBox + hrow * 128;
             // P row (bf16) into the K-major 128B-swizzled A operand of the PV MMA
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8) {
@@ -466,41 +474,50 @@ __device__ void softmax(const Params& P, const Ctx& c) {
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive_cluster(pfull);
+            if (lane == 0) ptx::mbar_arrive_cluster(sb ? pfull1 : pfull0);
             m_run = m_use;
         }
         // segment epilogue: normalise O and write the partial
-        if (!ptx::mbar_wait(c.bar(B_PVDONE), pv_wait & 1, c.abort)) return;
-        ++pv_wait;
+        if (!wait_pv(static_cast<int32_t>(tile_cnt) - 1)) return;
         ptx::tc_fence_after();
         float lpart;
         if (!xc.swap(l_run, lpart, t, c.abort)) return;
         const float l_tot = l_run + lpart;
         const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
-        // O rows go out through the (now idle) P buffer: each thread writes its row's
-        // 32-column slice to shared memory (16-byte chunks XOR-swizzled by row), then
-        // the warp stores its 32 rows with 8 lanes per 128-byte row segment, so every
-        // global store instruction covers whole 128-byte lines.
-        float* const o_base = P.o_part + static_cast<int64_t>(seg.slot) * kH * kDc;
+        // O rows go out, rounded to bf16, through the (now idle) P buffers: each thread
+        // writes a 64-column slice of its row (128 bytes, 16-byte chunks XOR-swizzled
+        // by row) to shared memory, then the warp stores its 32 rows with 8 lanes per
+        // 128-byte row segment, so every global store instruction covers whole lines.
+        uint16_t* const o_base = P.o_part + static_cast<int64_t>(seg.slot) * kH * kDc;
         uint8_t* const stage_buf = c.smem + kOffP;
         const int wrow0 = t & ~31;  // first row (thread) of this warp
 #pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
-            float o[32];
-            ptx::tmem_ld32(tl + kTmO + 32 * cc, o);
-            ptx::tmem_wait_ld();
+        for (int cc = 0; cc < 4; ++cc) {
+            float o[64];
+            {
+                float (&o0)[32] = *reinterpret_cast<float(*)[32]>(&o[0]);
+                float (&o1)[32] = *reinterpret_cast<float(*)[32]>(&o[32]);
+                ptx::tmem_ld32(tl + kTmO + 64 * cc, o0);
+                ptx::tmem_ld32(tl + kTmO + 64 * cc + 32, o1);
+                ptx::tmem_wait_ld();
+            }
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                *reinterpret_cast<float4*>(stage_buf + t * 128 + ((k ^ (t & 7)) << 4)) =
-                    make_float4(o[4 * k] * inv, o[4 * k + 1] * inv, o[4 * k + 2] * inv, o[4 * k + 3] * inv);
+            for (int k = 0; k < 8; ++k) {
+                uint4 u;
+                u.x = ptx::bf16x2(o[8 * k + 0] * inv, o[8 * k + 1] * inv);
+                u.y = ptx::bf16x2(o[8 * k + 2] * inv, o[8 * k + 3] * inv);
+                u.z = ptx::bf16x2(o[8 * k + 4] * inv, o[8 * k + 5] * inv);
+                u.w = ptx::bf16x2(o[8 * k + 6] * inv, o[8 * k + 7] * inv);
+                *reinterpret_cast<uint4*>(stage_buf + t * 128 + ((k ^ (t & 7)) << 4)) = u;
+            }
             __syncwarp();
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const int r = wrow0 + 4 * k + static_cast<int>(lane >> 3), ch = static_cast<int>(lane & 7);
-                const float4 v = *reinterpret_cast<const float4*>(stage_buf + r * 128 + ((ch ^ (r & 7)) << 4));
+                const uint4 v = *reinterpret_cast<const uint4*>(stage_buf + r * 128 + ((ch ^ (r & 7)) << 4));
                 const int r_head = 64 * static_cast<int>(c.rank) + (r & 63);
-                *reinterpret_cast<float4*>(o_base + static_cast<int64_t>(r_head) * kDc + 256 * (r >> 6) + 32 * cc +
-                                           4 * ch) = v;
+                *reinterpret_cast<uint4*>(o_base + static_cast<int64_t>(r_head) * kDc + 256 * (r >> 6) + 64 * cc +
+                                          8 * ch) = v;
             }
             __syncwarp();
         }
@@ -516,8 +533,9 @@ __device__ void softmax(const Params& P, const Ctx& c) {
 // ------------------------------------------------------------------ kernel
 // grid: 2 * workers CTAs (clusters of 2); block 256; dynamic smem kSmemBytes.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    pair_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const Params P) {
+    pair_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k3,
+                       const __grid_constant__ CUtensorMap tm_k2, const __grid_constant__ CUtensorMap tm_v,
+                       const Params P) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = ptx::smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -534,18 +552,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         *c.abort = 0;
         ptx::mbar_init(c.bar(B_QFULL), 2);
         ptx::mbar_init(c.bar(B_QEMPTY), 2);
-        ptx::mbar_init(c.bar(B_SFULL0), 1);
-        ptx::mbar_init(c.bar(B_SFULL1), 1);
+        ptx::mbar_init(c.bar(B_SFULL0), 2);
+        ptx::mbar_init(c.bar(B_SFULL1), 2);
         ptx::mbar_init(c.bar(B_SEMPTY0), 8);
         ptx::mbar_init(c.bar(B_SEMPTY1), 8);
-        ptx::mbar_init(c.bar(B_PFULL), 8);
-        ptx::mbar_init(c.bar(B_PVDONE), 1);
+        ptx::mbar_init(c.bar(B_PFULL0), 8);
+        ptx::mbar_init(c.bar(B_PFULL1), 8);
+        ptx::mbar_init(c.bar(B_PVDONE0), 1);
+        ptx::mbar_init(c.bar(B_PVDONE1), 1);
         ptx::mbar_init(c.bar(B_OEMPTY), 8);
         ptx::mbar_init(c.bar(B_PATCH), 1);
         ptx::mbar_init(c.bar(B_XCHG), 4);
         for (int s = 0; s < kKStages; ++s) {
             ptx::mbar_init(c.bar(B_KFULL0 + s), 2);
-            ptx::mbar_init(c.bar(B_KFULL0 + kKStages + s), 2);
             ptx::mbar_init(c.bar(B_KEMPTY0 + s), 1);
         }
         for (int s = 0; s < kVStages; ++s) {
@@ -556,7 +575,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     if (warp == 0 && ptx::lane_id() == 0) {
         ptx::prefetch_tmap(&tm_q);
-        ptx::prefetch_tmap(&tm_k);
+        ptx::prefetch_tmap(&tm_k3);
+        ptx::prefetch_tmap(&tm_k2);
         ptx::prefetch_tmap(&tm_v);
     }
     if (warp == 1) {
@@ -570,7 +590,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     c.tmem = *tmem_slot;
 
     if (warp == 0) {
-        if (ptx::lane_id() == 0) key_producer(P, &tm_q, &tm_k, c);
+        if (ptx::lane_id() == 0) key_producer(P, &tm_q, &tm_k3, &tm_k2, c);
     } else if (warp == 2) {
         value_producer(P, &tm_v, c);
     } else if (warp == 1 || warp == 3) {

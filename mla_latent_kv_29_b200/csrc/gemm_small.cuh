@@ -2,8 +2,8 @@
 // sizes are multiples of the tile: see tc_gemm_dims_ok in the ABI):
 //   absorb:    Q[g, h, 0:d_c] = bf16(q_nope[g, h] W_UK[h]),  Q[g, h, d_c:] = q_pe[g, h]
 //              (query absorption, "MLA架构：低秩注意力机制优化LLM显存与计算效率" 3.1)
-//   merge:     the split-KV partials of (g, h) into bf16 o_lat (log-sum-exp weights)
-//   UV:        out[g, h] = bf16(W_UV[h] o_lat[g, h])
+//   merge+UV:  the split-KV partials of (g, h) merged into o_lat (log-sum-exp
+//              weights), then out[g, h] = bf16(W_UV[h] o_lat[g, h])
 //   append:    split-K partial sums of x . W_kva (kv_a_proj_with_mqa, 2.2)
 // Each loads its weight tile once per CTA and runs 16 x 64 warp tiles.
 #pragma once
@@ -71,63 +71,38 @@ __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(
     }
 }
 
-// ------------------------------------------------------------------ merge
-// Log-sum-exp merge of the split partials of (g, h) into o_lat[g, h] (bf16):
-// one warp per (group, head); lane l owns latent columns 4l + 128j .. +3.
-// grid (G, ceil(H / 8)); block 256.
-__global__ void __launch_bounds__(256) merge_bf16_kernel(
-    const float* __restrict__ o_part, const float* __restrict__ lse_part, const int32_t* __restrict__ part_offsets,
-    int32_t G, int32_t H, int32_t dc, uint16_t* __restrict__ o_lat) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = blockIdx.x, h = blockIdx.y * 8 + warp;
-    if (h >= H) return;
-    const int32_t p0 = part_offsets[g], p1 = part_offsets[g + 1];
-    float M = -INFINITY;
-    for (int32_t p = p0 + lane; p < p1; p += 32) M = fmaxf(M, lse_part[static_cast<int64_t>(p) * H + h]);
-    M = warp_max(M);
-    const int nj = dc / 128;  // float4 column groups per lane (4 for d_c = 512)
-    float4 acc[4] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f),
-                     make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-    float den = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll 2
-        for (int32_t p = p0; p < p1; ++p) {
-            const float l = lse_part[static_cast<int64_t>(p) * H + h];
-            const float w = l == -INFINITY ? 0.f : __expf(l - M);
-            den += w;
-            const float4* src = reinterpret_cast<const float4*>(o_part + (static_cast<int64_t>(p) * H + h) * dc) + lane;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                if (j < nj) {
-                    const float4 u = src[32 * j];
-                    acc[j].x = fmaf(w, u.x, acc[j].x); acc[j].y = fmaf(w, u.y, acc[j].y);
-                    acc[j].z = fmaf(w, u.z, acc[j].z); acc[j].w = fmaf(w, u.w, acc[j].w);
-                }
-            }
-        }
-    }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    uint16_t* dst = o_lat + (static_cast<int64_t>(g) * H + h) * dc + 4 * lane;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-        if (j < nj)
-            *reinterpret_cast<uint2*>(dst + 128 * j) =
-                make_uint2(pack_bf16x2(acc[j].x * inv, acc[j].y * inv), pack_bf16x2(acc[j].z * inv, acc[j].w * inv));
-}
-
-// ------------------------------------------------------------ up-projection
-// out[g, h, :] = bf16(W_UV[h] o_lat[g, h, :]); grid (H, ceil(G / 64)); block 256;
-// dynamic smem uv_tc_smem(dc, dv).
+// -------------------------------------------------- merge + up-projection
+// Log-sum-exp merge of the split partials fused with the value up-projection:
+//   o_lat[g, h] = sum_i w_i o_i / sum_i w_i,  w_i = exp(lse_i - max_i lse_i)
+//   out[g, h, :] = bf16(W_UV[h] o_lat[g, h])
+// Partial i of (g, h) is o_part[i, h, :] (PartT: float, or bf16 bits in
+// uint16_t), already divided by its own softmax denominator; parts with
+// lse = -inf weigh 0 and a group without a finite part gives zeros. o_lat is
+// rounded to bf16 in shared memory (the GEMM's A operand) while W_UV[h]
+// streams in. grid (H, ceil(G / 64)); block 256; dynamic smem uv_tc_smem(dc, dv).
 __host__ __device__ inline size_t uv_tc_smem(int dc, int dv) {
     return sizeof(uint16_t) * (static_cast<size_t>(kTcRows) + dv) * (dc + 8);
 }
 
-__global__ void __launch_bounds__(kTcThreads) uv_tc_kernel(const uint16_t* __restrict__ o_lat,
-                                                            const uint16_t* __restrict__ w_uv, int32_t G, int32_t H,
-                                                            int32_t dc, int32_t dv, uint16_t* __restrict__ out) {
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+    const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const uint16_t* p, float (&v)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xffff0000u);
+    v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xffff0000u);
+    v[4] = __uint_as_float(u.z << 16); v[5] = __uint_as_float(u.z & 0xffff0000u);
+    v[6] = __uint_as_float(u.w << 16); v[7] = __uint_as_float(u.w & 0xffff0000u);
+}
+
+template <typename PartT>
+__global__ void __launch_bounds__(kTcThreads) merge_uv_tc_kernel(
+    const PartT* __restrict__ o_part, const float* __restrict__ lse_part, const int32_t* __restrict__ part_offsets,
+    const uint16_t* __restrict__ w_uv, int32_t G, int32_t H, int32_t dc, int32_t dv, uint16_t* __restrict__ out) {
     extern __shared__ __align__(16) uint16_t sm_uv[];
     const int ld = dc + 8;
-    uint16_t* As = sm_uv;               // [64][dc + 8]  o_lat rows of head h
+    uint16_t* As = sm_uv;               // [64][dc + 8]  o_lat rows of head h (bf16)
     uint16_t* Bs = As + kTcRows * ld;   // [dv][dc + 8]  W_UV[h] (latent column contiguous)
     const int h = blockIdx.x, g0 = blockIdx.y * kTcRows;
     const int c8s = dc / 8;
@@ -135,23 +110,62 @@ __global__ void __launch_bounds__(kTcThreads) uv_tc_kernel(const uint16_t* __res
         const int n = i / c8s, c8 = (i % c8s) * 8;
         wmma16::cp_async16(Bs + n * ld + c8, w_uv + (static_cast<int64_t>(h) * dv + n) * dc + c8);
     }
-    for (int i = threadIdx.x; i < kTcRows * c8s; i += blockDim.x) {
-        const int r = i / c8s, c8 = (i % c8s) * 8, g = g0 + r;
-        if (g < G)
-            wmma16::cp_async16(As + r * ld + c8, o_lat + (static_cast<int64_t>(g) * H + h) * dc + c8);
-        else
-            *reinterpret_cast<uint4*>(As + r * ld + c8) = make_uint4(0u, 0u, 0u, 0u);
-    }
     wmma16::cp_async_commit();
-    wmma16::cp_async_wait<0>();
-    __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rows_used = min(kTcRows, G - g0);
+    // merge: one warp per group row; lane l owns columns 256 j + 8 l .. +7
+    constexpr int kMaxJ = 2;  // dc <= 512
+    for (int r = warp; r < kTcRows; r += kTcThreads / 32) {
+        uint16_t* dst = As + r * ld;
+        float acc[kMaxJ][8];
+#pragma unroll
+        for (int j = 0; j < kMaxJ; ++j)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+        float den = 0.f;
+        if (r < rows_used) {
+            const int32_t g = g0 + r;
+            const int32_t p0 = part_offsets[g], p1 = part_offsets[g + 1];
+            float M = -INFINITY;
+            for (int32_t p = p0 + lane; p < p1; p += 32) M = fmaxf(M, lse_part[static_cast<int64_t>(p) * H + h]);
+            M = warp_max(M);
+            if (M != -INFINITY) {
+#pragma unroll 4
+                for (int32_t p = p0; p < p1; ++p) {
+                    const float l = lse_part[static_cast<int64_t>(p) * H + h];
+                    const float w = l == -INFINITY ? 0.f : __expf(l - M);
+                    den += w;
+                    const PartT* src = o_part + (static_cast<int64_t>(p) * H + h) * dc;
+#pragma unroll
+                    for (int j = 0; j < kMaxJ; ++j) {
+                        const int col = 256 * j + 8 * lane;
+                        if (col < dc) {
+                            float v[8];
+                            load8(src + col, v);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) acc[j][e] = fmaf(w, v[e], acc[j][e]);
+                        }
+                    }
+                }
+            }
+        }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxJ; ++j) {
+            const int col = 256 * j + 8 * lane;
+            if (col < dc)
+                *reinterpret_cast<uint4*>(dst + col) =
+                    make_uint4(pack_bf16x2(acc[j][0] * inv, acc[j][1] * inv), pack_bf16x2(acc[j][2] * inv, acc[j][3] * inv),
+                               pack_bf16x2(acc[j][4] * inv, acc[j][5] * inv), pack_bf16x2(acc[j][6] * inv, acc[j][7] * inv));
+        }
+    }
+    wmma16::cp_async_wait<0>();
+    __syncthreads();
     for (int wt = warp; wt < 4 * (dv / 64); wt += kTcThreads / 32) {
         const int r0 = 16 * (wt & 3), c0 = 64 * (wt >> 2);
         if (r0 >= rows_used) continue;  // an all-zero row block
-        float acc[8][4] = {};
-        for (int k0 = 0; k0 < dc; k0 += 16) wmma16::warp_tile_k16<true>(acc, As, ld, r0, Bs, ld, c0, k0);
+        float accg[8][4] = {};
+        for (int k0 = 0; k0 < dc; k0 += 16) wmma16::warp_tile_k16<true>(accg, As, ld, r0, Bs, ld, c0, k0);
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
             const int col = c0 + 8 * nt + 2 * (lane & 3);
@@ -160,7 +174,7 @@ __global__ void __launch_bounds__(kTcThreads) uv_tc_kernel(const uint16_t* __res
                 const int g = g0 + r0 + (lane >> 2) + 8 * hf;
                 if (g < G)
                     *reinterpret_cast<uint32_t*>(out + (static_cast<int64_t>(g) * H + h) * dv + col) =
-                        pack_bf16x2(acc[nt][2 * hf], acc[nt][2 * hf + 1]);
+                        pack_bf16x2(accg[nt][2 * hf], accg[nt][2 * hf + 1]);
             }
         }
     }

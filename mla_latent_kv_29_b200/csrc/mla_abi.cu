@@ -343,11 +343,15 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     const int32_t G = batch * q_len;
     const int H = dims->num_heads, dc = dims->kv_lora_rank, dr = dims->rope_dim;
 
+    const bool tc = tc_gemm_dims_ok(dims) && aligned(q_nope, 16) && aligned(w_uk, 16) && aligned(w_uv, 16) &&
+                    aligned(out, 16);
+    // the tensor-core kernel writes bf16 partials, which only the tensor-core merge reads
+    if (L.kernel == kKernelPair && !tc) return MLA_ERR_INVALID_ARG;
+
     plan_kernel<<<1, 1024, 0, st>>>(context_lens, batch, q_len, L.tile, L.workers, hdr, tile_prefix, part_offsets,
                                     worker_group);
     if (int rc = launch_status()) return rc;
 
-    const bool tc = tc_gemm_dims_ok(dims) && aligned(q_nope, 16) && aligned(w_uk, 16) && aligned(w_uv, 16);
     if (tc) {
         const size_t smem = absorb_tc_smem(dims->qk_nope_dim);
         if (int rc = ensure_smem(absorb_tc_kernel, smem)) return rc;
@@ -364,10 +368,11 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     if (int rc = launch_status()) return rc;
 
     if (L.kernel == kKernelPair) {
-        CUtensorMap tm_q, tm_k, tm_v;
+        CUtensorMap tm_q, tm_k3, tm_k2, tm_v;
         const uint64_t pool_rows = static_cast<uint64_t>(num_blocks) * dims->block_size;
         if (int rc = encode_row_blocks(&tm_q, q, pair::kD, static_cast<uint64_t>(G) * H, 64, pair::kQBoxes)) return rc;
-        if (int rc = encode_row_blocks(&tm_k, pool, pair::kD, pool_rows, 64, 3)) return rc;
+        if (int rc = encode_row_blocks(&tm_k3, pool, pair::kD, pool_rows, 64, 3)) return rc;
+        if (int rc = encode_row_blocks(&tm_k2, pool, pair::kD, pool_rows, 64, 2)) return rc;
         if (int rc = encode_row_blocks(&tm_v, pool, pair::kD, pool_rows, 32, 4)) return rc;
         pair::Params PP;
         PP.hdr = hdr;
@@ -376,8 +381,7 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         PP.part_offsets = part_offsets;
         PP.context_lens = context_lens;
         PP.block_table = block_table;
-        PP.pool = static_cast<const uint16_t*>(pool);
-        PP.o_part = o_part;
+        PP.o_part = reinterpret_cast<uint16_t*>(o_part);  // bf16 partials (the slot layout keeps fp32 size)
         PP.lse_part = lse_part;
         PP.num_blocks = num_blocks;
         PP.batch = batch;
@@ -387,7 +391,7 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         PP.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
         if (int rc = ensure_smem(pair::pair_decode_kernel, pair::kSmemBytes)) return rc;
         record_hook(opts ? opts->event_attn_begin : nullptr, st);
-        pair::pair_decode_kernel<<<2 * L.workers, pair::kThreads, pair::kSmemBytes, st>>>(tm_q, tm_k, tm_v, PP);
+        pair::pair_decode_kernel<<<2 * L.workers, pair::kThreads, pair::kSmemBytes, st>>>(tm_q, tm_k3, tm_k2, tm_v, PP);
         if (int rc = launch_status()) return rc;
         record_hook(opts ? opts->event_attn_end : nullptr, st);
     } else {
@@ -420,14 +424,19 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     }
 
     if (tc) {
-        // the absorbed queries are dead once the attention kernel is done: o_lat (bf16) reuses them
-        uint16_t* o_lat = q;
-        merge_bf16_kernel<<<dim3(G, (H + 7) / 8), 256, 0, st>>>(o_part, lse_part, part_offsets, G, H, dc, o_lat);
-        if (int rc = launch_status()) return rc;
         const size_t smem = uv_tc_smem(dc, dims->v_head_dim);
-        if (int rc = ensure_smem(uv_tc_kernel, smem)) return rc;
-        uv_tc_kernel<<<dim3(H, (G + kTcRows - 1) / kTcRows), kTcThreads, smem, st>>>(
-            o_lat, static_cast<const uint16_t*>(w_uv), G, H, dc, dims->v_head_dim, static_cast<uint16_t*>(out));
+        const dim3 grid(H, (G + kTcRows - 1) / kTcRows);
+        uint16_t* o = static_cast<uint16_t*>(out);
+        const uint16_t* wv = static_cast<const uint16_t*>(w_uv);
+        if (L.kernel == kKernelPair) {  // bf16 partials
+            if (int rc = ensure_smem(merge_uv_tc_kernel<uint16_t>, smem)) return rc;
+            merge_uv_tc_kernel<uint16_t><<<grid, kTcThreads, smem, st>>>(
+                reinterpret_cast<const uint16_t*>(o_part), lse_part, part_offsets, wv, G, H, dc, dims->v_head_dim, o);
+        } else {
+            if (int rc = ensure_smem(merge_uv_tc_kernel<float>, smem)) return rc;
+            merge_uv_tc_kernel<float><<<grid, kTcThreads, smem, st>>>(o_part, lse_part, part_offsets, wv, G, H, dc,
+                                                                     dims->v_head_dim, o);
+        }
     } else {
         const size_t uv_smem = sizeof(float) * kUvGroups * dc;
         if (int rc = ensure_smem(combine_uv_kernel, uv_smem)) return rc;
