@@ -19,6 +19,8 @@ __global__ void __launch_bounds__(kAbsorbThreads) absorb_q_kernel(
     const uint16_t* __restrict__ q_nope, const uint16_t* __restrict__ q_pe,
     const uint16_t* __restrict__ w_uk, uint16_t* __restrict__ q_out,
     int32_t G, int32_t H, int32_t dn, int32_t dc, int32_t dr) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ float qn[];  // [kAbsorbGroups][dn]
     const int h = blockIdx.x;
     const int g0 = blockIdx.y * kAbsorbGroups;

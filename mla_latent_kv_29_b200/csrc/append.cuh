@@ -21,6 +21,8 @@ constexpr int kApTileT = 64, kApTileN = 64, kApTileK = 32;
 __global__ void __launch_bounds__(256) append_gemm_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ w, float* __restrict__ part,
     int32_t T, int32_t K, int32_t N, int32_t k_per_split) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float xs[kApTileK][kApTileT + 4];  // k-major so the inner loop reads rows
     __shared__ float ws[kApTileK][kApTileN + 4];
     const int n0 = blockIdx.x * kApTileN, t0 = blockIdx.y * kApTileT;
@@ -82,22 +84,37 @@ struct AppendEpilogueParams {
 
 // grid (T); block 256; dynamic smem (dc + dr) floats.
 __global__ void __launch_bounds__(256) append_epilogue_kernel(AppendEpilogueParams P) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ float kv[];
     __shared__ float red[32];
     const int t = blockIdx.x;
     const int N = P.dc + P.dr;
     const int64_t split_stride = static_cast<int64_t>(P.T) * N;
-    for (int n = threadIdx.x; n < N; n += blockDim.x) {
-        // independent loads of all splits first, then the sum
-        const float* src = P.part + static_cast<int64_t>(t) * N + n;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        int k = 0;
-        for (; k + 8 <= P.splits; k += 8) {
+    // kv[n] = sum over splits; each thread owns columns threadIdx.x + 256 i (i < 3 for
+    // N = 576) and loads four splits of all its columns before summing them, so the
+    // loads of a thread are independent and few memory round trips are exposed.
+    constexpr int kCols = 4;  // N <= 1024
+    float acc[kCols] = {0.f, 0.f, 0.f, 0.f};
+    const float* src = P.part + static_cast<int64_t>(t) * N + threadIdx.x;
+    for (int k0 = 0; k0 < P.splits; k0 += 4) {
+        float v[4][kCols];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) acc[u] += __ldg(src + (k + u) * split_stride);
-        }
-        for (; k < P.splits; ++k) acc[0] += __ldg(src + k * split_stride);
-        kv[n] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int i = 0; i < kCols; ++i) {
+                const int n = static_cast<int>(threadIdx.x) + 256 * i;
+                v[u][i] = (k0 + u < P.splits && n < N) ? __ldg(src + (k0 + u) * split_stride + 256 * i) : 0.f;
+            }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int i = 0; i < kCols; ++i) acc[i] += v[u][i];
+    }
+#pragma unroll
+    for (int i = 0; i < kCols; ++i) {
+        const int n = static_cast<int>(threadIdx.x) + 256 * i;
+        if (n < N) kv[n] = acc[i];
     }
     __syncthreads();
     // RMSNorm over the latent part
@@ -146,6 +163,8 @@ __global__ void __launch_bounds__(256) append_epilogue_kernel(AppendEpiloguePara
 __global__ void resolve_slots_kernel(const int32_t* __restrict__ block_table, int32_t num_seqs, int32_t max_blocks_per_seq,
                                      int64_t num_blocks, int32_t block_size, const int32_t* __restrict__ seq_ids,
                                      const int32_t* __restrict__ positions, int32_t n, int64_t* __restrict__ rows) {
+    pdl_wait();
+    pdl_trigger();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) rows[i] = resolve_row(block_table, num_seqs, max_blocks_per_seq, num_blocks, block_size, seq_ids[i], positions[i]);
 }

@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(128) combine_kernel(
     const float* __restrict__ o_part, const float* __restrict__ lse_part,
     const int32_t* __restrict__ part_offsets, int32_t G, int32_t H, int32_t dc,
     float* __restrict__ o_lat, float* __restrict__ lse_out) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t gh = blockIdx.x;
     const int32_t g = static_cast<int32_t>(gh / H), h = static_cast<int32_t>(gh - static_cast<int64_t>(g) * H);
     const int32_t p0 = part_offsets[g], p1 = part_offsets[g + 1];
@@ -59,6 +61,8 @@ __global__ void __launch_bounds__(kUvThreads) combine_uv_kernel(
     const float* __restrict__ o_part, const float* __restrict__ lse_part,
     const int32_t* __restrict__ part_offsets, const uint16_t* __restrict__ w_uv,
     int32_t G, int32_t H, int32_t dc, int32_t dv, uint16_t* __restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ float ol[];  // [kUvGroups][dc]
     __shared__ float s_w[kUvGroups][kMaxMergeParts];
     __shared__ float s_inv[kUvGroups];

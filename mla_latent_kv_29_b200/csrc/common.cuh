@@ -46,6 +46,16 @@ __device__ __forceinline__ int64_t resolve_row(const int32_t* __restrict__ block
     return static_cast<int64_t>(blk) * block_size + (t - page * block_size);
 }
 
+// Programmatic dependent launch: every kernel of the library is launched
+// with programmatic stream serialization, so the next kernel in the stream may
+// start (launch, set up shared memory, barriers and tensor memory) while this
+// one finishes. pdl_wait() blocks until the preceding grid has completed and
+// its memory is visible; every kernel calls it before its first global access
+// of data another kernel produces or consumes (so the chain of waits also
+// orders it after all earlier work). pdl_trigger() lets the next kernel launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

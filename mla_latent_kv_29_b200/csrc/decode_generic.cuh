@@ -42,6 +42,8 @@ __host__ __device__ inline size_t generic_decode_smem(int dc, int dr) {
 }
 
 __global__ void __launch_bounds__(kGenThreads) generic_decode_kernel(GenericDecodeParams P) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ float sm[];
     const int D = P.dc + P.dr, Dp = D + 1;
     float* sq = sm;                              // [kGenHeads][Dp]

@@ -588,6 +588,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     ptx::cluster_sync();  // the peer's barriers exist before anyone arrives on them
     ptx::tc_fence_after();
     c.tmem = *tmem_slot;
+    pdl_wait();  // the schedule and the absorbed queries come from the preceding kernels
+    pdl_trigger();
 
     if (warp == 0) {
         if (ptx::lane_id() == 0) key_producer(P, &tm_q, &tm_k3, &tm_k2, c);

@@ -26,6 +26,8 @@ __host__ __device__ inline size_t absorb_tc_smem(int dn) {
 __global__ void __launch_bounds__(kTcThreads) absorb_tc_kernel(
     const uint16_t* __restrict__ q_nope, const uint16_t* __restrict__ q_pe, const uint16_t* __restrict__ w_uk,
     uint16_t* __restrict__ q_out, int32_t G, int32_t H, int32_t dn, int32_t dc, int32_t dr) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ __align__(16) uint16_t sm_abs[];
     const int lda = dn + 8, ldb = 128 + 8;
     uint16_t* As = sm_abs;                   // [64][dn + 8]   q_nope rows
@@ -100,6 +102,8 @@ template <typename PartT>
 __global__ void __launch_bounds__(kTcThreads) merge_uv_tc_kernel(
     const PartT* __restrict__ o_part, const float* __restrict__ lse_part, const int32_t* __restrict__ part_offsets,
     const uint16_t* __restrict__ w_uv, int32_t G, int32_t H, int32_t dc, int32_t dv, uint16_t* __restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ __align__(16) uint16_t sm_uv[];
     const int ld = dc + 8;
     uint16_t* As = sm_uv;               // [64][dc + 8]  o_lat rows of head h (bf16)
@@ -190,6 +194,8 @@ constexpr int kApTcLd = kApTc + 8;
 __global__ void __launch_bounds__(128) append_gemm_tc_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ w, float* __restrict__ part,
     int32_t T, int32_t K, int32_t N, int32_t k_per_split) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ __align__(16) uint16_t As[2][kApTc * kApTcLd];  // [t][k]
     __shared__ __align__(16) uint16_t Bs[2][kApTc * kApTcLd];  // [k][n]
     const int n0 = blockIdx.x * kApTc, t0 = blockIdx.y * kApTc;

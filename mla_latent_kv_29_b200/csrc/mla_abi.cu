@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "mla_b200.h"
 #include "common.cuh"
@@ -15,6 +16,7 @@
 #include "append.cuh"
 #include "decode_pair.cuh"
 #include "gemm_small.cuh"
+#include "gemm_tc05.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -55,6 +57,27 @@ int device_ok() {
     const int ok = major == 10 ? 1 : 2;
     if (dev >= 0 && dev < 64) cached[dev] = ok;
     return ok == 1 ? MLA_OK : MLA_ERR_NO_DEVICE;
+}
+
+// Launches `kernel` on `st` with programmatic stream serialization (the
+// kernels call pdl_wait() before touching data of earlier work, see common.cuh).
+template <typename... KArgs, typename... Args>
+int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    return MLA_OK;
 }
 
 int launch_status() {
@@ -131,6 +154,30 @@ int encode_row_blocks(CUtensorMap* m, const void* base, uint64_t cols, uint64_t 
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// 2-D bf16 tensor map over a row-major matrix [rows, cols] (row stride `cols`
+// * 2 bytes), box = {64 columns, box_rows rows}, 128-byte swizzle; rows past
+// the end are zero-filled.
+int encode_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return MLA_ERR_CUDA;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// The tcgen05 absorb / merge / UV kernels: d_n a multiple of 64 up to 256, d_c
+// a multiple of 256 up to 512, d_r a multiple of 8, d_v a multiple of 16 up
+// to 256, and 16-byte aligned operands.
+bool tc05_dims_ok(const mla_dims_t* d) {
+    return d->qk_nope_dim % 64 == 0 && d->qk_nope_dim <= 256 && d->kv_lora_rank % 256 == 0 &&
+           d->kv_lora_rank <= 512 && d->rope_dim % 8 == 0 && d->v_head_dim % 16 == 0 && d->v_head_dim <= 256;
 }
 
 int decode_layout(const mla_dims_t* d, int32_t batch, int32_t q_len, int32_t max_len,
@@ -259,6 +306,7 @@ int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32
     if (!(rms_eps >= 0.f) || !(rope_base > 0.f)) return MLA_ERR_INVALID_ARG;
     if (!aligned(workspace, kAlign) || !aligned(pool, 16)) return MLA_ERR_INVALID_ARG;
     if (workspace_bytes < mla_append_workspace_size(dims, n_tokens, hidden)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+    if (dims->kv_lora_rank + dims->rope_dim > 1024) return MLA_ERR_UNSUPPORTED_DIMS;  // epilogue: 4 columns per thread
     if (int rc = device_ok()) return rc;
     const int N = dims->kv_lora_rank + dims->rope_dim;
     const AppendPlan ap = append_plan(n_tokens, hidden, N);
@@ -268,13 +316,13 @@ int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32
     if (ap.tc) {
         if (!aligned(x, 16) || !aligned(w_kva, 16)) return MLA_ERR_INVALID_ARG;
         dim3 g1(N / kApTc, (n_tokens + kApTc - 1) / kApTc, splits);
-        append_gemm_tc_kernel<<<g1, 128, 0, st>>>(static_cast<const uint16_t*>(x),
+        if (int rc = launch(append_gemm_tc_kernel, g1, 128, 0, st, static_cast<const uint16_t*>(x),
                                                   static_cast<const uint16_t*>(w_kva), part, n_tokens, hidden, N,
-                                                  ap.k_per_split);
+                                                  ap.k_per_split)) return rc;
     } else {
         dim3 g1((N + kApTileN - 1) / kApTileN, (n_tokens + kApTileT - 1) / kApTileT, splits);
-        append_gemm_kernel<<<g1, 256, 0, st>>>(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w_kva),
-                                               part, n_tokens, hidden, N, ap.k_per_split);
+        if (int rc = launch(append_gemm_kernel, g1, 256, 0, st, static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w_kva),
+                                               part, n_tokens, hidden, N, ap.k_per_split)) return rc;
     }
     if (int rc = launch_status()) return rc;
     AppendEpilogueParams P;
@@ -294,7 +342,7 @@ int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32
     P.block_size = dims->block_size;
     P.eps = rms_eps;
     P.rope_base = rope_base;
-    append_epilogue_kernel<<<n_tokens, 256, sizeof(float) * N, st>>>(P);
+    if (int rc = launch(append_epilogue_kernel, n_tokens, 256, sizeof(float) * N, st, P)) return rc;
     return launch_status();
 }
 
@@ -348,22 +396,32 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     // the tensor-core kernel writes bf16 partials, which only the tensor-core merge reads
     if (L.kernel == kKernelPair && !tc) return MLA_ERR_INVALID_ARG;
 
-    plan_kernel<<<1, 1024, 0, st>>>(context_lens, batch, q_len, L.tile, L.workers, hdr, tile_prefix, part_offsets,
-                                    worker_group);
+    if (int rc = launch(plan_kernel, 1, 1024, 0, st, context_lens, batch, q_len, L.tile, L.workers, hdr, tile_prefix, part_offsets,
+                                    worker_group)) return rc;
     if (int rc = launch_status()) return rc;
 
-    if (tc) {
+    const bool tc05 = tc && tc05_dims_ok(dims) && aligned(q_pe, 16);
+    if (tc05) {
+        CUtensorMap tm_qn, tm_wuk;
+        if (int rc = encode_2d(&tm_qn, q_nope, static_cast<uint64_t>(H) * dims->qk_nope_dim, G, tc05::kRows)) return rc;
+        if (int rc = encode_2d(&tm_wuk, w_uk, dc, static_cast<uint64_t>(H) * dims->qk_nope_dim, dims->qk_nope_dim))
+            return rc;
+        const size_t smem = tc05::absorb_smem(dims->qk_nope_dim, dc);
+        if (int rc = ensure_smem(tc05::absorb_kernel, smem)) return rc;
+        if (int rc = launch(tc05::absorb_kernel, dim3(H, (G + tc05::kRows - 1) / tc05::kRows), tc05::kThreads, smem, st,
+            tm_qn, tm_wuk, static_cast<const uint16_t*>(q_pe), G, H, dims->qk_nope_dim, dc, dr, q)) return rc;
+    } else if (tc) {
         const size_t smem = absorb_tc_smem(dims->qk_nope_dim);
         if (int rc = ensure_smem(absorb_tc_kernel, smem)) return rc;
-        absorb_tc_kernel<<<dim3(H, dc / 128, (G + kTcRows - 1) / kTcRows), kTcThreads, smem, st>>>(
+        if (int rc = launch(absorb_tc_kernel, dim3(H, dc / 128, (G + kTcRows - 1) / kTcRows), kTcThreads, smem, st,
             static_cast<const uint16_t*>(q_nope), static_cast<const uint16_t*>(q_pe),
-            static_cast<const uint16_t*>(w_uk), q, G, H, dims->qk_nope_dim, dc, dr);
+            static_cast<const uint16_t*>(w_uk), q, G, H, dims->qk_nope_dim, dc, dr)) return rc;
     } else {
         const size_t absorb_smem = sizeof(float) * kAbsorbGroups * dims->qk_nope_dim;
         if (int rc = ensure_smem(absorb_q_kernel, absorb_smem)) return rc;
-        absorb_q_kernel<<<dim3(H, (G + kAbsorbGroups - 1) / kAbsorbGroups), kAbsorbThreads, absorb_smem, st>>>(
+        if (int rc = launch(absorb_q_kernel, dim3(H, (G + kAbsorbGroups - 1) / kAbsorbGroups), kAbsorbThreads, absorb_smem, st,
             static_cast<const uint16_t*>(q_nope), static_cast<const uint16_t*>(q_pe),
-            static_cast<const uint16_t*>(w_uk), q, G, H, dims->qk_nope_dim, dc, dr);
+            static_cast<const uint16_t*>(w_uk), q, G, H, dims->qk_nope_dim, dc, dr)) return rc;
     }
     if (int rc = launch_status()) return rc;
 
@@ -391,7 +449,7 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         PP.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
         if (int rc = ensure_smem(pair::pair_decode_kernel, pair::kSmemBytes)) return rc;
         record_hook(opts ? opts->event_attn_begin : nullptr, st);
-        pair::pair_decode_kernel<<<2 * L.workers, pair::kThreads, pair::kSmemBytes, st>>>(tm_q, tm_k3, tm_k2, tm_v, PP);
+        if (int rc = launch(pair::pair_decode_kernel, 2 * L.workers, pair::kThreads, pair::kSmemBytes, st, tm_q, tm_k3, tm_k2, tm_v, PP)) return rc;
         if (int rc = launch_status()) return rc;
         record_hook(opts ? opts->event_attn_end : nullptr, st);
     } else {
@@ -418,31 +476,54 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     const size_t gsmem = generic_decode_smem(dc, dr);
     if (int rc = ensure_smem(generic_decode_kernel, gsmem)) return rc;
     record_hook(opts ? opts->event_attn_begin : nullptr, st);
-    generic_decode_kernel<<<dim3(L.workers, (H + kGenHeads - 1) / kGenHeads), kGenThreads, gsmem, st>>>(P);
+    if (int rc = launch(generic_decode_kernel, dim3(L.workers, (H + kGenHeads - 1) / kGenHeads), kGenThreads, gsmem, st, P)) return rc;
     if (int rc = launch_status()) return rc;
     record_hook(opts ? opts->event_attn_end : nullptr, st);
     }
 
-    if (tc) {
+    if (tc05) {
+        // merge into bf16 o_lat (the absorbed queries are dead once the attention is done:
+        // o_lat reuses their space), then the up-projection
+        uint16_t* o_lat = q;
+        const dim3 mgrid(G, (H + 3) / 4);
+        if (L.kernel == kKernelPair) {
+            if (int rc = launch(tc05::merge_kernel<uint16_t>, mgrid, 128, 0, st,
+                                reinterpret_cast<const uint16_t*>(o_part), lse_part, part_offsets, G, H, dc, o_lat))
+                return rc;
+        } else {
+            if (int rc = launch(tc05::merge_kernel<float>, mgrid, 128, 0, st, o_part, lse_part, part_offsets, G, H, dc,
+                                o_lat))
+                return rc;
+        }
+        if (int rc = launch_status()) return rc;
+        CUtensorMap tm_ol, tm_wuv;
+        if (int rc = encode_2d(&tm_ol, o_lat, static_cast<uint64_t>(H) * dc, G, tc05::kRows)) return rc;
+        if (int rc = encode_2d(&tm_wuv, w_uv, dc, static_cast<uint64_t>(H) * dims->v_head_dim, dims->v_head_dim))
+            return rc;
+        const size_t smem = tc05::uv_smem(dims->v_head_dim);
+        if (int rc = ensure_smem(tc05::uv_kernel, smem)) return rc;
+        if (int rc = launch(tc05::uv_kernel, dim3(H, (G + tc05::kRows - 1) / tc05::kRows), tc05::kThreads, smem, st,
+            tm_ol, tm_wuv, G, H, dc, dims->v_head_dim, static_cast<uint16_t*>(out))) return rc;
+    } else if (tc) {
         const size_t smem = uv_tc_smem(dc, dims->v_head_dim);
         const dim3 grid(H, (G + kTcRows - 1) / kTcRows);
         uint16_t* o = static_cast<uint16_t*>(out);
         const uint16_t* wv = static_cast<const uint16_t*>(w_uv);
         if (L.kernel == kKernelPair) {  // bf16 partials
             if (int rc = ensure_smem(merge_uv_tc_kernel<uint16_t>, smem)) return rc;
-            merge_uv_tc_kernel<uint16_t><<<grid, kTcThreads, smem, st>>>(
-                reinterpret_cast<const uint16_t*>(o_part), lse_part, part_offsets, wv, G, H, dc, dims->v_head_dim, o);
+            if (int rc = launch(merge_uv_tc_kernel<uint16_t>, grid, kTcThreads, smem, st,
+                reinterpret_cast<const uint16_t*>(o_part), lse_part, part_offsets, wv, G, H, dc, dims->v_head_dim, o)) return rc;
         } else {
             if (int rc = ensure_smem(merge_uv_tc_kernel<float>, smem)) return rc;
-            merge_uv_tc_kernel<float><<<grid, kTcThreads, smem, st>>>(o_part, lse_part, part_offsets, wv, G, H, dc,
-                                                                     dims->v_head_dim, o);
+            if (int rc = launch(merge_uv_tc_kernel<float>, grid, kTcThreads, smem, st, o_part, lse_part, part_offsets, wv, G, H, dc,
+                                                                     dims->v_head_dim, o)) return rc;
         }
     } else {
         const size_t uv_smem = sizeof(float) * kUvGroups * dc;
         if (int rc = ensure_smem(combine_uv_kernel, uv_smem)) return rc;
-        combine_uv_kernel<<<dim3(H, (G + kUvGroups - 1) / kUvGroups), kUvThreads, uv_smem, st>>>(
+        if (int rc = launch(combine_uv_kernel, dim3(H, (G + kUvGroups - 1) / kUvGroups), kUvThreads, uv_smem, st,
             o_part, lse_part, part_offsets, static_cast<const uint16_t*>(w_uv), G, H, dc, dims->v_head_dim,
-            static_cast<uint16_t*>(out));
+            static_cast<uint16_t*>(out))) return rc;
     }
     return launch_status();
 }
@@ -453,8 +534,8 @@ int mla_combine(const mla_dims_t* dims, const float* o_part, const float* lse_pa
     if (!o_part || !lse_part || !part_offsets || !o_lat || n_groups < 1) return MLA_ERR_INVALID_ARG;
     if (static_cast<int64_t>(n_groups) * dims->num_heads >= (int64_t(1) << 31)) return MLA_ERR_UNSUPPORTED_DIMS;
     if (int rc = device_ok()) return rc;
-    combine_kernel<<<n_groups * dims->num_heads, 128, 0, as_stream(stream)>>>(
-        o_part, lse_part, part_offsets, n_groups, dims->num_heads, dims->kv_lora_rank, o_lat, lse_out);
+    if (int rc = launch(combine_kernel, n_groups * dims->num_heads, 128, 0, as_stream(stream),
+        o_part, lse_part, part_offsets, n_groups, dims->num_heads, dims->kv_lora_rank, o_lat, lse_out)) return rc;
     return launch_status();
 }
 
@@ -465,8 +546,8 @@ int mla_debug_resolve_slots(const mla_dims_t* dims, const int32_t* block_table, 
     if (!block_table || !seq_ids || !positions || !rows || n < 1 || num_seqs < 1 || max_blocks_per_seq < 1)
         return MLA_ERR_INVALID_ARG;
     if (int rc = device_ok()) return rc;
-    resolve_slots_kernel<<<(n + 255) / 256, 256, 0, as_stream(stream)>>>(
-        block_table, num_seqs, max_blocks_per_seq, num_blocks, dims->block_size, seq_ids, positions, n, rows);
+    if (int rc = launch(resolve_slots_kernel, (n + 255) / 256, 256, 0, as_stream(stream),
+        block_table, num_seqs, max_blocks_per_seq, num_blocks, dims->block_size, seq_ids, positions, n, rows)) return rc;
     return launch_status();
 }
 

@@ -101,6 +101,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
                                                     int32_t* __restrict__ tile_prefix,
                                                     int32_t* __restrict__ part_offsets,
                                                     int32_t* __restrict__ worker_group) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int32_t warp_tot[32];
     __shared__ int32_t chunk_total;
     const int32_t G = batch * q_len;
