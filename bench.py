@@ -125,6 +125,36 @@ def roofline(bytes_, flops, seconds, peaks):
                 frac=round(tfs / peaks["bf16_tflops"], 4)), gbs, tfs
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# the attention kernel from an ncu capture of this bench's workload, valid only
+# for the kernel sources it was taken on (their SHA-256 below; the capture and
+# its command are summarised under profiles/). Any change to those sources
+# turns the reported traffic into null until a new capture is recorded here.
+KERNEL_SOURCES = ("decode_pair.cuh", "plan.cuh", "sm100.cuh", "common.cuh")
+TRAFFIC = {
+    # profiles/pair_decode_kernel_v3_b64_l1k_8k.md (ncu --set full, one launch)
+    "v3_b64_l1k_8k": {"bytes": 347966720 + 11035904,
+                      "sources_sha256": "4be4c9561fbf8a6e0d4af19b816923ef35c5842676cbac244ae794675d7c4866"},
+}
+
+
+def kernel_sources_sha256() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "mla_latent_kv_29_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str):
+    rec = TRAFFIC.get(workload)
+    if rec is None or rec["sources_sha256"] != kernel_sources_sha256():
+        return None
+    return rec["bytes"]
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -312,8 +342,8 @@ def count_library_launches(step, device):
     with profile(activities=[ProfilerActivity.CUDA]) as prof:
         step()
         torch.cuda.synchronize(device)
-    names = [e.name for e in prof.events() if "CUDA" in str(e.device_type) and e.name.startswith("mla::")]
-    return len(names), sorted(set(n.split("(")[0] for n in names))
+    names = [e.name for e in prof.events() if "CUDA" in str(e.device_type) and "mla::" in e.name]
+    return len(names), sorted(set(n.split("(")[0].replace("void ", "") for n in names))
 
 
 def run_ours(args, w):
@@ -414,7 +444,7 @@ def run_ours(args, w):
     tot = workload_totals(w, st["lengths"].tolist())
     peaks = load_peaks()
     roof, attn_gbs, attn_tfs = roofline(tot["attn_bytes"], tot["attn_flops"], t_attn / 1e3, peaks)
-    roof["traffic"] = None
+    roof["traffic"] = recorded_traffic(w.name) if args.kernel in (0, 1) else None
     roof["kernel"] = "split-KV attention" + (" (CUDA cores)" if args.kernel == 2 else "")
     roof["peak_source"] = peaks["source"]
     nominal_step = max(tot["step_bytes"] / (NOMINAL["hbm_gbs"] * 1e9), tot["step_flops"] / (NOMINAL["bf16_tflops"] * 1e12))
