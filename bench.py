@@ -317,18 +317,37 @@ def setup_gpu(w, device, rank):
     return st
 
 
-def make_step(w, st, kernel):
+def make_step(w, st, kernel, overlap=True):
+    """One step: the append of the batch's new tokens, then the decode. With
+    overlap the append runs on a side stream beside the decode's schedule and
+    query absorption, and the decode's attention waits for it (cache_ready)."""
+    import torch
+
     from mla_latent_kv_29_b200 import lib
 
     d = st["d"]
+    side = torch.cuda.Stream() if overlap else None
+    fork, ready = torch.cuda.Event(), torch.cuda.Event()
+    fork.record()
+    ready.record()  # the handles exist before any capture
+
+    def append(x_new, stream=None):
+        lib.append_kv(d, st["x_new"] if x_new is None else x_new, st["w_kva"], st["new_seq"], st["new_pos"],
+                      st["table"], st["pool"], workspace=st["ws_append"], stream=stream)
 
     def step(x_new=None, q_nope=None, q_pe=None, events=None):
-        lib.append_kv(d, st["x_new"] if x_new is None else x_new, st["w_kva"], st["new_seq"], st["new_pos"],
-                      st["table"], st["pool"], workspace=st["ws_append"])
+        if side is not None:
+            cur = torch.cuda.current_stream()
+            fork.record(cur)
+            side.wait_event(fork)
+            append(x_new, stream=side)
+            ready.record(side)
+        else:
+            append(x_new)
         lib.decode(d, w.softmax_scale, st["q_nope"] if q_nope is None else q_nope,
                    st["q_pe"] if q_pe is None else q_pe, st["pool"], st["table"], st["lengths_d"], st["max_len"],
                    st["w_uk"], st["w_uv"], out=st["out"], workspace=st["ws_decode"], kernel=kernel,
-                   attn_events=events)
+                   attn_events=events, cache_ready=ready if side is not None else None)
 
     return step
 
@@ -357,7 +376,7 @@ def run_ours(args, w):
 
     lib.load()
     st = setup_gpu(w, device, rank)
-    step = make_step(w, st, args.kernel)
+    step = make_step(w, st, args.kernel, overlap=args.overlap)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     for _ in range(args.warmup):
         step()
@@ -456,7 +475,8 @@ def run_ours(args, w):
                    "context": f"U[{w.length_range[0]},{w.length_range[1]}]", "cached_tokens_per_gpu": tot["T"],
                    "heads": w.dims.num_heads, "latent": w.dims.kv_lora_rank, "rope": w.dims.rope_dim,
                    "page": w.dims.block_size, "paged": "shuffled", "l2": "flushed (256 MB write) before each step",
-                   "step": "append of the batch's new tokens + absorbed decode",
+                   "step": "append of the batch's new tokens + absorbed decode" +
+                           (" (append on a side stream; the attention waits for it)" if args.overlap else ""),
                    "launch": "CUDA graph replay" if args.graph else "direct launches"},
         "roofline": roof,
         "attn_us": round(t_attn * 1e3, 2),
@@ -520,6 +540,8 @@ def main(argv=None):
     ap.add_argument("--soak", type=float, default=1.5, help="seconds of untimed steps while clocks are sampled")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--overlap", action=argparse.BooleanOptionalAction, default=True,
+                    help="run the append on a side stream beside the decode's query-side launches")
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="replay each step from a captured CUDA graph")
     args = ap.parse_args(argv)

@@ -86,6 +86,15 @@ typedef struct mla_decode_opts {
                                Under stream capture both are captured as
                                external event-record nodes, so a graph
                                replay records them again. */
+    void* cache_ready;      /* NULL or a cudaEvent_t that the attention
+                               launch (the first launch that reads the
+                               cache) waits for (cudaStreamWaitEvent on
+                               `stream`). Record it after an mla_append_kv
+                               issued on another stream: the append then
+                               runs beside the schedule and the query
+                               absorption, which do not read the cache.
+                               Under stream capture it joins the two
+                               streams' work into one graph. */
 } mla_decode_opts_t;
 
 /* Paged latent cache ("pool"), [MLA-arch] 3.2 kept as one row per token:

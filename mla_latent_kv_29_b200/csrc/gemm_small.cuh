@@ -184,65 +184,4 @@ __global__ void __launch_bounds__(kTcThreads) merge_uv_tc_kernel(
     }
 }
 
-// ----------------------------------------------------------------- append
-// part[z][t][n] = sum over split z's K range of x[t][k] * w[k][n].
-// grid (N / 64, ceil(T / 64), splits); block 128 (4 warps x 16 rows);
-// K range per split a multiple of 64; 2-stage cp.async pipeline over 64-wide K chunks.
-constexpr int kApTc = 64;
-constexpr int kApTcLd = kApTc + 8;
-
-__global__ void __launch_bounds__(128) append_gemm_tc_kernel(
-    const uint16_t* __restrict__ x, const uint16_t* __restrict__ w, float* __restrict__ part,
-    int32_t T, int32_t K, int32_t N, int32_t k_per_split) {
-    pdl_wait();
-    pdl_trigger();
-    __shared__ __align__(16) uint16_t As[2][kApTc * kApTcLd];  // [t][k]
-    __shared__ __align__(16) uint16_t Bs[2][kApTc * kApTcLd];  // [k][n]
-    const int n0 = blockIdx.x * kApTc, t0 = blockIdx.y * kApTc;
-    const int k_begin = blockIdx.z * k_per_split;
-    const int k_end = min(K, k_begin + k_per_split);
-    const int nchunks = k_end > k_begin ? (k_end - k_begin) / kApTc : 0;
-    auto load = [&](int chunk, int buf) {
-        const int k0 = k_begin + chunk * kApTc;
-        for (int i = threadIdx.x; i < kApTc * 8; i += 128) {
-            const int r = i >> 3, c8 = (i & 7) * 8;
-            const int t = t0 + r;
-            if (t < T)
-                wmma16::cp_async16(&As[buf][r * kApTcLd + c8], x + static_cast<int64_t>(t) * K + k0 + c8);
-            else
-                *reinterpret_cast<uint4*>(&As[buf][r * kApTcLd + c8]) = make_uint4(0u, 0u, 0u, 0u);
-            wmma16::cp_async16(&Bs[buf][r * kApTcLd + c8], w + static_cast<int64_t>(k0 + r) * N + n0 + c8);
-        }
-        wmma16::cp_async_commit();
-    };
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float acc[8][4] = {};
-    if (nchunks > 0) load(0, 0);
-    for (int ch = 0; ch < nchunks; ++ch) {
-        if (ch + 1 < nchunks) {
-            load(ch + 1, (ch + 1) & 1);
-            wmma16::cp_async_wait<1>();
-        } else {
-            wmma16::cp_async_wait<0>();
-        }
-        __syncthreads();
-#pragma unroll
-        for (int k0 = 0; k0 < kApTc; k0 += 16)
-            wmma16::warp_tile_k16<false>(acc, As[ch & 1], kApTcLd, 16 * warp, Bs[ch & 1], kApTcLd, 0, k0);
-        __syncthreads();
-    }
-    float* dst = part + static_cast<int64_t>(blockIdx.z) * T * N;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-        const int col = n0 + 8 * nt + 2 * (lane & 3);
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            const int t = t0 + 16 * warp + (lane >> 2) + 8 * hf;
-            if (t < T)
-                *reinterpret_cast<float2*>(dst + static_cast<int64_t>(t) * N + col) =
-                    make_float2(acc[nt][2 * hf], acc[nt][2 * hf + 1]);
-        }
-    }
-}
-
 }  // namespace mla

@@ -52,39 +52,46 @@ __global__ void __launch_bounds__(128) merge_kernel(const PartT* __restrict__ o_
                                                     int32_t dc, uint16_t* __restrict__ o_lat) {
     pdl_wait();
     pdl_trigger();
-    // lane l owns columns 16 l .. 16 l + 15 (d_c = 512); the weights of up to 32
-    // parts are computed by the lanes at once, and the part rows are loaded four
-    // at a time before they are used, so a warp waits on few memory round trips.
+    // Lane l owns columns ncol * l .. + ncol - 1. The lse values of up to 32 parts
+    // (one per lane) and the rows of four parts are requested together, so a group
+    // with at most four parts costs one memory round trip; more parts follow four
+    // rows at a time, their weights taken from the lanes by shuffles.
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = blockIdx.x, h = blockIdx.y * 4 + warp;
     if (h >= H) return;
     const int32_t p0 = part_offsets[g], p1 = part_offsets[g + 1];
-    float M = -INFINITY;
-    for (int32_t p = p0 + lane; p < p1; p += 32) M = fmaxf(M, lse_part[static_cast<int64_t>(p) * H + h]);
-    M = warp_max(M);
     const int ncol = dc / 32;  // columns per lane: 16 for d_c = 512, 8 for 256
+    auto load_row = [&](int32_t p, float (&v)[16]) {
+        const PartT* src = o_part + (static_cast<int64_t>(p) * H + h) * dc + ncol * lane;
+        float (&v0)[8] = *reinterpret_cast<float(*)[8]>(&v[0]);
+        float (&v1)[8] = *reinterpret_cast<float(*)[8]>(&v[8]);
+        load8(src, v0);
+        if (ncol == 16) load8(src + 8, v1);
+    };
+    float v[4][16];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        if (p0 + u < p1) load_row(p0 + u, v[u]);
+    float lse_first = p0 + lane < p1 ? lse_part[static_cast<int64_t>(p0 + lane) * H + h] : -INFINITY;
+    float M = lse_first;
+    for (int32_t p = p0 + 32 + lane; p < p1; p += 32) M = fmaxf(M, lse_part[static_cast<int64_t>(p) * H + h]);
+    M = warp_max(M);
     float acc[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) acc[e] = 0.f;
     float den = 0.f;
     if (M != -INFINITY) {
         for (int32_t c0 = p0; c0 < p1; c0 += 32) {
-            const int32_t pl = c0 + lane;
-            const float l = pl < p1 ? lse_part[static_cast<int64_t>(pl) * H + h] : -INFINITY;
+            const float l = c0 == p0 ? lse_first
+                                     : (c0 + lane < p1 ? lse_part[static_cast<int64_t>(c0 + lane) * H + h] : -INFINITY);
             const float wl = l == -INFINITY ? 0.f : __expf(l - M);
             den += warp_sum(wl);
             const int n = min(32, p1 - c0);
             for (int i0 = 0; i0 < n; i0 += 4) {
-                float v[4][16];
+                if (c0 != p0 || i0 != 0) {  // the first four rows are already in flight
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (i0 + u < n) {
-                        const PartT* src = o_part + (static_cast<int64_t>(c0 + i0 + u) * H + h) * dc + ncol * lane;
-                        float (&v0)[8] = *reinterpret_cast<float(*)[8]>(&v[u][0]);
-                        float (&v1)[8] = *reinterpret_cast<float(*)[8]>(&v[u][8]);
-                        load8(src, v0);
-                        if (ncol == 16) load8(src + 8, v1);
-                    }
+                    for (int u = 0; u < 4; ++u)
+                        if (i0 + u < n) load_row(c0 + i0 + u, v[u]);
                 }
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -188,6 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1) uv_kernel(const __grid_constant__
     if (ok) {
         const int g = g0 + static_cast<int>(threadIdx.x);
         const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+#pragma unroll 1
         for (int c0 = 0; c0 < dv; c0 += 32) {
             float v[32];
             ptx::tmem_ld32(tl + c0, v);
@@ -210,33 +218,251 @@ __global__ void __launch_bounds__(kThreads, 1) uv_kernel(const __grid_constant__
     }
 }
 
-// --------------------------------------------------------------- absorb
-// Q[g, h, 0:d_c] = bf16(q_nope[g, h, :] W_UK[h]) and Q[g, h, d_c:] = q_pe[g, h]
-// for g in [g0, g0 + 128). tm_q: q_nope as 2-D [G rows, H * d_n columns], box
-// {64, 128} (K-major A); tm_w: W_UK as 2-D [H * d_n rows, d_c columns], box
-// {64, d_n} (MN-major B: the latent index is contiguous). All d_n / 64 A boxes
-// and d_c / 64 B boxes are loaded at once (d_n = 128, d_c = 512: 160 KB), then
-// the (d_c / 256) x (d_n / 16) MMAs of N = 256 run into d_c TMEM columns.
-// grid (H, ceil(G / 128)); block 128; dynamic smem absorb_smem(d_n, d_c).
-__host__ __device__ inline size_t absorb_a_bytes(int dn) { return static_cast<size_t>(dn / 64) * kRows * kBoxBytes; }
-__host__ __device__ inline size_t absorb_smem(int dn, int dc) {
-    return absorb_a_bytes(dn) + static_cast<size_t>(dc / 64) * dn * kBoxBytes + 256 + 1024;
+// ------------------------------------------------------------ merge + UV
+// out[g, h, :] = bf16(W_UV[h] o_lat[g, h, :]) for the kMuvRows groups g of
+// block blockIdx.y, where o_lat[g, h] is the log-sum-exp merge of group g's
+// bf16 split-KV partials (the merge_kernel rule, rounded to bf16). o_lat
+// never goes to memory: the product is taken transposed, D[d, g] = sum_c
+// W_UV[h][d, c] o_lat[g, c], with M = d_v = 128 rows of W_UV[h] (A) and
+// N = 64 groups (B), so a small batch pads no MMA row, and each 64-column
+// block kb of B is merged straight into shared memory, in the 128-byte
+// swizzled K-major layout, from the partial rows of the block's groups.
+// The CTA's groups own the consecutive partial slots [P0, P1); per block kb a
+// ring stage receives, by TMA, W_UV[h][:, 64 kb ..] (box {64, 128} of tm_w =
+// W_UV as 2-D [H * d_v rows, d_c columns]) and the slots' columns 64 kb ..
+// (n_box boxes {64 columns, 1 head, 64 slots} of tm_p = the partials as 3-D
+// [slots][H][d_c]), so the stages are in flight together and no warp waits
+// on a chain of dependent loads; thread 0 refills the stage of block kb - 1
+// with block kb + 3 at the top of block kb. The weights exp(lse - max) / sum
+// come first: the slots' lse into shared memory in one round trip, then one
+// warp per group with lanes over its slots. Thread t merges group t / 4,
+// columns 16 (t % 4) .. + 15 of a block.
+// grid (H, ceil(G / 64)); block 256; dynamic smem merge_uv_smem(n_box);
+// d_v = 128, d_c a multiple of 64 up to 512, P1 - P0 <= 64 n_box, n_box <= 4.
+constexpr int kMuvThreads = 256;
+constexpr int kMuvRows = 64;     // groups per CTA (the MMA's N)
+constexpr int kMuvDv = 128;      // the MMA's M
+constexpr int kMuvStages = 4;
+constexpr int kMuvMaxBox = 4;    // slot boxes of 64 per stage at most
+constexpr int kMuvSlotBox = 64 * kBoxBytes;  // 8 KB: 64 slots x 64 columns
+__host__ __device__ inline int merge_uv_stage_bytes(int n_box) {
+    return n_box * kMuvSlotBox + kMuvDv * kBoxBytes + kMuvRows * kBoxBytes;
+}
+__host__ __device__ inline size_t merge_uv_smem(int n_box) {
+    return static_cast<size_t>(kMuvStages) * merge_uv_stage_bytes(n_box) + 256 + 512 + 4 * 64 * kMuvMaxBox + 1024;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) absorb_kernel(const __grid_constant__ CUtensorMap tm_q,
-                                                            const __grid_constant__ CUtensorMap tm_w,
-                                                            const uint16_t* __restrict__ q_pe, int32_t G,
-                                                            int32_t H, int32_t dn, int32_t dc, int32_t dr,
-                                                            uint16_t* __restrict__ q_out) {
+__global__ void __launch_bounds__(kMuvThreads, 1) merge_uv_kernel(const __grid_constant__ CUtensorMap tm_w,
+                                                                 const __grid_constant__ CUtensorMap tm_p,
+                                                                 const float* __restrict__ lse_part,
+                                                                 const int32_t* __restrict__ part_offsets,
+                                                                 int32_t G, int32_t H, int32_t dc, int32_t n_box,
+                                                                 uint16_t* __restrict__ out) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int nk = dc / 64;
+    const int stage_bytes = merge_uv_stage_bytes(n_box);
+    const int off_w = n_box * kMuvSlotBox, off_bm = off_w + kMuvDv * kBoxBytes;  // within a stage
+    const int off_bar = kMuvStages * stage_bytes;  // full[s], empty[s], done
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + off_bar + 8 * (2 * kMuvStages + 1));
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + 8 * (2 * kMuvStages + 1) + 16);
+    int32_t* offs = reinterpret_cast<int32_t*>(smem + off_bar + 256);          // kMuvRows + 1 entries
+    float* wgt = reinterpret_cast<float*>(smem + off_bar + 256 + 512);         // per slot of [P0, P1)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.x, g0 = blockIdx.y * kMuvRows;
+    const int R = min(kMuvRows, G - g0);
+    if (threadIdx.x == 0) {
+        *abort = 0;
+        for (int i = 0; i <= 2 * kMuvStages; ++i) ptx::mbar_init(bar_addr(smem, off_bar, i), 1);
+        ptx::fence_mbar_init();
+        ptx::prefetch_tmap(&tm_w);
+        ptx::prefetch_tmap(&tm_p);
+    }
+    if (warp == 2) {
+        ptx::tmem_alloc_1(ptx::smem_u32(tmem_slot), kMuvRows);
+        ptx::tmem_relinquish_1();
+    }
+    // part_offsets come from the plan launch, which finished before the attention
+    // launch (this one's predecessor) could pass its own dependency wait
+    if (static_cast<int>(threadIdx.x) <= R) offs[threadIdx.x] = part_offsets[g0 + threadIdx.x];
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int32_t P0 = offs[0], NP = offs[R] - P0;
+    const int nb = NP > 0 ? (NP + 63) / 64 : 0;  // slot boxes this CTA needs
+    const bool fits = nb <= n_box;
+    if (!fits && threadIdx.x == 0) record_status(MLA_ERR_DEVICE_FAULT);
+    auto stage_tx = [&]() { return static_cast<uint32_t>(nb * kMuvSlotBox + kMuvDv * kBoxBytes); };
+    if (threadIdx.x == 0) {  // the weights are not written by earlier launches: request them now
+        for (int kb = 0; kb < min(nk, kMuvStages); ++kb) {
+            const uint32_t full = bar_addr(smem, off_bar, kb);
+            ptx::mbar_arrive_expect_tx_local(full, fits ? stage_tx() : kMuvDv * kBoxBytes);
+            ptx::tma_load_2d(ptx::smem_u32(smem + kb * stage_bytes + off_w), &tm_w, 64 * kb, h * kMuvDv, full);
+        }
+    }
+    pdl_wait();
+    pdl_trigger();
+    auto load_slots = [&](int kb, uint32_t full) {
+        if (!fits) return;
+        for (int b = 0; b < nb; ++b)
+            ptx::tma_load_3d(ptx::smem_u32(smem + (kb % kMuvStages) * stage_bytes + b * kMuvSlotBox), &tm_p, 64 * kb, h,
+                             P0 + 64 * b, full);
+    };
+    if (threadIdx.x == 0)
+        for (int kb = 0; kb < min(nk, kMuvStages); ++kb) load_slots(kb, bar_addr(smem, off_bar, kb));
+
+    // ---- weights. This code runs once per CTA, so it is kept short (loops, not
+    // unrolled copies): on a cold instruction cache every new line of code costs
+    // a round trip to L2. (1) every slot's lse into shared memory, one round trip.
+    if (fits)
+        for (int i = threadIdx.x; i < NP; i += kMuvThreads) wgt[i] = lse_part[static_cast<int64_t>(P0 + i) * H + h];
+    __syncthreads();
+    // (2) per group (a warp, lanes over its slots): max, sum, then the normalised
+    // weights in place (each lane rewrites only the slots it read)
+    if (fits) {
+#pragma unroll 1
+        for (int jj = warp; jj < R; jj += kMuvThreads / 32) {
+            const int32_t a = offs[jj] - P0, b = offs[jj + 1] - P0;
+            float M = -INFINITY;
+            for (int32_t i = a + lane; i < b; i += 32) M = fmaxf(M, wgt[i]);
+            M = warp_max(M);
+            float den = 0.f;
+            if (M != -INFINITY)
+                for (int32_t i = a + lane; i < b; i += 32) den += wgt[i] == -INFINITY ? 0.f : __expf(wgt[i] - M);
+            den = warp_sum(den);
+            const float inv = den > 0.f ? __fdividef(1.f, den) : 0.f;
+            for (int32_t i = a + lane; i < b; i += 32) {
+                const float l = wgt[i];
+                wgt[i] = l == -INFINITY || M == -INFINITY ? 0.f : __expf(l - M) * inv;
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- per 64-column block: merge into B, then 4 MMAs
+    const int j = static_cast<int>(threadIdx.x) >> 2, q = static_cast<int>(threadIdx.x) & 3;
+    const int32_t s0 = j < R ? offs[j] - P0 : 0, s1 = j < R ? offs[j + 1] - P0 : 0;
+#pragma unroll 1
+    for (int kb = 0; kb < nk; ++kb) {
+        const int st = kb % kMuvStages;
+        uint8_t* stage = smem + st * stage_bytes;
+        if (threadIdx.x == 0 && kb >= 1 && kb - 1 + kMuvStages < nk) {
+            // refill the previous block's stage with block kb + 3 once its MMAs are done
+            const int ps = (kb - 1) % kMuvStages;
+            if (ptx::mbar_wait(bar_addr(smem, off_bar, kMuvStages + ps), ((kb - 1) / kMuvStages) & 1, abort)) {
+                const uint32_t full = bar_addr(smem, off_bar, ps);
+                ptx::mbar_arrive_expect_tx_local(full, fits ? stage_tx() : kMuvDv * kBoxBytes);
+                ptx::tma_load_2d(ptx::smem_u32(smem + ps * stage_bytes + off_w), &tm_w, 64 * (kb - 1 + kMuvStages),
+                                 h * kMuvDv, full);
+                load_slots(kb - 1 + kMuvStages, full);
+            }
+        }
+        const bool ok = ptx::mbar_wait(bar_addr(smem, off_bar, st), (kb / kMuvStages) & 1, abort);
+        if (j < R) {
+            float acc[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+            if (ok && fits) {
+#pragma unroll 1
+                for (int32_t i = s0; i < s1; ++i) {  // slot i: box i / 64, swizzled row i % 64
+                    const float w = wgt[i];
+                    const uint8_t* row = stage + (i >> 6) * kMuvSlotBox + (i & 63) * kBoxBytes;
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const uint4 u = *reinterpret_cast<const uint4*>(row + (((2 * q + c) ^ (i & 7)) << 4));
+                        const uint32_t x[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            acc[8 * c + 2 * k] = fmaf(w, __uint_as_float(x[k] << 16), acc[8 * c + 2 * k]);
+                            acc[8 * c + 2 * k + 1] = fmaf(w, __uint_as_float(x[k] & 0xffff0000u), acc[8 * c + 2 * k + 1]);
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+                *reinterpret_cast<uint4*>(stage + off_bm + j * kBoxBytes + (((2 * q + c) ^ (j & 7)) << 4)) =
+                    make_uint4(ptx::bf16x2(acc[8 * c], acc[8 * c + 1]), ptx::bf16x2(acc[8 * c + 2], acc[8 * c + 3]),
+                               ptx::bf16x2(acc[8 * c + 4], acc[8 * c + 5]), ptx::bf16x2(acc[8 * c + 6], acc[8 * c + 7]));
+        }
+        ptx::fence_proxy_async_smem();  // B was written through the generic proxy
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            ptx::tc_fence_after();
+            constexpr uint32_t idesc = ptx::idesc_bf16(kMuvDv, kMuvRows, false, false);
+            const uint64_t da = ptx::smem_desc_sw128(ptx::smem_u32(stage + off_w), 16, 1024);
+            const uint64_t db = ptx::smem_desc_sw128(ptx::smem_u32(stage + off_bm), 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) ptx::mma_bf16_1(tmem, da + 2 * kk, db + 2 * kk, idesc, (kb | kk) != 0);
+            ptx::mma_commit_1(bar_addr(smem, off_bar, kMuvStages + st));
+        }
+    }
+    if (threadIdx.x == 0) ptx::mma_commit_1(bar_addr(smem, off_bar, 2 * kMuvStages));
+    __syncwarp();
+
+    // ---- epilogue: thread t < 128 = TMEM lane t = output column d; TMEM column j = group g0 + j.
+    // D goes through shared memory (stage 0, free once every MMA is done) as bf16 [64 groups][128]
+    // so that the stores are whole 16-byte pieces of the output rows.
+    const bool done = ptx::mbar_wait(bar_addr(smem, off_bar, 2 * kMuvStages), 0, abort) && !*abort;
+    ptx::tc_fence_after();
+    uint16_t* stg = reinterpret_cast<uint16_t*>(smem);
+    if (warp < 4) {
+        const int d = static_cast<int>(threadIdx.x);
+#pragma unroll 1
+        for (int c0 = 0; c0 < R; c0 += 32) {
+            float v[32];
+            ptx::tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                stg[(c0 + i) * kMuvDv + d] = static_cast<uint16_t>(ptx::bf16x2(v[i], 0.f) & 0xffffu);
+        }
+    }
+    __syncthreads();
+    if (done) {
+        for (int idx = threadIdx.x; idx < R * (kMuvDv / 8); idx += kMuvThreads) {
+            const int jj = idx / (kMuvDv / 8), c8 = idx % (kMuvDv / 8);
+            *reinterpret_cast<uint4*>(out + (static_cast<int64_t>(g0 + jj) * H + h) * kMuvDv + 8 * c8) =
+                *reinterpret_cast<const uint4*>(stg + jj * kMuvDv + 8 * c8);
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc_1(tmem, kMuvRows);
+    }
+}
+
+// --------------------------------------------------------------- absorb
+// Q[g, h, 256 z .. 256 z + 255] = bf16(q_nope[g, h, :] W_UK[h][:, 256 z ..]) for
+// g in [g0, g0 + 128), and (z = 0) Q[g, h, d_c:] = q_pe[g, h]. tm_q: q_nope as
+// 2-D [G rows, H * d_n columns], box {64, 128} (K-major A); tm_w: W_UK as 2-D
+// [H * d_n rows, d_c columns], box {64, d_n} (MN-major B: the latent index is
+// contiguous). Each CTA loads its d_n / 64 A boxes and the 4 B boxes of its
+// 256 output columns at once (d_n = 128: 96 KB, two CTAs per SM), then runs
+// d_n / 16 MMAs of N = 256 into 256 TMEM columns.
+// grid (H, ceil(G / 128), d_c / 256); block 128; dynamic smem absorb_smem(d_n).
+__host__ __device__ inline size_t absorb_a_bytes(int dn) { return static_cast<size_t>(dn / 64) * kRows * kBoxBytes; }
+__host__ __device__ inline size_t absorb_smem(int dn) {
+    return absorb_a_bytes(dn) + static_cast<size_t>(4) * dn * kBoxBytes + 256 + 1024;
+}
+
+__global__ void __launch_bounds__(kThreads) absorb_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                          const __grid_constant__ CUtensorMap tm_w,
+                                                          const uint16_t* __restrict__ q_pe, int32_t G, int32_t H,
+                                                          int32_t dn, int32_t dc, int32_t dr,
+                                                          uint16_t* __restrict__ q_out) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
     const int a_bytes = static_cast<int>(absorb_a_bytes(dn));
     const int b_box = dn * kBoxBytes;  // one [d_n x 64] box of W_UK[h]
-    const int off_bar = a_bytes + (dc / 64) * b_box;  // full, done
+    const int off_bar = a_bytes + 4 * b_box;  // full, done
     volatile int* abort = reinterpret_cast<volatile int*>(smem + off_bar + 16);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + 32);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.x, g0 = blockIdx.y * kRows;
+    const int h = blockIdx.x, g0 = blockIdx.y * kRows, z = blockIdx.z;
     if (threadIdx.x == 0) {
         *abort = 0;
         ptx::mbar_init(bar_addr(smem, off_bar, 0), 1);
@@ -246,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) absorb_kernel(const __grid_consta
         ptx::prefetch_tmap(&tm_w);
     }
     if (warp == 2) {
-        ptx::tmem_alloc_1(ptx::smem_u32(tmem_slot), 512);
+        ptx::tmem_alloc_1(ptx::smem_u32(tmem_slot), 256);
         ptx::tmem_relinquish_1();
     }
     ptx::tc_fence_before();
@@ -258,25 +484,22 @@ __global__ void __launch_bounds__(kThreads, 1) absorb_kernel(const __grid_consta
     const uint32_t full = bar_addr(smem, off_bar, 0), done = bar_addr(smem, off_bar, 1);
 
     if (warp == 0 && lane == 0) {  // producer: everything at once
-        ptx::mbar_arrive_expect_tx_local(full, a_bytes + (dc / 64) * b_box);
+        ptx::mbar_arrive_expect_tx_local(full, a_bytes + 4 * b_box);
         for (int kb = 0; kb < dn / 64; ++kb)
             ptx::tma_load_2d(ptx::smem_u32(smem + kb * kRows * kBoxBytes), &tm_q, h * dn + 64 * kb, g0, full);
-        for (int nb = 0; nb < dc / 64; ++nb)
-            ptx::tma_load_2d(ptx::smem_u32(smem + a_bytes + nb * b_box), &tm_w, 64 * nb, h * dn, full);
+        for (int nb = 0; nb < 4; ++nb)
+            ptx::tma_load_2d(ptx::smem_u32(smem + a_bytes + nb * b_box), &tm_w, 256 * z + 64 * nb, h * dn, full);
     } else if (warp == 1 && lane == 0) {  // MMA issuer
         constexpr uint32_t idesc = ptx::idesc_bf16(kRows, 256, false, true);
         if (ptx::mbar_wait(full, 0, abort)) {
             ptx::tc_fence_after();
             const uint32_t sa = ptx::smem_u32(smem), sb = ptx::smem_u32(smem + a_bytes);
-            for (int nh = 0; nh < dc / 256; ++nh) {
-                // B: rows (k) 16 ks .. +15 = two 8-row atoms (2 KB), columns 256 nh .. +255 = 4 boxes (LBO = box)
-                const uint64_t db = ptx::smem_desc_sw128(sb + 4 * nh * b_box, b_box, 1024);
-                for (int ks = 0; ks < dn / 16; ++ks) {
-                    const uint64_t da = ptx::smem_desc_sw128(sa + (ks >> 2) * kRows * kBoxBytes, 16, 1024) +
-                                        static_cast<uint64_t>(2 * (ks & 3));
-                    ptx::mma_bf16_1(tmem + 256 * nh, da, db + static_cast<uint64_t>((2048 * ks) >> 4), idesc,
-                                    ks != 0);
-                }
+            // B: rows (k) 16 ks .. +15 = two 8-row atoms (2 KB), the 4 boxes of 64 columns LBO apart
+            const uint64_t db = ptx::smem_desc_sw128(sb, b_box, 1024);
+            for (int ks = 0; ks < dn / 16; ++ks) {
+                const uint64_t da = ptx::smem_desc_sw128(sa + (ks >> 2) * kRows * kBoxBytes, 16, 1024) +
+                                    static_cast<uint64_t>(2 * (ks & 3));
+                ptx::mma_bf16_1(tmem, da, db + static_cast<uint64_t>((2048 * ks) >> 4), idesc, ks != 0);
             }
         }
         ptx::mma_commit_1(done);
@@ -288,12 +511,13 @@ __global__ void __launch_bounds__(kThreads, 1) absorb_kernel(const __grid_consta
         const int g = g0 + static_cast<int>(threadIdx.x);
         const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         const int D = dc + dr;
-        for (int c0 = 0; c0 < dc; c0 += 32) {
+#pragma unroll 1  // one-shot code: kept short for a cold instruction cache
+        for (int c0 = 0; c0 < 256; c0 += 32) {
             float v[32];
             ptx::tmem_ld32(tl + c0, v);
             ptx::tmem_wait_ld();
             if (g < G) {
-                uint4* dst = reinterpret_cast<uint4*>(q_out + (static_cast<int64_t>(g) * H + h) * D + c0);
+                uint4* dst = reinterpret_cast<uint4*>(q_out + (static_cast<int64_t>(g) * H + h) * D + 256 * z + c0);
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     dst[i] = make_uint4(ptx::bf16x2(v[8 * i], v[8 * i + 1]), ptx::bf16x2(v[8 * i + 2], v[8 * i + 3]),
@@ -301,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1) absorb_kernel(const __grid_consta
                                         ptx::bf16x2(v[8 * i + 6], v[8 * i + 7]));
             }
         }
-        if (g < G) {  // the RoPE part of the query row
+        if (g < G && z == 0) {  // the RoPE part of the query row
             const uint4* src = reinterpret_cast<const uint4*>(q_pe + (static_cast<int64_t>(g) * H + h) * dr);
             uint4* dst = reinterpret_cast<uint4*>(q_out + (static_cast<int64_t>(g) * H + h) * D + dc);
             for (int i = 0; i < dr / 8; ++i) dst[i] = src[i];
@@ -311,7 +535,154 @@ __global__ void __launch_bounds__(kThreads, 1) absorb_kernel(const __grid_consta
     __syncthreads();
     if (warp == 2) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc_1(tmem, 512);
+        ptx::tmem_dealloc_1(tmem, 256);
+    }
+}
+
+// --------------------------------------------------------------- append
+// kv[t, n0 .. n0 + 63] = x[t, :] W_kva[:, n0 .. n0 + 63] (fp32) for t in
+// [m0, m0 + 128): the joint down-projection of the cache append
+// (kv_a_proj_with_mqa, "MLA架构：低秩注意力机制优化LLM显存与计算效率" 2.2).
+// The hidden dimension is split over the S CTAs of a cluster (grid z,
+// cluster (1, 1, S)); each streams its K-blocks of 64 through a ring of
+// (x box {64, 128 rows}, W box {64 columns, 64 rows}) stages into a
+// M 128 x N 64 TMEM accumulator, the S partial tiles meet in shared memory
+// and CTA r of the cluster sums rows [r 128 / S, (r + 1) 128 / S) over the
+// cluster (distributed shared memory) and stores them. S = 1 stores directly.
+// tm_x: x as 2-D [T rows, hidden columns]; tm_w: W_kva as 2-D [hidden rows,
+// N columns], box {64, 64} (MN-major B). grid (N / 64, ceil(T / 128), S);
+// block 128; dynamic smem append_smem().
+constexpr int kApStages = 6;
+constexpr int kApStageBytes = kRows * kBoxBytes + 64 * kBoxBytes;  // 24 KB
+__host__ __device__ inline size_t append_smem() { return static_cast<size_t>(kApStages) * kApStageBytes + 256 + 1024; }
+
+__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t cluster_addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(cluster_addr)
+                 : "memory");
+    return v;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) append_kernel(const __grid_constant__ CUtensorMap tm_x,
+                                                            const __grid_constant__ CUtensorMap tm_w, int32_t T,
+                                                            int32_t N, int32_t k_blocks, int32_t k_blocks_per_cta,
+                                                            int32_t S, float* __restrict__ kv) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int off_bar = kApStages * kApStageBytes;  // full[s], empty[s], done
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + off_bar + 8 * (2 * kApStages + 1));
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + 8 * (2 * kApStages + 1) + 16);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * 64, m0 = blockIdx.y * kRows, z = blockIdx.z;
+    const int kb0 = z * k_blocks_per_cta;
+    const int nk = max(0, min(k_blocks_per_cta, k_blocks - kb0));  // this CTA's K-blocks of 64
+    if (threadIdx.x == 0) {
+        *abort = 0;
+        for (int i = 0; i < kApStages; ++i) {
+            ptx::mbar_init(bar_addr(smem, off_bar, i), 1);
+            ptx::mbar_init(bar_addr(smem, off_bar, kApStages + i), 1);
+        }
+        ptx::mbar_init(bar_addr(smem, off_bar, 2 * kApStages), 1);
+        ptx::fence_mbar_init();
+        ptx::prefetch_tmap(&tm_x);
+        ptx::prefetch_tmap(&tm_w);
+    }
+    if (warp == 2) {
+        ptx::tmem_alloc_1(ptx::smem_u32(tmem_slot), 64);
+        ptx::tmem_relinquish_1();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp == 0 && lane == 0) {  // producer
+        for (int i = 0; i < nk; ++i) {
+            const int st = i % kApStages;
+            if (!ptx::mbar_wait(bar_addr(smem, off_bar, kApStages + st), ((i / kApStages) & 1) ^ 1, abort)) break;
+            const uint32_t full = bar_addr(smem, off_bar, st);
+            const uint32_t dst = ptx::smem_u32(smem + st * kApStageBytes);
+            ptx::mbar_arrive_expect_tx_local(full, kApStageBytes);
+            ptx::tma_load_2d(dst, &tm_x, 64 * (kb0 + i), m0, full);
+            ptx::tma_load_2d(dst + kRows * kBoxBytes, &tm_w, n0, 64 * (kb0 + i), full);
+        }
+    } else if (warp == 1 && lane == 0) {  // MMA issuer
+        constexpr uint32_t idesc = ptx::idesc_bf16(kRows, 64, false, true);
+        for (int i = 0; i < nk; ++i) {
+            const int st = i % kApStages;
+            if (!ptx::mbar_wait(bar_addr(smem, off_bar, st), (i / kApStages) & 1, abort)) break;
+            ptx::tc_fence_after();
+            const uint32_t base = ptx::smem_u32(smem + st * kApStageBytes);
+            const uint64_t da = ptx::smem_desc_sw128(base, 16, 1024);
+            const uint64_t db = ptx::smem_desc_sw128(base + kRows * kBoxBytes, 64 * kBoxBytes, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                ptx::mma_bf16_1(tmem, da + 2 * kk, db + static_cast<uint64_t>((2048 * kk) >> 4), idesc,
+                                (i | kk) != 0);
+            ptx::mma_commit_1(bar_addr(smem, off_bar, kApStages + st));
+        }
+        ptx::mma_commit_1(bar_addr(smem, off_bar, 2 * kApStages));
+    }
+    // thread t = TMEM lane t = token row m0 + t: the CTA's partial tile into shared memory
+    // (row t: 64 floats = 16 chunks of 16 B, chunk c at (c ^ (t & 15)) to spread the banks);
+    // the ring is free once every MMA is done
+    const bool ok = ptx::mbar_wait(bar_addr(smem, off_bar, 2 * kApStages), 0, abort);
+    ptx::tc_fence_after();
+    const int t = static_cast<int>(threadIdx.x);
+    float* red = reinterpret_cast<float*>(smem);
+    {
+        float v[64];
+        float (&v0)[32] = *reinterpret_cast<float(*)[32]>(&v[0]);
+        float (&v1)[32] = *reinterpret_cast<float(*)[32]>(&v[32]);
+        const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        ptx::tmem_ld32(tl, v0);
+        ptx::tmem_ld32(tl + 32, v1);
+        ptx::tmem_wait_ld();
+        if (!ok || nk == 0) {  // nothing accumulated (or a wait gave up): contribute zeros
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] = 0.f;
+        }
+        if (S == 1) {
+            if (m0 + t < T) {
+                float4* dst = reinterpret_cast<float4*>(kv + static_cast<int64_t>(m0 + t) * N + n0);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                *reinterpret_cast<float4*>(red + t * 64 + ((c ^ (t & 15)) << 2)) =
+                    make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        }
+    }
+    if (S > 1) {
+        ptx::cluster_sync();  // every partial tile of the cluster is in shared memory
+        const int rows = kRows / S, r0 = static_cast<int>(ptx::cluster_ctarank()) * rows;  // this CTA's rows
+        const uint32_t red_s = ptx::smem_u32(red);
+        for (int idx = t; idx < rows * 16; idx += kThreads) {
+            const int row = r0 + idx / 16, c = idx % 16;
+            const uint32_t off = static_cast<uint32_t>(row * 64 + ((c ^ (row & 15)) << 2)) * 4;
+            float4 b[8];  // every peer's chunk is requested before any is summed
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (q < S) b[q] = ld_dsmem_v4(ptx::mapa(red_s + off, static_cast<uint32_t>(q)));
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (q < S) { a.x += b[q].x; a.y += b[q].y; a.z += b[q].z; a.w += b[q].w; }
+            if (m0 + row < T) *reinterpret_cast<float4*>(kv + static_cast<int64_t>(m0 + row) * N + n0 + 4 * c) = a;
+        }
+        ptx::cluster_sync();  // peers stay resident until every read of their tile is done
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc_1(tmem, 64);
     }
 }
 

@@ -3,6 +3,7 @@
 // allocates, frees or synchronises (except mla_get_device_error, whose job
 // is to synchronise and read the device status word).
 #include <cmath>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <utility>
@@ -62,22 +63,35 @@ int device_ok() {
 // Launches `kernel` on `st` with programmatic stream serialization (the
 // kernels call pdl_wait() before touching data of earlier work, see common.cuh).
 template <typename... KArgs, typename... Args>
-int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+int launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, dim3 cluster,
+                   Args&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (cluster.x * cluster.y * cluster.z > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = cluster.x;
+        attr[1].val.clusterDim.y = cluster.y;
+        attr[1].val.clusterDim.z = cluster.z;
+        cfg.numAttrs = 2;
+    }
     if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
         cudaGetLastError();
         return MLA_ERR_CUDA;
     }
     return MLA_OK;
+}
+
+template <typename... KArgs, typename... Args>
+int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+    return launch_cluster(kernel, grid, block, smem, st, dim3(1, 1, 1), std::forward<Args>(args)...);
 }
 
 int launch_status() {
@@ -172,6 +186,21 @@ int encode_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
     return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// 3-D bf16 tensor map over the split-KV partials [slots][H][d_c]: box {64
+// columns, 1 head, 64 slots}, 128-byte swizzle; slots past the end read 0.
+int encode_parts(CUtensorMap* m, const void* base, uint64_t dc, uint64_t H, uint64_t slots) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return MLA_ERR_CUDA;
+    cuuint64_t dims[3] = {dc, H, slots};
+    cuuint64_t strides[2] = {dc * 2, H * dc * 2};
+    cuuint32_t box[3] = {64, 1, 64};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
 // The tcgen05 absorb / merge / UV kernels: d_n a multiple of 64 up to 256, d_c
 // a multiple of 256 up to 512, d_r a multiple of 8, d_v a multiple of 16 up
 // to 256, and 16-byte aligned operands.
@@ -230,6 +259,9 @@ bool tc_gemm_dims_ok(const mla_dims_t* d) {
 }
 
 // ---- append split-K plan ----------------------------------------------
+// tc: the tcgen05 GEMM (N and hidden multiples of 64), its K split over a
+// cluster of `splits` CTAs that reduce on chip, so the epilogue sees one
+// partial; otherwise the CUDA-core GEMM writes `splits` partials.
 struct AppendPlan {
     bool tc;
     int splits, k_per_split;
@@ -237,8 +269,17 @@ struct AppendPlan {
 
 AppendPlan append_plan(int32_t n_tokens, int32_t hidden, int32_t N) {
     AppendPlan a;
-    a.tc = (N % kApTc == 0) && (hidden % kApTc == 0);
-    const int tile_n = a.tc ? kApTc : kApTileN, tile_t = a.tc ? kApTc : kApTileT, tile_k = a.tc ? kApTc : kApTileK;
+    a.tc = (N % 64 == 0) && (hidden % 64 == 0);
+    if (a.tc) {
+        const int64_t tiles = static_cast<int64_t>(N / 64) * ((n_tokens + tc05::kRows - 1) / tc05::kRows);
+        const int k_blocks = hidden / 64;
+        int s = 8;  // a portable cluster; it must divide the 128 rows of a tile
+        while (s > 1 && (tiles * s > num_sms() || s > k_blocks)) s /= 2;
+        a.splits = s;
+        a.k_per_split = (k_blocks + s - 1) / s;  // in K-blocks of 64
+        return a;
+    }
+    const int tile_n = kApTileN, tile_t = kApTileT, tile_k = kApTileK;
     const int64_t tiles = static_cast<int64_t>((N + tile_n - 1) / tile_n) * ((n_tokens + tile_t - 1) / tile_t);
     const int64_t target = 2 * num_sms();
     const int64_t chunks = (hidden + tile_k - 1) / tile_k;
@@ -291,7 +332,7 @@ size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t n_tokens, int32
     if (check_dims(dims) || n_tokens < 1 || hidden < 1) return 0;
     const int N = dims->kv_lora_rank + dims->rope_dim;
     const AppendPlan a = append_plan(n_tokens, hidden, N);
-    return align_up(sizeof(float) * static_cast<size_t>(a.splits) * n_tokens * N);
+    return align_up(sizeof(float) * static_cast<size_t>(a.tc ? 1 : a.splits) * n_tokens * N);
 }
 
 int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t hidden, const void* w_kva,
@@ -310,15 +351,19 @@ int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32
     if (int rc = device_ok()) return rc;
     const int N = dims->kv_lora_rank + dims->rope_dim;
     const AppendPlan ap = append_plan(n_tokens, hidden, N);
-    const int splits = ap.splits;
+    const int splits = ap.tc ? 1 : ap.splits;  // partials the epilogue sums
     float* part = static_cast<float*>(workspace);
     cudaStream_t st = as_stream(stream);
     if (ap.tc) {
         if (!aligned(x, 16) || !aligned(w_kva, 16)) return MLA_ERR_INVALID_ARG;
-        dim3 g1(N / kApTc, (n_tokens + kApTc - 1) / kApTc, splits);
-        if (int rc = launch(append_gemm_tc_kernel, g1, 128, 0, st, static_cast<const uint16_t*>(x),
-                                                  static_cast<const uint16_t*>(w_kva), part, n_tokens, hidden, N,
-                                                  ap.k_per_split)) return rc;
+        CUtensorMap tm_x, tm_w;
+        if (int rc = encode_2d(&tm_x, x, hidden, n_tokens, tc05::kRows)) return rc;
+        if (int rc = encode_2d(&tm_w, w_kva, N, hidden, 64)) return rc;
+        const size_t smem = tc05::append_smem();
+        if (int rc = ensure_smem(tc05::append_kernel, smem)) return rc;
+        const dim3 grid(N / 64, (n_tokens + tc05::kRows - 1) / tc05::kRows, ap.splits);
+        if (int rc = launch_cluster(tc05::append_kernel, grid, tc05::kThreads, smem, st, dim3(1, 1, ap.splits), tm_x,
+                                    tm_w, n_tokens, N, hidden / 64, ap.k_per_split, ap.splits, part)) return rc;
     } else {
         dim3 g1((N + kApTileN - 1) / kApTileN, (n_tokens + kApTileT - 1) / kApTileT, splits);
         if (int rc = launch(append_gemm_kernel, g1, 256, 0, st, static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w_kva),
@@ -365,6 +410,12 @@ static void record_hook(void* ev, cudaStream_t st) {
         cudaEventRecord(static_cast<cudaEvent_t>(ev), st);
 }
 
+// The attention launch waits for the caller's cache-ready event, if any.
+static int wait_hook(void* ev, cudaStream_t st) {
+    if (!ev) return MLA_OK;
+    return cudaStreamWaitEvent(st, static_cast<cudaEvent_t>(ev), 0) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int32_t batch, int32_t q_len,
                const void* pool, int64_t num_blocks, const int32_t* block_table, int32_t max_blocks_per_seq,
                const int32_t* context_lens, int32_t max_context_len, const void* w_uk, const void* w_uv,
@@ -406,9 +457,9 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         if (int rc = encode_2d(&tm_qn, q_nope, static_cast<uint64_t>(H) * dims->qk_nope_dim, G, tc05::kRows)) return rc;
         if (int rc = encode_2d(&tm_wuk, w_uk, dc, static_cast<uint64_t>(H) * dims->qk_nope_dim, dims->qk_nope_dim))
             return rc;
-        const size_t smem = tc05::absorb_smem(dims->qk_nope_dim, dc);
+        const size_t smem = tc05::absorb_smem(dims->qk_nope_dim);
         if (int rc = ensure_smem(tc05::absorb_kernel, smem)) return rc;
-        if (int rc = launch(tc05::absorb_kernel, dim3(H, (G + tc05::kRows - 1) / tc05::kRows), tc05::kThreads, smem, st,
+        if (int rc = launch(tc05::absorb_kernel, dim3(H, (G + tc05::kRows - 1) / tc05::kRows, dc / 256), tc05::kThreads, smem, st,
             tm_qn, tm_wuk, static_cast<const uint16_t*>(q_pe), G, H, dims->qk_nope_dim, dc, dr, q)) return rc;
     } else if (tc) {
         const size_t smem = absorb_tc_smem(dims->qk_nope_dim);
@@ -448,6 +499,7 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         PP.q_len = q_len;
         PP.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
         if (int rc = ensure_smem(pair::pair_decode_kernel, pair::kSmemBytes)) return rc;
+        if (int rc = wait_hook(opts ? opts->cache_ready : nullptr, st)) return rc;
         record_hook(opts ? opts->event_attn_begin : nullptr, st);
         if (int rc = launch(pair::pair_decode_kernel, 2 * L.workers, pair::kThreads, pair::kSmemBytes, st, tm_q, tm_k3, tm_k2, tm_v, PP)) return rc;
         if (int rc = launch_status()) return rc;
@@ -475,13 +527,27 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     P.scale = dims->softmax_scale;
     const size_t gsmem = generic_decode_smem(dc, dr);
     if (int rc = ensure_smem(generic_decode_kernel, gsmem)) return rc;
+    if (int rc = wait_hook(opts ? opts->cache_ready : nullptr, st)) return rc;
     record_hook(opts ? opts->event_attn_begin : nullptr, st);
     if (int rc = launch(generic_decode_kernel, dim3(L.workers, (H + kGenHeads - 1) / kGenHeads), kGenThreads, gsmem, st, P)) return rc;
     if (int rc = launch_status()) return rc;
     record_hook(opts ? opts->event_attn_end : nullptr, st);
     }
 
-    if (tc05) {
+    // the fused merge + up-projection takes bf16 partials, d_v = 128 and at most
+    // 64 * kMuvMaxBox partial slots per block of 64 groups (<= 64 + workers - 1)
+    const int muv_box = static_cast<int>((std::min<int64_t>(G, tc05::kMuvRows) + L.workers - 1 + 63) / 64);
+    if (tc05 && L.kernel == kKernelPair && dims->v_head_dim == tc05::kMuvDv && muv_box <= tc05::kMuvMaxBox) {
+        CUtensorMap tm_wuv, tm_p;
+        if (int rc = encode_2d(&tm_wuv, w_uv, dc, static_cast<uint64_t>(H) * tc05::kMuvDv, tc05::kMuvDv)) return rc;
+        if (int rc = encode_parts(&tm_p, o_part, dc, H, L.max_parts)) return rc;
+        const size_t smem = tc05::merge_uv_smem(muv_box);
+        if (int rc = ensure_smem(tc05::merge_uv_kernel, smem)) return rc;
+        if (int rc = launch(tc05::merge_uv_kernel, dim3(H, (G + tc05::kMuvRows - 1) / tc05::kMuvRows),
+                            tc05::kMuvThreads, smem, st, tm_wuv, tm_p, lse_part, part_offsets, G, H, dc, muv_box,
+                            static_cast<uint16_t*>(out)))
+            return rc;
+    } else if (tc05) {
         // merge into bf16 o_lat (the absorbed queries are dead once the attention is done:
         // o_lat reuses their space), then the up-projection
         uint16_t* o_lat = q;

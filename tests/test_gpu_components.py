@@ -78,7 +78,8 @@ def _append_case(n_seqs, per_seq, hidden, seed):
     return w
 
 
-@pytest.mark.parametrize("n_seqs,per_seq,hidden", [(3, 1, 256), (5, 4, 7168), (16, 4, 7168), (2, 40, 512)])
+@pytest.mark.parametrize("n_seqs,per_seq,hidden", [(3, 1, 256), (5, 4, 7168), (16, 4, 7168), (2, 40, 512),
+                                                   (3, 50, 320), (10, 110, 512)])
 def test_append_matches_oracle_and_touches_only_its_rows(n_seqs, per_seq, hidden):
     L = _lib()
     w = _append_case(n_seqs, per_seq, hidden, 31 + n_seqs)

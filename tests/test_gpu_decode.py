@@ -168,6 +168,66 @@ def test_graph_replay_matches_direct_launches(kernel):
         assert ev[0].elapsed_time(ev[1]) > 0.0
 
 
+def test_append_on_a_side_stream_with_cache_ready():
+    """The append may run on another stream: the decode's attention waits for the
+    cache_ready event, directly and inside a captured graph, and gives the same
+    bits as append-then-decode on one stream (the appended rows start as NaN, so
+    an attention that did not wait would read them)."""
+    L = _lib()
+    w = I.scaled(I.WORKLOADS["v3_b16_sq4_l16k_append"], batch=3, q_len=2, length=700, name="side_append", seed=57)
+    data = build(w, fill=float("nan"))
+    B, Sq, max_len = w.batch, w.q_len, int(data["lengths"].max())
+
+    def fresh():
+        dd = to_device(data)
+        out = torch.zeros(B, Sq, w.dims.num_heads, w.dims.v_head_dim, dtype=torch.bfloat16, device="cuda")
+        return dd, out
+
+    def append(dd, stream=None):
+        ap = dd["append"]
+        L.append_kv(w.dims, ap["x"], ap["w_kva"], ap["seq_ids"], ap["positions"], dd["table"], dd["pool"],
+                    stream=stream)
+
+    def decode(dd, out, ready=None):
+        L.decode(w.dims, w.softmax_scale, dd["q_nope"], dd["q_pe"], dd["pool"], dd["table"], dd["lengths"],
+                 max_len, dd["w_uk"], dd["w_uv"], out=out, cache_ready=ready)
+
+    dd, out = fresh()
+    append(dd)
+    decode(dd, out)
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    serial = out.float().cpu().numpy()
+    ids = [0, 2]
+    check(serial, oracle_out(w, data, batch_ids=ids, pool=oracle_append_pool(w, data)), ids=ids)
+
+    side, fork, ready = torch.cuda.Stream(), torch.cuda.Event(), torch.cuda.Event()
+    fork.record()
+    ready.record()
+
+    def step(dd, out):
+        fork.record(torch.cuda.current_stream())
+        side.wait_event(fork)
+        append(dd, stream=side)
+        ready.record(side)
+        decode(dd, out, ready)
+
+    dd, out = fresh()
+    step(dd, out)
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    np.testing.assert_array_equal(out.float().cpu().numpy(), serial)
+
+    dd, out = fresh()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step(dd, out)
+    g.replay()
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    np.testing.assert_array_equal(out.float().cpu().numpy(), serial)
+
+
 # ---------------------------------------------------------------- full size
 def _sample(w, k):
     g = torch.Generator().manual_seed(w.seed + 77)
