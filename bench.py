@@ -132,9 +132,10 @@ def roofline(bytes_, flops, seconds, peaks):
 # turns the reported traffic into null until a new capture is recorded here.
 KERNEL_SOURCES = ("decode_pair.cuh", "plan.cuh", "sm100.cuh", "common.cuh")
 TRAFFIC = {
-    # profiles/pair_decode_kernel_v3_b64_l1k_8k.md (ncu --set full, one launch)
-    "v3_b64_l1k_8k": {"bytes": 347966720 + 11035904,
-                      "sources_sha256": "4be4c9561fbf8a6e0d4af19b816923ef35c5842676cbac244ae794675d7c4866"},
+    # profiles/pair_decode_kernel_v3_b64_l1k_8k.md (ncu launch list of one step, the attention launch:
+    # dram__bytes_read.sum + dram__bytes_write.sum)
+    "v3_b64_l1k_8k": {"bytes": 357413632 + 6190336,
+                      "sources_sha256": "4aa3b05c0112b687b2e42b853cb84ab7862955e617074b06f879e28b79ec3953"},
 }
 
 
@@ -395,15 +396,25 @@ def run_ours(args, w):
     ea = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
     ea[0].record()
     ea[1].record()  # the handles exist before any capture
-    graph = None
-    if args.graph:
-        # the step's launches are replayed from one CUDA graph (no host launch gaps)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            step(events=ea)
-        graph.replay()
+    # The timed region is K steps without timing events inside them: an event
+    # recorded between two launches stands between them in the graph and takes
+    # away their programmatic overlap. The attention kernel's time comes from a
+    # second pass of K steps right after it, whose steps record events right
+    # before and after its launch.
+    def capture(events):
+        if not args.graph:
+            return lambda: step(events=events)
+        g = torch.cuda.CUDAGraph()  # the step's launches replayed from one graph (no host launch gaps)
+        with torch.cuda.graph(g):
+            step(events=events)
+        g.replay()
         torch.cuda.synchronize(device)
-    run = graph.replay if graph is not None else (lambda: step(events=ea))
+        graphs.append(g)
+        return g.replay
+
+    graphs = []
+    run, run_attn = capture(None), capture(ea)
+    ev_attn = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     attn_ms = []
     barrier(device)
     torch.cuda.synchronize(device)
@@ -412,12 +423,20 @@ def run_ours(args, w):
         ev[k][0].record()
         run()
         ev[k][1].record()
-        ev[k][1].synchronize()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    for k in range(K):  # the attention pass (after the timed region)
+        flush.zero_()
+        ev_attn[k][0].record()
+        run_attn()
+        ev_attn[k][1].record()
+        ev_attn[k][1].synchronize()
         attn_ms.append(ea[0].elapsed_time(ea[1]))
     torch.cuda.synchronize(device)
     barrier(device)
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
+    step_ms_attn_pass = [a.elapsed_time(b) for a, b in ev_attn]
     assert lib.device_error() == 0, "device fault during the timed steps"
 
     # end to end through the public API with host buffers (pinned)
@@ -480,6 +499,8 @@ def run_ours(args, w):
                    "launch": "CUDA graph replay" if args.graph else "direct launches"},
         "roofline": roof,
         "attn_us": round(t_attn * 1e3, 2),
+        "attn_timing": "CUDA events around the attention launch, in a second pass of K steps "
+                       f"(step time in that pass {statistics.mean(step_ms_attn_pass) * 1e3:.2f} us)",
         "attn_hbm_gbs": round(attn_gbs, 1), "attn_tflops": round(attn_tfs, 2),
         "cache_tokens_per_s": round(world * tot["T"] / (t_step / 1e3), 1),
         "decode_tokens_per_s": round(world * tot["G"] / (t_step / 1e3), 1),
@@ -496,6 +517,31 @@ def run_ours(args, w):
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, st["lengths"].tolist(), args.cpu_seconds)
     return line
+
+
+def profile_step(args, w):
+    """One direct-launch step of the workload between cudaProfilerStart and
+    cudaProfilerStop (for `ncu --profile-from-start off`), after the cache fill
+    and the warm-up steps, with L2 flushed before it. Prints nothing."""
+    import torch
+
+    from mla_latent_kv_29_b200 import lib
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    lib.load()
+    st = setup_gpu(w, device, 0)
+    step = make_step(w, st, args.kernel, overlap=args.overlap)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device).zero_()
+    torch.cuda.synchronize(device)
+    torch.cuda.profiler.start()
+    step()
+    torch.cuda.synchronize(device)
+    torch.cuda.profiler.stop()
+    assert lib.device_error() == 0, "device fault in the profiled step"
 
 
 def run_reference(args, w):
@@ -544,6 +590,8 @@ def main(argv=None):
                     help="run the append on a side stream beside the decode's query-side launches")
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="replay each step from a captured CUDA graph")
+    ap.add_argument("--profile-step", action="store_true",
+                    help="run one step between profiler start/stop (for ncu --profile-from-start off) and exit")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -554,6 +602,9 @@ def main(argv=None):
     import dataclasses
 
     w = dataclasses.replace(w, seed=rank_seed(w.seed, rank))
+    if args.profile_step:
+        profile_step(args, w)
+        return
     line = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
     if line is not None:
         print(json.dumps(line), flush=True)

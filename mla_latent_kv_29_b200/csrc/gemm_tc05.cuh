@@ -504,11 +504,21 @@ __global__ void __launch_bounds__(kThreads) absorb_kernel(const __grid_constant_
         }
         ptx::mma_commit_1(done);
     }
-    // epilogue: thread t = TMEM lane t = token row g0 + t
+    // epilogue: thread t = TMEM lane t = token row g0 + t. The RoPE part of the
+    // query row (CTAs with z = 0) is requested before the wait for the MMAs.
+    const int g = g0 + static_cast<int>(threadIdx.x);
+    constexpr int kPe = 8;  // d_r / 8 uint4 pieces, d_r <= 64 on this path
+    uint4 pe[kPe];
+    const bool copy_pe = g < G && z == 0;
+    if (copy_pe) {
+        const uint4* src = reinterpret_cast<const uint4*>(q_pe + (static_cast<int64_t>(g) * H + h) * dr);
+#pragma unroll
+        for (int i = 0; i < kPe; ++i)
+            if (i < dr / 8) pe[i] = src[i];
+    }
     const bool ok = ptx::mbar_wait(done, 0, abort);
     ptx::tc_fence_after();
     if (ok) {
-        const int g = g0 + static_cast<int>(threadIdx.x);
         const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         const int D = dc + dr;
 #pragma unroll 1  // one-shot code: kept short for a cold instruction cache
@@ -525,10 +535,11 @@ __global__ void __launch_bounds__(kThreads) absorb_kernel(const __grid_constant_
                                         ptx::bf16x2(v[8 * i + 6], v[8 * i + 7]));
             }
         }
-        if (g < G && z == 0) {  // the RoPE part of the query row
-            const uint4* src = reinterpret_cast<const uint4*>(q_pe + (static_cast<int64_t>(g) * H + h) * dr);
+        if (copy_pe) {  // the RoPE part of the query row
             uint4* dst = reinterpret_cast<uint4*>(q_out + (static_cast<int64_t>(g) * H + h) * D + dc);
-            for (int i = 0; i < dr / 8; ++i) dst[i] = src[i];
+#pragma unroll
+            for (int i = 0; i < kPe; ++i)
+                if (i < dr / 8) dst[i] = pe[i];
         }
     }
     ptx::tc_fence_before();

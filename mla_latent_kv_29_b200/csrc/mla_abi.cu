@@ -202,11 +202,12 @@ int encode_parts(CUtensorMap* m, const void* base, uint64_t dc, uint64_t H, uint
 }
 
 // The tcgen05 absorb / merge / UV kernels: d_n a multiple of 64 up to 256, d_c
-// a multiple of 256 up to 512, d_r a multiple of 8, d_v a multiple of 16 up
+// a multiple of 256 up to 512, d_r a multiple of 8 up to 64, d_v a multiple of 16 up
 // to 256, and 16-byte aligned operands.
 bool tc05_dims_ok(const mla_dims_t* d) {
     return d->qk_nope_dim % 64 == 0 && d->qk_nope_dim <= 256 && d->kv_lora_rank % 256 == 0 &&
-           d->kv_lora_rank <= 512 && d->rope_dim % 8 == 0 && d->v_head_dim % 16 == 0 && d->v_head_dim <= 256;
+           d->kv_lora_rank <= 512 && d->rope_dim % 8 == 0 && d->rope_dim <= 64 && d->v_head_dim % 16 == 0 &&
+           d->v_head_dim <= 256;
 }
 
 int decode_layout(const mla_dims_t* d, int32_t batch, int32_t q_len, int32_t max_len,
@@ -447,8 +448,10 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     // the tensor-core kernel writes bf16 partials, which only the tensor-core merge reads
     if (L.kernel == kKernelPair && !tc) return MLA_ERR_INVALID_ARG;
 
-    if (int rc = launch(plan_kernel, 1, 1024, 0, st, context_lens, batch, q_len, L.tile, L.workers, hdr, tile_prefix, part_offsets,
-                                    worker_group)) return rc;
+    const size_t plan_smem = sizeof(int32_t) * (static_cast<size_t>(G) + 1);
+    const int32_t prefix_in_smem = plan_smem <= 48 * 1024 ? 1 : 0;
+    if (int rc = launch(plan_kernel, 1, 1024, prefix_in_smem ? plan_smem : 0, st, context_lens, batch, q_len, L.tile,
+                        L.workers, hdr, tile_prefix, part_offsets, worker_group, prefix_in_smem)) return rc;
     if (int rc = launch_status()) return rc;
 
     const bool tc05 = tc && tc05_dims_ok(dims) && aligned(q_pe, 16);

@@ -93,38 +93,49 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
     return r;
 }
 
-// <<<1, 1024>>>. tile_prefix and part_offsets have G + 1 entries,
-// worker_group max_workers entries.
+// <<<1, 1024, smem>>>. tile_prefix and part_offsets have G + 1 entries,
+// worker_group max_workers entries. With smem = 4 (G + 1) bytes of dynamic
+// shared memory (prefix_in_smem) the later passes read the prefix, and the
+// binary searches of group_of_unit run, in shared memory instead of chains of
+// dependent global loads.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ context_lens, int32_t batch,
                                                     int32_t q_len, int32_t tile, int32_t max_workers,
                                                     PlanHeader* __restrict__ hdr,
                                                     int32_t* __restrict__ tile_prefix,
                                                     int32_t* __restrict__ part_offsets,
-                                                    int32_t* __restrict__ worker_group) {
+                                                    int32_t* __restrict__ worker_group, int32_t prefix_in_smem) {
     pdl_wait();
     pdl_trigger();
     __shared__ int32_t warp_tot[32];
     __shared__ int32_t chunk_total;
+    extern __shared__ int32_t s_prefix[];
+    int32_t* tp = prefix_in_smem ? s_prefix : tile_prefix;  // where the later passes read the prefix
     const int32_t G = batch * q_len;
     int32_t carry = 0;
     for (int32_t base = 0; base < G; base += 1024) {
         const int32_t g = base + threadIdx.x;
         const int32_t n = g < G ? group_tiles(context_lens, q_len, g, tile) : 0;
         const int32_t ex = block_exclusive_scan(n, warp_tot, &chunk_total);
-        if (g < G) tile_prefix[g] = carry + ex;
+        if (g < G) {
+            tile_prefix[g] = carry + ex;
+            if (prefix_in_smem) s_prefix[g] = carry + ex;
+        }
         carry += chunk_total;
         __syncthreads();
     }
     const int32_t W = carry > 0 ? carry + kSegUnits * G : 0;
     const int32_t P = W > 0 ? min(max_workers, W) : 0;
-    if (threadIdx.x == 0) tile_prefix[G] = carry;
+    if (threadIdx.x == 0) {
+        tile_prefix[G] = carry;
+        if (prefix_in_smem) s_prefix[G] = carry;
+    }
     __syncthreads();
     carry = 0;
     for (int32_t base = 0; base < G; base += 1024) {
         const int32_t g = base + threadIdx.x;
         int32_t n = 0;
         if (g < G) {
-            const int32_t t0 = tile_prefix[g], t1 = tile_prefix[g + 1];
+            const int32_t t0 = tp[g], t1 = tp[g + 1];
             if (t1 > t0) {
                 const int32_t v0 = t0 + kSegUnits * (g + 1);  // unit of the group's first tile
                 n = worker_of_unit(v0 + (t1 - t0) - 1, W, P) - worker_of_unit(v0, W, P) + 1;
@@ -136,7 +147,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
         __syncthreads();
     }
     for (int32_t p = threadIdx.x; p < P; p += 1024)
-        worker_group[p] = group_of_unit(tile_prefix, G, worker_begin(p, W, P));
+        worker_group[p] = group_of_unit(tp, G, worker_begin(p, W, P));
     if (threadIdx.x == 0) {
         part_offsets[G] = carry;
         hdr->total_units = W;
