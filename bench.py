@@ -94,7 +94,10 @@ def load_peaks():
 
 
 def workload_totals(w, lengths):
-    """Algorithmic units of one decode step (measurement)."""
+    """Algorithmic units of one decode step. Attention: every cached token's
+    576 bf16 values read once plus the absorbed queries; FLOPs 2 H (576 + 512)
+    per visible (query, token) pair. Step: the attention's cache bytes, the
+    W_UK / W_UV / W_kva weights, the new tokens' inputs and the outputs."""
     d = w.dims
     L = [int(v) for v in lengths]
     T = sum(L)  # unique cached tokens read
@@ -134,7 +137,7 @@ KERNEL_SOURCES = ("decode_pair.cuh", "plan.cuh", "sm100.cuh", "common.cuh")
 TRAFFIC = {
     # profiles/pair_decode_kernel_v3_b64_l1k_8k.md (ncu launch list of one step, the attention launch:
     # dram__bytes_read.sum + dram__bytes_write.sum)
-    "v3_b64_l1k_8k": {"bytes": 357413632 + 6190336,
+    "v3_b64_l1k_8k": {"bytes": 354286848 + 6138368,
                       "sources_sha256": "4aa3b05c0112b687b2e42b853cb84ab7862955e617074b06f879e28b79ec3953"},
 }
 

@@ -232,19 +232,24 @@ __global__ void __launch_bounds__(kThreads, 1) uv_kernel(const __grid_constant__
 // W_UV as 2-D [H * d_v rows, d_c columns]) and the slots' columns 64 kb ..
 // (n_box boxes {64 columns, 1 head, 64 slots} of tm_p = the partials as 3-D
 // [slots][H][d_c]), so the stages are in flight together and no warp waits
-// on a chain of dependent loads; thread 0 refills the stage of block kb - 1
-// with block kb + 3 at the top of block kb. The weights exp(lse - max) / sum
-// come first: the slots' lse into shared memory in one round trip, then one
-// warp per group with lanes over its slots. Thread t merges group t / 4,
-// columns 16 (t % 4) .. + 15 of a block.
-// grid (H, ceil(G / 64)); block 256; dynamic smem merge_uv_smem(n_box);
+// on a chain of dependent loads. Warp 8 is the producer: it refills the stage
+// of block kb with block kb + 4 as soon as block kb's MMAs are done, so no
+// merge warp waits on an MMA. The weights exp(lse - max) / sum come first:
+// the slots' lse into shared memory in one round trip, then a thread (or, for
+// fewer than 32 groups, a warp) per group. Merge thread t merges group t / 4,
+// columns 16 (t % 4) .. + 15 of a block; thread 0 issues the MMAs.
+// grid (H, ceil(G / 64)); block 288; dynamic smem merge_uv_smem(n_box);
 // d_v = 128, d_c a multiple of 64 up to 512, P1 - P0 <= 64 n_box, n_box <= 4.
-constexpr int kMuvThreads = 256;
+constexpr int kMuvThreads = 288;       // 8 merge warps + 1 producer warp
+constexpr int kMuvMergeThreads = 256;
 constexpr int kMuvRows = 64;     // groups per CTA (the MMA's N)
 constexpr int kMuvDv = 128;      // the MMA's M
 constexpr int kMuvStages = 4;
 constexpr int kMuvMaxBox = 4;    // slot boxes of 64 per stage at most
 constexpr int kMuvSlotBox = 64 * kBoxBytes;  // 8 KB: 64 slots x 64 columns
+__device__ __forceinline__ void merge_sync() {  // the 8 merge warps only (named barrier 1)
+    asm volatile("bar.sync 1, %0;" ::"n"(kMuvMergeThreads) : "memory");
+}
 __host__ __device__ inline int merge_uv_stage_bytes(int n_box) {
     return n_box * kMuvSlotBox + kMuvDv * kBoxBytes + kMuvRows * kBoxBytes;
 }
@@ -268,10 +273,11 @@ __global__ void __launch_bounds__(kMuvThreads, 1) merge_uv_kernel(const __grid_c
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + 8 * (2 * kMuvStages + 1) + 16);
     int32_t* offs = reinterpret_cast<int32_t*>(smem + off_bar + 256);          // kMuvRows + 1 entries
     float* wgt = reinterpret_cast<float*>(smem + off_bar + 256 + 512);         // per slot of [P0, P1)
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = static_cast<int>(threadIdx.x), warp = t >> 5, lane = t & 31;
+    const bool producer = warp == kMuvMergeThreads / 32;
     const int h = blockIdx.x, g0 = blockIdx.y * kMuvRows;
     const int R = min(kMuvRows, G - g0);
-    if (threadIdx.x == 0) {
+    if (t == 0) {
         *abort = 0;
         for (int i = 0; i <= 2 * kMuvStages; ++i) ptx::mbar_init(bar_addr(smem, off_bar, i), 1);
         ptx::fence_mbar_init();
@@ -284,7 +290,7 @@ __global__ void __launch_bounds__(kMuvThreads, 1) merge_uv_kernel(const __grid_c
     }
     // part_offsets come from the plan launch, which finished before the attention
     // launch (this one's predecessor) could pass its own dependency wait
-    if (static_cast<int>(threadIdx.x) <= R) offs[threadIdx.x] = part_offsets[g0 + threadIdx.x];
+    if (t <= R) offs[t] = part_offsets[g0 + t];
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -292,114 +298,139 @@ __global__ void __launch_bounds__(kMuvThreads, 1) merge_uv_kernel(const __grid_c
     const int32_t P0 = offs[0], NP = offs[R] - P0;
     const int nb = NP > 0 ? (NP + 63) / 64 : 0;  // slot boxes this CTA needs
     const bool fits = nb <= n_box;
-    if (!fits && threadIdx.x == 0) record_status(MLA_ERR_DEVICE_FAULT);
-    auto stage_tx = [&]() { return static_cast<uint32_t>(nb * kMuvSlotBox + kMuvDv * kBoxBytes); };
-    if (threadIdx.x == 0) {  // the weights are not written by earlier launches: request them now
-        for (int kb = 0; kb < min(nk, kMuvStages); ++kb) {
-            const uint32_t full = bar_addr(smem, off_bar, kb);
-            ptx::mbar_arrive_expect_tx_local(full, fits ? stage_tx() : kMuvDv * kBoxBytes);
-            ptx::tma_load_2d(ptx::smem_u32(smem + kb * stage_bytes + off_w), &tm_w, 64 * kb, h * kMuvDv, full);
-        }
-    }
-    pdl_wait();
-    pdl_trigger();
+    if (!fits && t == 0) record_status(MLA_ERR_DEVICE_FAULT);
+    const uint32_t stage_tx = fits ? static_cast<uint32_t>(nb * kMuvSlotBox + kMuvDv * kBoxBytes)
+                                   : static_cast<uint32_t>(kMuvDv * kBoxBytes);
+    auto load_w = [&](int kb, uint32_t full) {
+        ptx::tma_load_2d(ptx::smem_u32(smem + (kb % kMuvStages) * stage_bytes + off_w), &tm_w, 64 * kb, h * kMuvDv,
+                         full);
+    };
     auto load_slots = [&](int kb, uint32_t full) {
         if (!fits) return;
         for (int b = 0; b < nb; ++b)
             ptx::tma_load_3d(ptx::smem_u32(smem + (kb % kMuvStages) * stage_bytes + b * kMuvSlotBox), &tm_p, 64 * kb, h,
                              P0 + 64 * b, full);
     };
-    if (threadIdx.x == 0)
-        for (int kb = 0; kb < min(nk, kMuvStages); ++kb) load_slots(kb, bar_addr(smem, off_bar, kb));
-
-    // ---- weights. This code runs once per CTA, so it is kept short (loops, not
-    // unrolled copies): on a cold instruction cache every new line of code costs
-    // a round trip to L2. (1) every slot's lse into shared memory, one round trip.
-    if (fits)
-        for (int i = threadIdx.x; i < NP; i += kMuvThreads) wgt[i] = lse_part[static_cast<int64_t>(P0 + i) * H + h];
-    __syncthreads();
-    // (2) per group (a warp, lanes over its slots): max, sum, then the normalised
-    // weights in place (each lane rewrites only the slots it read)
-    if (fits) {
-#pragma unroll 1
-        for (int jj = warp; jj < R; jj += kMuvThreads / 32) {
-            const int32_t a = offs[jj] - P0, b = offs[jj + 1] - P0;
-            float M = -INFINITY;
-            for (int32_t i = a + lane; i < b; i += 32) M = fmaxf(M, wgt[i]);
-            M = warp_max(M);
-            float den = 0.f;
-            if (M != -INFINITY)
-                for (int32_t i = a + lane; i < b; i += 32) den += wgt[i] == -INFINITY ? 0.f : __expf(wgt[i] - M);
-            den = warp_sum(den);
-            const float inv = den > 0.f ? __fdividef(1.f, den) : 0.f;
-            for (int32_t i = a + lane; i < b; i += 32) {
-                const float l = wgt[i];
-                wgt[i] = l == -INFINITY || M == -INFINITY ? 0.f : __expf(l - M) * inv;
-            }
+    if (producer && lane == 0) {  // the weights are not written by earlier launches: request them now
+        for (int kb = 0; kb < min(nk, kMuvStages); ++kb) {
+            ptx::mbar_arrive_expect_tx_local(bar_addr(smem, off_bar, kb), stage_tx);
+            load_w(kb, bar_addr(smem, off_bar, kb));
         }
     }
-    __syncthreads();
+    pdl_wait();
+    pdl_trigger();
 
-    // ---- per 64-column block: merge into B, then 4 MMAs
-    const int j = static_cast<int>(threadIdx.x) >> 2, q = static_cast<int>(threadIdx.x) & 3;
-    const int32_t s0 = j < R ? offs[j] - P0 : 0, s1 = j < R ? offs[j + 1] - P0 : 0;
-#pragma unroll 1
-    for (int kb = 0; kb < nk; ++kb) {
-        const int st = kb % kMuvStages;
-        uint8_t* stage = smem + st * stage_bytes;
-        if (threadIdx.x == 0 && kb >= 1 && kb - 1 + kMuvStages < nk) {
-            // refill the previous block's stage with block kb + 3 once its MMAs are done
-            const int ps = (kb - 1) % kMuvStages;
-            if (ptx::mbar_wait(bar_addr(smem, off_bar, kMuvStages + ps), ((kb - 1) / kMuvStages) & 1, abort)) {
-                const uint32_t full = bar_addr(smem, off_bar, ps);
-                ptx::mbar_arrive_expect_tx_local(full, fits ? stage_tx() : kMuvDv * kBoxBytes);
-                ptx::tma_load_2d(ptx::smem_u32(smem + ps * stage_bytes + off_w), &tm_w, 64 * (kb - 1 + kMuvStages),
-                                 h * kMuvDv, full);
-                load_slots(kb - 1 + kMuvStages, full);
+    if (producer) {
+        // ---- producer: the slots of the first stages, then each later block into the
+        // stage its block kb - 4 leaves once that block's MMAs are done
+        if (lane == 0) {
+            for (int kb = 0; kb < min(nk, kMuvStages); ++kb) load_slots(kb, bar_addr(smem, off_bar, kb));
+            for (int kb = kMuvStages; kb < nk; ++kb) {
+                const int st = kb % kMuvStages;
+                if (!ptx::mbar_wait(bar_addr(smem, off_bar, kMuvStages + st), ((kb / kMuvStages) - 1) & 1, abort))
+                    break;
+                const uint32_t full = bar_addr(smem, off_bar, st);
+                ptx::mbar_arrive_expect_tx_local(full, stage_tx);
+                load_w(kb, full);
+                load_slots(kb, full);
             }
         }
-        const bool ok = ptx::mbar_wait(bar_addr(smem, off_bar, st), (kb / kMuvStages) & 1, abort);
-        if (j < R) {
-            float acc[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-            if (ok && fits) {
+    } else {
+        // ---- weights (merge warps). This code runs once per CTA, so it is kept short
+        // (loops, not unrolled copies): on a cold instruction cache every new line of
+        // code costs a round trip to L2. (1) every slot's lse into shared memory.
+        if (fits)
+            for (int i = t; i < NP; i += kMuvMergeThreads) wgt[i] = lse_part[static_cast<int64_t>(P0 + i) * H + h];
+        merge_sync();
+        // (2) per group: max, sum, then the normalised weights in place. Many groups:
+        // a thread each; few (long groups, small batches): a warp each, lanes over slots.
+        if (fits && R >= 32) {
+            if (t < R) {
+                const int32_t a = offs[t] - P0, b = offs[t + 1] - P0;
+                float M = -INFINITY;
+                for (int32_t i = a; i < b; ++i) M = fmaxf(M, wgt[i]);
+                float den = 0.f;
+                if (M != -INFINITY)
+                    for (int32_t i = a; i < b; ++i) den += wgt[i] == -INFINITY ? 0.f : __expf(wgt[i] - M);
+                const float inv = den > 0.f ? __fdividef(1.f, den) : 0.f;
+                for (int32_t i = a; i < b; ++i) {
+                    const float l = wgt[i];
+                    wgt[i] = l == -INFINITY || M == -INFINITY ? 0.f : __expf(l - M) * inv;
+                }
+            }
+        } else if (fits) {
 #pragma unroll 1
-                for (int32_t i = s0; i < s1; ++i) {  // slot i: box i / 64, swizzled row i % 64
-                    const float w = wgt[i];
-                    const uint8_t* row = stage + (i >> 6) * kMuvSlotBox + (i & 63) * kBoxBytes;
+            for (int jj = warp; jj < R; jj += kMuvMergeThreads / 32) {
+                const int32_t a = offs[jj] - P0, b = offs[jj + 1] - P0;
+                float M = -INFINITY;
+                for (int32_t i = a + lane; i < b; i += 32) M = fmaxf(M, wgt[i]);
+                M = warp_max(M);
+                float den = 0.f;
+                if (M != -INFINITY)
+                    for (int32_t i = a + lane; i < b; i += 32) den += wgt[i] == -INFINITY ? 0.f : __expf(wgt[i] - M);
+                den = warp_sum(den);
+                const float inv = den > 0.f ? __fdividef(1.f, den) : 0.f;
+                for (int32_t i = a + lane; i < b; i += 32) {  // each lane rewrites only the slots it read
+                    const float l = wgt[i];
+                    wgt[i] = l == -INFINITY || M == -INFINITY ? 0.f : __expf(l - M) * inv;
+                }
+            }
+        }
+        merge_sync();
+
+        // ---- per 64-column block: merge into B, then 4 MMAs (thread 0)
+        const int j = t >> 2, q = t & 3;
+        const int32_t s0 = j < R ? offs[j] - P0 : 0, s1 = j < R ? offs[j + 1] - P0 : 0;
+#pragma unroll 1
+        for (int kb = 0; kb < nk; ++kb) {
+            const int st = kb % kMuvStages;
+            uint8_t* stage = smem + st * stage_bytes;
+            const bool ok = ptx::mbar_wait(bar_addr(smem, off_bar, st), (kb / kMuvStages) & 1, abort);
+            if (j < R) {
+                float acc[16];
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const uint4 u = *reinterpret_cast<const uint4*>(row + (((2 * q + c) ^ (i & 7)) << 4));
-                        const uint32_t x[4] = {u.x, u.y, u.z, u.w};
+                for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+                if (ok && fits) {
+#pragma unroll 1
+                    for (int32_t i = s0; i < s1; ++i) {  // slot i: box i / 64, swizzled row i % 64
+                        const float w = wgt[i];
+                        const uint8_t* row = stage + (i >> 6) * kMuvSlotBox + (i & 63) * kBoxBytes;
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            acc[8 * c + 2 * k] = fmaf(w, __uint_as_float(x[k] << 16), acc[8 * c + 2 * k]);
-                            acc[8 * c + 2 * k + 1] = fmaf(w, __uint_as_float(x[k] & 0xffff0000u), acc[8 * c + 2 * k + 1]);
+                        for (int c = 0; c < 2; ++c) {
+                            const uint4 u = *reinterpret_cast<const uint4*>(row + (((2 * q + c) ^ (i & 7)) << 4));
+                            const uint32_t x[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                acc[8 * c + 2 * k] = fmaf(w, __uint_as_float(x[k] << 16), acc[8 * c + 2 * k]);
+                                acc[8 * c + 2 * k + 1] =
+                                    fmaf(w, __uint_as_float(x[k] & 0xffff0000u), acc[8 * c + 2 * k + 1]);
+                            }
                         }
                     }
                 }
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+                    *reinterpret_cast<uint4*>(stage + off_bm + j * kBoxBytes + (((2 * q + c) ^ (j & 7)) << 4)) =
+                        make_uint4(ptx::bf16x2(acc[8 * c], acc[8 * c + 1]), ptx::bf16x2(acc[8 * c + 2], acc[8 * c + 3]),
+                                   ptx::bf16x2(acc[8 * c + 4], acc[8 * c + 5]),
+                                   ptx::bf16x2(acc[8 * c + 6], acc[8 * c + 7]));
             }
+            ptx::fence_proxy_async_smem();  // B was written through the generic proxy
+            merge_sync();
+            if (t == 0) {
+                ptx::tc_fence_after();
+                constexpr uint32_t idesc = ptx::idesc_bf16(kMuvDv, kMuvRows, false, false);
+                const uint64_t da = ptx::smem_desc_sw128(ptx::smem_u32(stage + off_w), 16, 1024);
+                const uint64_t db = ptx::smem_desc_sw128(ptx::smem_u32(stage + off_bm), 16, 1024);
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
-                *reinterpret_cast<uint4*>(stage + off_bm + j * kBoxBytes + (((2 * q + c) ^ (j & 7)) << 4)) =
-                    make_uint4(ptx::bf16x2(acc[8 * c], acc[8 * c + 1]), ptx::bf16x2(acc[8 * c + 2], acc[8 * c + 3]),
-                               ptx::bf16x2(acc[8 * c + 4], acc[8 * c + 5]), ptx::bf16x2(acc[8 * c + 6], acc[8 * c + 7]));
+                for (int kk = 0; kk < 4; ++kk) ptx::mma_bf16_1(tmem, da + 2 * kk, db + 2 * kk, idesc, (kb | kk) != 0);
+                ptx::mma_commit_1(bar_addr(smem, off_bar, kMuvStages + st));
+            }
         }
-        ptx::fence_proxy_async_smem();  // B was written through the generic proxy
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            ptx::tc_fence_after();
-            constexpr uint32_t idesc = ptx::idesc_bf16(kMuvDv, kMuvRows, false, false);
-            const uint64_t da = ptx::smem_desc_sw128(ptx::smem_u32(stage + off_w), 16, 1024);
-            const uint64_t db = ptx::smem_desc_sw128(ptx::smem_u32(stage + off_bm), 16, 1024);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) ptx::mma_bf16_1(tmem, da + 2 * kk, db + 2 * kk, idesc, (kb | kk) != 0);
-            ptx::mma_commit_1(bar_addr(smem, off_bar, kMuvStages + st));
-        }
+        if (t == 0) ptx::mma_commit_1(bar_addr(smem, off_bar, 2 * kMuvStages));
     }
-    if (threadIdx.x == 0) ptx::mma_commit_1(bar_addr(smem, off_bar, 2 * kMuvStages));
     __syncwarp();
+    __syncthreads();
 
     // ---- epilogue: thread t < 128 = TMEM lane t = output column d; TMEM column j = group g0 + j.
     // D goes through shared memory (stage 0, free once every MMA is done) as bf16 [64 groups][128]
@@ -408,20 +439,18 @@ __global__ void __launch_bounds__(kMuvThreads, 1) merge_uv_kernel(const __grid_c
     ptx::tc_fence_after();
     uint16_t* stg = reinterpret_cast<uint16_t*>(smem);
     if (warp < 4) {
-        const int d = static_cast<int>(threadIdx.x);
 #pragma unroll 1
         for (int c0 = 0; c0 < R; c0 += 32) {
             float v[32];
             ptx::tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                stg[(c0 + i) * kMuvDv + d] = static_cast<uint16_t>(ptx::bf16x2(v[i], 0.f) & 0xffffu);
+            for (int i = 0; i < 32; ++i) stg[(c0 + i) * kMuvDv + t] = static_cast<uint16_t>(ptx::bf16x2(v[i], 0.f) & 0xffffu);
         }
     }
     __syncthreads();
     if (done) {
-        for (int idx = threadIdx.x; idx < R * (kMuvDv / 8); idx += kMuvThreads) {
+        for (int idx = t; idx < R * (kMuvDv / 8); idx += kMuvThreads) {
             const int jj = idx / (kMuvDv / 8), c8 = idx % (kMuvDv / 8);
             *reinterpret_cast<uint4*>(out + (static_cast<int64_t>(g0 + jj) * H + h) * kMuvDv + 8 * c8) =
                 *reinterpret_cast<const uint4*>(stg + jj * kMuvDv + 8 * c8);
