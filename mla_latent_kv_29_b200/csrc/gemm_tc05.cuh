@@ -508,7 +508,11 @@ __global__ void __launch_bounds__(kThreads) absorb_kernel(const __grid_constant_
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    pdl_wait();
+    // This kernel reads only the caller's inputs and writes only the query region
+    // of the workspace. It follows the plan launch, which started it only after its
+    // own dependency wait (so all earlier work is complete) and which it does not
+    // read: the whole kernel runs beside the plan, and its dependency wait comes
+    // last, so that its completion still implies the plan's.
     pdl_trigger();
     const uint32_t full = bar_addr(smem, off_bar, 0), done = bar_addr(smem, off_bar, 1);
 
@@ -577,20 +581,23 @@ __global__ void __launch_bounds__(kThreads) absorb_kernel(const __grid_constant_
         ptx::tc_fence_after();
         ptx::tmem_dealloc_1(tmem, 256);
     }
+    pdl_wait();
 }
 
 // --------------------------------------------------------------- append
 // kv[t, n0 .. n0 + 63] = x[t, :] W_kva[:, n0 .. n0 + 63] (fp32) for t in
 // [m0, m0 + 128): the joint down-projection of the cache append
 // (kv_a_proj_with_mqa, "MLA架构：低秩注意力机制优化LLM显存与计算效率" 2.2).
-// The hidden dimension is split over the S CTAs of a cluster (grid z,
-// cluster (1, 1, S)); each streams its K-blocks of 64 through a ring of
-// (x box {64, 128 rows}, W box {64 columns, 64 rows}) stages into a
-// M 128 x N 64 TMEM accumulator, the S partial tiles meet in shared memory
-// and CTA r of the cluster sums rows [r 128 / S, (r + 1) 128 / S) over the
-// cluster (distributed shared memory) and stores them. S = 1 stores directly.
+// The hidden dimension is split over the S * Z CTAs along grid z, in Z
+// clusters of S (cluster (1, 1, S)); each CTA streams its K-blocks of 64
+// through a ring of (x box {64, 128 rows}, W box {64 columns, 64 rows})
+// stages into a M 128 x N 64 TMEM accumulator, the S partial tiles of a
+// cluster meet in shared memory and CTA r of the cluster sums rows
+// [r 128 / S, (r + 1) 128 / S) over the cluster (distributed shared memory)
+// and stores them into partial z / S of kv ([Z][T][N]; the epilogue adds the
+// Z partials). S = 1 stores directly.
 // tm_x: x as 2-D [T rows, hidden columns]; tm_w: W_kva as 2-D [hidden rows,
-// N columns], box {64, 64} (MN-major B). grid (N / 64, ceil(T / 128), S);
+// N columns], box {64, 64} (MN-major B). grid (N / 64, ceil(T / 128), S Z);
 // block 128; dynamic smem append_smem().
 constexpr int kApStages = 6;
 constexpr int kApStageBytes = kRows * kBoxBytes + 64 * kBoxBytes;  // 24 KB
@@ -616,6 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1) append_kernel(const __grid_consta
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + 8 * (2 * kApStages + 1) + 16);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * 64, m0 = blockIdx.y * kRows, z = blockIdx.z;
+    kv += static_cast<int64_t>(z / S) * T * N;  // this cluster's partial
     const int kb0 = z * k_blocks_per_cta;
     const int nk = max(0, min(k_blocks_per_cta, k_blocks - kb0));  // this CTA's K-blocks of 64
     if (threadIdx.x == 0) {

@@ -260,24 +260,32 @@ bool tc_gemm_dims_ok(const mla_dims_t* d) {
 }
 
 // ---- append split-K plan ----------------------------------------------
-// tc: the tcgen05 GEMM (N and hidden multiples of 64), its K split over a
-// cluster of `splits` CTAs that reduce on chip, so the epilogue sees one
-// partial; otherwise the CUDA-core GEMM writes `splits` partials.
+// tc: the tcgen05 GEMM (N and hidden multiples of 64), its K split over
+// `cluster` * `splits` CTAs: `splits` clusters of `cluster` CTAs that reduce
+// on chip, so the epilogue sums `splits` partials; otherwise the CUDA-core
+// GEMM writes `splits` partials.
 struct AppendPlan {
     bool tc;
-    int splits, k_per_split;
+    int splits, k_per_split, cluster;
 };
 
 AppendPlan append_plan(int32_t n_tokens, int32_t hidden, int32_t N) {
     AppendPlan a;
     a.tc = (N % 64 == 0) && (hidden % 64 == 0);
+    a.cluster = 1;
     if (a.tc) {
         const int64_t tiles = static_cast<int64_t>(N / 64) * ((n_tokens + tc05::kRows - 1) / tc05::kRows);
         const int k_blocks = hidden / 64;
+        const int sms = num_sms();
         int s = 8;  // a portable cluster; it must divide the 128 rows of a tile
-        while (s > 1 && (tiles * s > num_sms() || s > k_blocks)) s /= 2;
-        a.splits = s;
-        a.k_per_split = (k_blocks + s - 1) / s;  // in K-blocks of 64
+        while (s > 1 && (tiles * s > sms || s > k_blocks)) s /= 2;
+        // One cluster along K: two clusters of 8 per column tile (144 CTAs for 64
+        // tokens) measured slower than one (15.3 against 10.2 us), so the kernel's
+        // support for several clusters along K is not used here.
+        const int z = 1;
+        a.cluster = s;
+        a.splits = z;
+        a.k_per_split = (k_blocks + s * z - 1) / (s * z);  // in K-blocks of 64 per CTA
         return a;
     }
     const int tile_n = kApTileN, tile_t = kApTileT, tile_k = kApTileK;
@@ -333,7 +341,7 @@ size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t n_tokens, int32
     if (check_dims(dims) || n_tokens < 1 || hidden < 1) return 0;
     const int N = dims->kv_lora_rank + dims->rope_dim;
     const AppendPlan a = append_plan(n_tokens, hidden, N);
-    return align_up(sizeof(float) * static_cast<size_t>(a.tc ? 1 : a.splits) * n_tokens * N);
+    return align_up(sizeof(float) * static_cast<size_t>(a.splits) * n_tokens * N);
 }
 
 int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t hidden, const void* w_kva,
@@ -352,7 +360,7 @@ int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32
     if (int rc = device_ok()) return rc;
     const int N = dims->kv_lora_rank + dims->rope_dim;
     const AppendPlan ap = append_plan(n_tokens, hidden, N);
-    const int splits = ap.tc ? 1 : ap.splits;  // partials the epilogue sums
+    const int splits = ap.splits;  // partials the epilogue sums
     float* part = static_cast<float*>(workspace);
     cudaStream_t st = as_stream(stream);
     if (ap.tc) {
@@ -362,9 +370,9 @@ int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32
         if (int rc = encode_2d(&tm_w, w_kva, N, hidden, 64)) return rc;
         const size_t smem = tc05::append_smem();
         if (int rc = ensure_smem(tc05::append_kernel, smem)) return rc;
-        const dim3 grid(N / 64, (n_tokens + tc05::kRows - 1) / tc05::kRows, ap.splits);
-        if (int rc = launch_cluster(tc05::append_kernel, grid, tc05::kThreads, smem, st, dim3(1, 1, ap.splits), tm_x,
-                                    tm_w, n_tokens, N, hidden / 64, ap.k_per_split, ap.splits, part)) return rc;
+        const dim3 grid(N / 64, (n_tokens + tc05::kRows - 1) / tc05::kRows, ap.cluster * ap.splits);
+        if (int rc = launch_cluster(tc05::append_kernel, grid, tc05::kThreads, smem, st, dim3(1, 1, ap.cluster), tm_x,
+                                    tm_w, n_tokens, N, hidden / 64, ap.k_per_split, ap.cluster, part)) return rc;
     } else {
         dim3 g1((N + kApTileN - 1) / kApTileN, (n_tokens + kApTileT - 1) / kApTileT, splits);
         if (int rc = launch(append_gemm_kernel, g1, 256, 0, st, static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w_kva),
