@@ -442,14 +442,25 @@ def run_ours(args, w):
     step_ms_attn_pass = [a.elapsed_time(b) for a, b in ev_attn]
     assert lib.device_error() == 0, "device fault during the timed steps"
 
-    # end to end through the public API with host buffers (pinned)
-    h_x = st["x_new"].cpu().pin_memory()
-    h_qn = st["q_nope"].cpu().pin_memory()
-    h_qp = st["q_pe"].cpu().pin_memory()
-    h_seq = st["new_seq"].cpu().pin_memory()
-    h_pos = st["new_pos"].cpu().pin_memory()
+    # end to end through the public API with host buffers: the step's inputs sit
+    # back to back in one pinned host buffer and cross to the device in one copy
+    # (one copy instead of five: each copy has its own fixed cost); the step
+    # reads them through device views of the staging buffer
+    pieces = [st["x_new"], st["q_nope"], st["q_pe"], st["new_seq"], st["new_pos"]]
+    offs, total = [], 0
+    for t_ in pieces:
+        offs.append(total)
+        total += (t_.numel() * t_.element_size() + 255) // 256 * 256
+    h_in = torch.empty(total, dtype=torch.uint8).pin_memory()
+    d_in = torch.empty(total, dtype=torch.uint8, device=device)
+    views = []
+    for t_, o in zip(pieces, offs):
+        n = t_.numel() * t_.element_size()
+        h_in[o:o + n].copy_(t_.reshape(-1).view(torch.uint8).cpu())
+        views.append(d_in[o:o + n].view(t_.dtype).view(t_.shape))
+    d_x, d_qn, d_qp, d_seq, d_pos = views
+    st["new_seq"], st["new_pos"] = d_seq, d_pos  # the e2e step's append reads its slots from the staging buffer
     h_out = torch.empty(st["out"].shape, dtype=torch.bfloat16).pin_memory()
-    d_x, d_qn, d_qp = torch.empty_like(st["x_new"]), torch.empty_like(st["q_nope"]), torch.empty_like(st["q_pe"])
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     e2e_graph = None
     if args.graph:
@@ -462,11 +473,7 @@ def run_ours(args, w):
     for k in range(K):
         flush.zero_()
         e2e_ev[k][0].record()
-        d_x.copy_(h_x, non_blocking=True)
-        d_qn.copy_(h_qn, non_blocking=True)
-        d_qp.copy_(h_qp, non_blocking=True)
-        st["new_seq"].copy_(h_seq, non_blocking=True)
-        st["new_pos"].copy_(h_pos, non_blocking=True)
+        d_in.copy_(h_in, non_blocking=True)
         if e2e_graph is not None:
             e2e_graph.replay()
         else:
@@ -510,8 +517,7 @@ def run_ours(args, w):
         "step_roofline_nominal_us": round(nominal_step * 1e6, 2),
         "step_frac_of_nominal_roofline": round(nominal_step / (t_step / 1e3), 4),
         "e2e": {"value": round(t_e2e * 1e3, 2), "unit": UNIT,
-                "h2d_bytes_per_step": (h_x.numel() + h_qn.numel() + h_qp.numel()) * 2
-                                      + (h_seq.numel() + h_pos.numel()) * 4,
+                "h2d_bytes_per_step": h_in.numel(),
                 "d2h_bytes_per_step": h_out.numel() * 2},
         "gpu_launches": launches_per_step * K,
         "kernels": kernel_names,

@@ -168,6 +168,19 @@ def test_graph_replay_matches_direct_launches(kernel):
         assert ev[0].elapsed_time(ev[1]) > 0.0
 
 
+@pytest.mark.parametrize("workers", [0, 37])
+def test_merge_up_projection_over_several_group_blocks(workers):
+    """G = 130 groups: the fused merge + up-projection runs three blocks of
+    groups per head (64, 64 and a ragged 2), with partial slots from many
+    workers; every output row is compared with the oracle."""
+    rng = np.random.default_rng(5)
+    lens = [int(v) for v in rng.integers(2, 400, size=65)]
+    w, lengths = small_v3("muv_blocks", 65, 2, lens)
+    data = build(w, lengths=lengths)
+    got = run_decode(w, to_device(data), kernel=0, num_workers=workers)
+    check(got, oracle_out(w, data))
+
+
 def test_append_on_a_side_stream_with_cache_ready():
     """The append may run on another stream: the decode's attention waits for the
     cache_ready event, directly and inside a captured graph, and gives the same
