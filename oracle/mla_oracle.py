@@ -10,7 +10,8 @@ Sources (cited by page title and section):
 
 * [MLA-arch] "MLA架构：低秩注意力机制优化LLM显存与计算效率"
   (intelliparadigm.com) -- section 1 (128 heads, qk_head_dim = 128 nope +
-  64 rope, RoPE part shared by all heads), section 2.2 (kv_a_proj_with_mqa
+  64 rope, RoPE part shared by all heads), section 2.1 (q_a_proj hidden ->
+  q_lora_rank, q_a_layernorm, q_b_proj -> H * qk_head_dim), section 2.2 (kv_a_proj_with_mqa
   hidden -> kv_lora_rank + rope, kv_a_layernorm = RMSNorm(kv_lora_rank),
   kv_b_proj -> per-head K-nope and V), section 3.1 (absorption is matrix
   associativity), section 3.2 (cache = c_kv [bsz, seq, 512] + pe
@@ -130,6 +131,24 @@ def append_rows(x, w_kva, positions, kv_lora_rank: int, gamma=None,
     c = rmsnorm(kv[:, :kv_lora_rank], gamma, eps)
     k_pe = rope(kv[:, kv_lora_rank:], np.asarray(positions), base)
     return np.concatenate([c, k_pe], axis=-1)
+
+
+# ---------------------------------------------------- query projection ----
+def query_projection(x, w_qa, w_qb, positions, num_heads: int, qk_nope_dim: int, rope_dim: int,
+                     gamma=None, eps: float = 1e-6, base: float = 10000.0):
+    """Queries of new tokens from their hidden states: [MLA-arch] 2.1 and 1.
+
+    c_q = RMSNorm(x . W_qa) (q_a_proj, hidden -> q_lora_rank, then
+    q_a_layernorm), q = c_q . W_qb (q_b_proj, q_lora_rank -> H * qk_head_dim),
+    each head's qk_head_dim values being the d_n non-RoPE part followed by the
+    d_r RoPE part (section 1 names them in that order); the RoPE part is
+    rotated at the token's position. Returns float64 (q_nope [T, H, d_n],
+    q_pe [T, H, d_r]).
+    """
+    c_q = rmsnorm(_f64(x) @ _f64(w_qa), gamma, eps)
+    q = (c_q @ _f64(w_qb)).reshape(c_q.shape[0], num_heads, qk_nope_dim + rope_dim)
+    pos = np.asarray(positions)
+    return q[..., :qk_nope_dim], rope(q[..., qk_nope_dim:], pos[:, None], base)
 
 
 # ------------------------------------------------------------ decode ----

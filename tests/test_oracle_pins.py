@@ -404,6 +404,67 @@ def test_append_chain_invariants():
     np.testing.assert_allclose(rows[:2, 16:], kv[:2, 16:], rtol=1e-14)  # position 0 = no rotation
 
 
+def test_query_projection_head_layout():
+    """A one-hot W_qb column lands in exactly one (head, index) of q_nope or q_pe:
+    heads are the outer index of each row and the non-RoPE part comes first
+    (a transposed view or a swapped split fails)."""
+    H, dn, dr, R = 3, 4, 2, 8
+    x = np.array([[1.0, -1, 1, 1, -1, 1, -1, -1], [-1.0, 1, 1, -1, 1, 1, 1, -1]])  # RMS 1 per row
+    w_qa = np.eye(R)
+    for h, j, r in [(0, 0, 3), (1, 2, 0), (2, 5, 7), (0, 4, 1), (2, 3, 6)]:
+        w_qb = np.zeros((R, H * (dn + dr)))
+        w_qb[r, h * (dn + dr) + j] = 1.0
+        qn, qp = O.query_projection(x, w_qa, w_qb, np.zeros(2, dtype=int), H, dn, dr, eps=0.0)
+        assert qn.shape == (2, H, dn) and qp.shape == (2, H, dr)
+        want_n, want_p = np.zeros_like(qn), np.zeros_like(qp)
+        if j < dn:
+            want_n[:, h, j] = x[:, r]
+        else:
+            want_p[:, h, j - dn] = x[:, r]
+        np.testing.assert_array_equal(qn, want_n)
+        np.testing.assert_array_equal(qp, want_p)
+
+
+def test_query_projection_matches_library_layers():
+    """Against torch's own linear and rms_norm layers (float64): the non-RoPE part
+    everywhere and the RoPE part at position 0 (no rotation) agree to rounding;
+    at other positions each rotate-half pair keeps its norm."""
+    rng = _rng(21)
+    T, hid, R, H, dn, dr = 5, 24, 16, 3, 6, 4
+    x = rng.standard_normal((T, hid))
+    w_qa, w_qb = rng.standard_normal((hid, R)), rng.standard_normal((R, H * (dn + dr)))
+    gamma = rng.uniform(0.5, 1.5, R)
+    tx = torch.tensor(x)
+    c = torch.nn.functional.rms_norm(torch.nn.functional.linear(tx, torch.tensor(w_qa.T)), (R,),
+                                     weight=torch.tensor(gamma), eps=1e-6)
+    q = torch.nn.functional.linear(c, torch.tensor(w_qb.T)).reshape(T, H, dn + dr).numpy()
+    qn, qp0 = O.query_projection(x, w_qa, w_qb, np.zeros(T, dtype=int), H, dn, dr, gamma=gamma)
+    np.testing.assert_allclose(qn, q[..., :dn], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(qp0, q[..., dn:], rtol=1e-12, atol=1e-12)
+    pos = np.array([1, 7, 100, 4096, 16383])
+    qn2, qp = O.query_projection(x, w_qa, w_qb, pos, H, dn, dr, gamma=gamma)
+    np.testing.assert_array_equal(qn2, qn)  # the position touches only the RoPE part
+    half = dr // 2
+    np.testing.assert_allclose(np.hypot(qp[..., :half], qp[..., half:]), np.hypot(qp0[..., :half], qp0[..., half:]),
+                               rtol=1e-12)
+    assert not np.allclose(qp, qp0)
+    # the rotation angle of pair i is position * base^(-2i/d_r)
+    ang = pos[:, None, None] * O.rope_inv_freq(dr)[None, None, :]
+    z0 = qp0[..., :half] + 1j * qp0[..., half:]
+    np.testing.assert_allclose(qp[..., :half] + 1j * qp[..., half:], z0 * np.exp(1j * ang), rtol=1e-11, atol=1e-11)
+
+
+def test_query_projection_is_scale_free_in_x():
+    """The RMSNorm after q_a_proj makes the queries independent of the scale of x (eps = 0)."""
+    rng = _rng(22)
+    x = rng.standard_normal((3, 16))
+    w_qa, w_qb = rng.standard_normal((16, 8)), rng.standard_normal((8, 2 * 6))
+    a = O.query_projection(x, w_qa, w_qb, np.array([0, 5, 9]), 2, 4, 2, eps=0.0)
+    b = O.query_projection(37.5 * x, w_qa, w_qb, np.array([0, 5, 9]), 2, 4, 2, eps=0.0)
+    for u, v in zip(a, b):
+        np.testing.assert_allclose(u, v, rtol=1e-12)
+
+
 # ------------------------------------------------------------------------
 # 11. the pages' printed structural numbers
 # ------------------------------------------------------------------------
