@@ -116,6 +116,24 @@ def workload_totals(w, lengths):
                 step_flops=step_flops)
 
 
+Q_RANK = 1536  # q_lora_rank of the DeepSeek-V3 query path
+
+
+def q_proj_line(w, ms, peaks):
+    """Roofline of mla_q_proj for the step's G new tokens: bytes = W_qa + W_qb +
+    x + q_nope + q_pe (bf16); FLOPs = 2 G (hidden q_rank + q_rank H (d_n + d_r))."""
+    d = w.dims
+    G = w.batch * w.q_len
+    n2 = d.num_heads * (d.qk_nope_dim + d.rope_dim)
+    bytes_ = 2 * (HIDDEN * Q_RANK + Q_RANK * n2 + G * HIDDEN + G * n2)
+    flops = 2 * G * (HIDDEN * Q_RANK + Q_RANK * n2)
+    gbs = bytes_ / (ms * 1e-3) / 1e9
+    return {"us": round(ms * 1e3, 2), "tokens": G, "hidden": HIDDEN, "q_rank": Q_RANK,
+            "bytes": bytes_, "achieved_gbs": round(gbs, 1), "peak_gbs": peaks["hbm_gbs"],
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+            "timing": "CUDA events around each call, L2 flushed before each, K calls"}
+
+
 def roofline(bytes_, flops, seconds, peaks):
     gbs = bytes_ / seconds / 1e9
     tfs = flops / seconds / 1e12
@@ -376,6 +394,7 @@ def run_ours(args, w):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     init_dist("nccl", world)
+    from mla_latent_kv_29_b200 import inputs as I
     from mla_latent_kv_29_b200 import lib
 
     lib.load()
@@ -486,6 +505,32 @@ def run_ours(args, w):
 
     t_step = max_over_ranks(statistics.mean(step_ms), device)
     t_attn = max_over_ranks(statistics.mean(attn_ms), device)
+    # the query projection of the step's new tokens (mla_q_proj, a separate pass:
+    # the decode above takes its queries as inputs), each call after an L2 flush
+    d = st["d"]
+    qin = I.q_proj_inputs(d, w.batch * w.q_len, HIDDEN, Q_RANK, seed=w.seed)
+    qdev = {k: v.to(device) for k, v in qin.items()}
+    q_ws = torch.empty(lib.q_proj_workspace_size(d, w.batch * w.q_len, HIDDEN, Q_RANK), dtype=torch.uint8,
+                       device=device)
+    q_out = (torch.empty_like(st["q_nope"]).view(-1, d.num_heads, d.qk_nope_dim),
+             torch.empty_like(st["q_pe"]).view(-1, d.num_heads, d.rope_dim))
+
+    def q_proj():
+        lib.q_proj(d, qdev["x"], qdev["w_qa"], qdev["w_qb"], qdev["positions"], q_gamma=qdev["gamma"],
+                   q_nope=q_out[0], q_pe=q_out[1], workspace=q_ws)
+
+    for _ in range(args.warmup):
+        q_proj()
+    q_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    torch.cuda.synchronize(device)
+    for k in range(K):
+        flush.zero_()
+        q_ev[k][0].record()
+        q_proj()
+        q_ev[k][1].record()
+    torch.cuda.synchronize(device)
+    assert lib.device_error() == 0, "device fault in the query projection"
+    t_q = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in q_ev), device)
     t_e2e = max_over_ranks(statistics.mean(e2e_ms), device)
     if rank != 0:
         return None
@@ -520,6 +565,7 @@ def run_ours(args, w):
                 "h2d_bytes_per_step": h_in.numel(),
                 "d2h_bytes_per_step": h_out.numel() * 2},
         "gpu_launches": launches_per_step * K,
+        "q_proj": q_proj_line(w, t_q, peaks),
         "kernels": kernel_names,
         "clocks": clocks,
     }

@@ -136,6 +136,39 @@ MLA_API int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_token
 MLA_API size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t n_tokens, int32_t hidden);
 
 /* ------------------------------------------------------------------ */
+/* Query projection of new tokens, the step before the absorption:
+ * [MLA-arch] 2.1 (q_a_proj hidden -> q_lora_rank, q_a_layernorm, q_b_proj
+ * q_lora_rank -> H * qk_head_dim) and 1 (qk_head_dim = the d_n non-RoPE part
+ * followed by the d_r RoPE part); RoPE as in [MQA-MLA] "MLA的实现".
+ *   c_q   = x . w_qa / sqrt(mean((x . w_qa)^2) + rms_eps) * q_gamma
+ *   q     = bf16(c_q) . w_qb, viewed as [n_tokens, H, d_n + d_r]
+ *   q_nope[t, h, :] = bf16(q[t, h, :d_n])
+ *   q_pe[t, h, :]   = bf16(rotate-half RoPE of q[t, h, d_n:] at positions[t])
+ * Arguments:
+ *   x        bf16 [n_tokens, hidden], 16-byte aligned
+ *   w_qa     bf16 [hidden, q_rank], 16-byte aligned
+ *   q_gamma  bf16 [q_rank] or NULL (= ones)
+ *   w_qb     bf16 [q_rank, H * (qk_nope_dim + rope_dim)], 16-byte aligned
+ *   positions int32 [n_tokens] on the device (absolute token positions)
+ *   q_nope   bf16 [n_tokens, H, qk_nope_dim] (output; the layout mla_decode
+ *            takes with n_tokens = batch * q_len)
+ *   q_pe     bf16 [n_tokens, H, rope_dim] (output)
+ *   workspace >= mla_q_proj_workspace_size(dims, n_tokens, hidden, q_rank)
+ *            bytes, 256-byte aligned, contents need not be initialised.
+ * hidden, q_rank and H * (qk_nope_dim + rope_dim) must be multiples of 64 and
+ * rope_dim even and <= 128 (else MLA_ERR_UNSUPPORTED_DIMS). Accumulation is
+ * fp32; c_q is rounded to bf16 before the second product. */
+MLA_API int mla_q_proj(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t hidden,
+                       const void* w_qa, int32_t q_rank, const void* q_gamma, float rms_eps,
+                       const void* w_qb, const int32_t* positions, float rope_base,
+                       void* q_nope, void* q_pe, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace mla_q_proj needs; 0 if the arguments are invalid or the
+ * dims unsupported. */
+MLA_API size_t mla_q_proj_workspace_size(const mla_dims_t* dims, int32_t n_tokens, int32_t hidden,
+                                         int32_t q_rank);
+
+/* ------------------------------------------------------------------ */
 /* Absorbed decode: [MQA-MLA] "MLA的实现" forward_inference_absorbed with the
  * query absorption of [MLA-arch] 3.1, restated for q_len new tokens per
  * sequence over the paged cache. For sequence b (context_lens[b] = L

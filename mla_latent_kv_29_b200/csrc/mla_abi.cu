@@ -18,6 +18,7 @@
 #include "decode_pair.cuh"
 #include "gemm_small.cuh"
 #include "gemm_tc05.cuh"
+#include "qproj.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -302,6 +303,45 @@ AppendPlan append_plan(int32_t n_tokens, int32_t hidden, int32_t N) {
     return a;
 }
 
+// part[z][t][n] (fp32 [ap.splits][T][N]) = the K-range z of x . w on the
+// tcgen05 GEMM: x bf16 [T, K], w bf16 [K, N], K and N multiples of 64,
+// x and w 16-byte aligned.
+int launch_row_gemm(const void* x, int32_t T, int32_t K, const void* w, int32_t N, const AppendPlan& ap,
+                    float* part, cudaStream_t st) {
+    if (!aligned(x, 16) || !aligned(w, 16)) return MLA_ERR_INVALID_ARG;
+    CUtensorMap tm_x, tm_w;
+    if (int rc = encode_2d(&tm_x, x, K, T, tc05::kRows)) return rc;
+    if (int rc = encode_2d(&tm_w, w, N, K, 64)) return rc;
+    const size_t smem = tc05::append_smem();
+    if (int rc = ensure_smem(tc05::append_kernel, smem)) return rc;
+    const dim3 grid(N / 64, (T + tc05::kRows - 1) / tc05::kRows, ap.cluster * ap.splits);
+    return launch_cluster(tc05::append_kernel, grid, tc05::kThreads, smem, st, dim3(1, 1, ap.cluster), tm_x, tm_w, T,
+                          N, K / 64, ap.k_per_split, ap.cluster, part);
+}
+
+// ---- query projection workspace: GEMM 1 partials | c_q bf16 | GEMM 2 partials
+struct QProjLayout {
+    AppendPlan g1, g2;
+    size_t part1, cq, part2, total;
+};
+
+int q_proj_layout(const mla_dims_t* d, int32_t T, int32_t hidden, int32_t R, QProjLayout* L) {
+    if (int rc = check_dims(d)) return rc;
+    if (T < 1 || hidden < 1 || R < 1) return MLA_ERR_INVALID_ARG;
+    const int64_t N2 = static_cast<int64_t>(d->num_heads) * (d->qk_nope_dim + d->rope_dim);
+    if (hidden % 64 || R % 64 || N2 % 64 || N2 >= (int64_t(1) << 30) || d->rope_dim % 2 ||
+        d->rope_dim > 2 * kQMaxRopePairs || d->qk_nope_dim + d->rope_dim / 2 > 1024)
+        return MLA_ERR_UNSUPPORTED_DIMS;
+    L->g1 = append_plan(T, hidden, R);
+    L->g2 = append_plan(T, R, static_cast<int32_t>(N2));
+    size_t off = 0;
+    L->part1 = off; off = align_up(off + sizeof(float) * static_cast<size_t>(L->g1.splits) * T * R);
+    L->cq = off; off = align_up(off + sizeof(uint16_t) * static_cast<size_t>(T) * R);
+    L->part2 = off; off = align_up(off + sizeof(float) * static_cast<size_t>(L->g2.splits) * T * N2);
+    L->total = off;
+    return MLA_OK;
+}
+
 }  // namespace
 }  // namespace mla
 
@@ -364,15 +404,7 @@ int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32
     float* part = static_cast<float*>(workspace);
     cudaStream_t st = as_stream(stream);
     if (ap.tc) {
-        if (!aligned(x, 16) || !aligned(w_kva, 16)) return MLA_ERR_INVALID_ARG;
-        CUtensorMap tm_x, tm_w;
-        if (int rc = encode_2d(&tm_x, x, hidden, n_tokens, tc05::kRows)) return rc;
-        if (int rc = encode_2d(&tm_w, w_kva, N, hidden, 64)) return rc;
-        const size_t smem = tc05::append_smem();
-        if (int rc = ensure_smem(tc05::append_kernel, smem)) return rc;
-        const dim3 grid(N / 64, (n_tokens + tc05::kRows - 1) / tc05::kRows, ap.cluster * ap.splits);
-        if (int rc = launch_cluster(tc05::append_kernel, grid, tc05::kThreads, smem, st, dim3(1, 1, ap.cluster), tm_x,
-                                    tm_w, n_tokens, N, hidden / 64, ap.k_per_split, ap.cluster, part)) return rc;
+        if (int rc = launch_row_gemm(x, n_tokens, hidden, w_kva, N, ap, part, st)) return rc;
     } else {
         dim3 g1((N + kApTileN - 1) / kApTileN, (n_tokens + kApTileT - 1) / kApTileT, splits);
         if (int rc = launch(append_gemm_kernel, g1, 256, 0, st, static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w_kva),
@@ -397,6 +429,51 @@ int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32
     P.eps = rms_eps;
     P.rope_base = rope_base;
     if (int rc = launch(append_epilogue_kernel, n_tokens, 256, sizeof(float) * N, st, P)) return rc;
+    return launch_status();
+}
+
+size_t mla_q_proj_workspace_size(const mla_dims_t* dims, int32_t n_tokens, int32_t hidden, int32_t q_rank) {
+    QProjLayout L;
+    return q_proj_layout(dims, n_tokens, hidden, q_rank, &L) ? 0 : L.total;
+}
+
+int mla_q_proj(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t hidden, const void* w_qa,
+               int32_t q_rank, const void* q_gamma, float rms_eps, const void* w_qb, const int32_t* positions,
+               float rope_base, void* q_nope, void* q_pe, void* workspace, size_t workspace_bytes, void* stream) {
+    QProjLayout L;
+    if (int rc = q_proj_layout(dims, n_tokens, hidden, q_rank, &L)) return rc;
+    if (!x || !w_qa || !w_qb || !positions || !q_nope || !q_pe || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!(rms_eps >= 0.f) || !(rope_base > 0.f)) return MLA_ERR_INVALID_ARG;
+    if (!aligned(workspace, kAlign)) return MLA_ERR_INVALID_ARG;
+    if (workspace_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+    if (int rc = device_ok()) return rc;
+    cudaStream_t st = as_stream(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* part1 = reinterpret_cast<float*>(ws + L.part1);
+    uint16_t* cq = reinterpret_cast<uint16_t*>(ws + L.cq);
+    float* part2 = reinterpret_cast<float*>(ws + L.part2);
+    const int32_t H = dims->num_heads, dn = dims->qk_nope_dim, dr = dims->rope_dim;
+    const int32_t N2 = H * (dn + dr);
+    // c_q = RMSNorm(x . W_qa) * gamma, rounded to bf16 as the second GEMM's operand
+    if (int rc = launch_row_gemm(x, n_tokens, hidden, w_qa, q_rank, L.g1, part1, st)) return rc;
+    if (int rc = launch(q_norm_kernel, n_tokens, kQNormThreads, sizeof(float) * q_rank, st, part1, L.g1.splits,
+                        n_tokens, q_rank, static_cast<const uint16_t*>(q_gamma), rms_eps, cq)) return rc;
+    // q = c_q . W_qb, then the per-head split and the RoPE of the rope part
+    if (int rc = launch_row_gemm(cq, n_tokens, q_rank, w_qb, N2, L.g2, part2, st)) return rc;
+    QSplitParams P;
+    P.part = part2;
+    P.positions = positions;
+    P.q_nope = static_cast<uint16_t*>(q_nope);
+    P.q_pe = static_cast<uint16_t*>(q_pe);
+    P.splits = L.g2.splits;
+    P.T = n_tokens;
+    P.H = H;
+    P.dn = dn;
+    P.dr = dr;
+    for (int i = 0; i < kQMaxRopePairs; ++i)
+        P.inv_freq[i] = i < dr / 2 ? std::pow(static_cast<double>(rope_base), -2.0 * i / static_cast<double>(dr)) : 0.0;
+    const int threads = (dn + dr / 2 + 31) / 32 * 32;
+    if (int rc = launch(q_split_rope_kernel, dim3(n_tokens, H), threads, 0, st, P)) return rc;
     return launch_status();
 }
 

@@ -116,6 +116,7 @@ WORKLOADS = {
 # Salts for independent streams.
 _S_LEN, _S_TABLE, _S_Q_NOPE, _S_Q_PE, _S_W_UK, _S_W_UV = 1, 2, 3, 4, 5, 6
 _S_X, _S_W_KVA, _S_GAMMA = 7, 8, 9
+_S_QX, _S_W_QA, _S_W_QB, _S_QGAMMA, _S_QPOS = 10, 11, 12, 13, 14
 _S_CACHE = 1 << 20  # + sequence index
 
 
@@ -222,6 +223,23 @@ def append_inputs(w: Workload):
     offs = torch.arange(w.q_len, dtype=torch.int32).repeat(w.batch)
     positions = lengths.repeat_interleave(w.q_len) - w.q_len + offs
     return dict(x=x, w_kva=w_kva, seq_ids=seq_ids, positions=positions.to(torch.int32))
+
+
+def q_proj_inputs(dims: Dims, n_tokens: int, hidden: int, q_rank: int, seed: int, gamma: bool = True,
+                  max_position: int = 32768):
+    """bf16 inputs of the query projection: x [T, hidden] ~ N(0,1), W_qa
+    [hidden, q_rank] ~ N(0, 1/hidden), W_qb [q_rank, H (d_n + d_r)] ~
+    N(0, 1/q_rank), gamma [q_rank] ~ U[0.5, 1.5] (or None) and positions
+    int32 [T] ~ U[0, max_position)."""
+    x = bf16(normal((n_tokens, hidden), 1.0, seed, _S_QX))
+    w_qa = bf16(normal((hidden, q_rank), hidden ** -0.5, seed, _S_W_QA))
+    n2 = dims.num_heads * (dims.qk_nope_dim + dims.rope_dim)
+    w_qb = bf16(normal((q_rank, n2), q_rank ** -0.5, seed, _S_W_QB))
+    g = None
+    if gamma:
+        g = bf16(0.5 + torch.rand(q_rank, generator=generator(seed, _S_QGAMMA)))
+    pos = torch.randint(0, max_position, (n_tokens,), generator=generator(seed, _S_QPOS), dtype=torch.int32)
+    return dict(x=x, w_qa=w_qa, w_qb=w_qb, gamma=g, positions=pos)
 
 
 def scaled(w: Workload, batch: Optional[int] = None, length: Optional[int] = None,

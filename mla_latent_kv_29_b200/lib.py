@@ -30,7 +30,7 @@ KERNEL_AUTO, KERNEL_SM100, KERNEL_GENERIC = 0, 1, 2
 
 EXPORTED = ("mla_append_kv", "mla_append_workspace_size", "mla_decode", "mla_decode_workspace_size",
             "mla_combine", "mla_debug_resolve_slots", "mla_get_device_error", "mla_error_string",
-            "mla_version", "mla_decode_no_alloc")
+            "mla_version", "mla_decode_no_alloc", "mla_q_proj", "mla_q_proj_workspace_size")
 
 
 class MLAError(RuntimeError):
@@ -76,6 +76,8 @@ def load():
         "mla_error_string": (ctypes.c_char_p, [_I32]),
         "mla_version": (_I32, []),
         "mla_decode_no_alloc": (_I32, [D, _P, _P, _I32, _I32, _P, _I64, _P, _I32, _P, _I32, _P, _P, _P, O, _P]),
+        "mla_q_proj": (_I32, [D, _P, _I32, _I32, _P, _I32, _P, _F, _P, _P, _F, _P, _P, _P, _SZ, _P]),
+        "mla_q_proj_workspace_size": (_SZ, [D, _I32, _I32, _I32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -156,6 +158,37 @@ def append_kv(dims: Dims, x, w_kva, seq_ids, positions, block_table, pool, rms_g
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "mla_append_kv")
     return pool
+
+
+# -------------------------------------------------------- query projection
+def q_proj_workspace_size(dims: Dims, n_tokens: int, hidden: int, q_rank: int) -> int:
+    return int(load().mla_q_proj_workspace_size(ctypes.byref(c_dims(dims, 1.0)), n_tokens, hidden, q_rank))
+
+
+def q_proj(dims: Dims, x, w_qa, w_qb, positions, q_gamma=None, rms_eps: float = 1e-6, rope_base: float = 10000.0,
+           q_nope=None, q_pe=None, workspace=None, stream=None):
+    """mla_q_proj: (q_nope [T, H, d_n], q_pe [T, H, d_r]) bf16 from x [T, hidden]."""
+    lib = load()
+    cd = c_dims(dims, 1.0)
+    T, hidden = x.shape
+    q_rank = w_qa.shape[1]
+    need = lib.mla_q_proj_workspace_size(ctypes.byref(cd), T, hidden, q_rank)
+    if need == 0:
+        raise MLAError(-2, "mla_q_proj_workspace_size")
+    if workspace is None:
+        workspace = _workspace(need, x.device)
+    if q_nope is None:
+        q_nope = torch.empty(T, dims.num_heads, dims.qk_nope_dim, dtype=torch.bfloat16, device=x.device)
+    if q_pe is None:
+        q_pe = torch.empty(T, dims.num_heads, dims.rope_dim, dtype=torch.bfloat16, device=x.device)
+    st = lib.mla_q_proj(
+        ctypes.byref(cd), _ptr(x, torch.bfloat16, "x"), T, hidden, _ptr(w_qa, torch.bfloat16, "w_qa"), q_rank,
+        _ptr(q_gamma, torch.bfloat16, "q_gamma"), float(rms_eps), _ptr(w_qb, torch.bfloat16, "w_qb"),
+        _ptr(positions, torch.int32, "positions"), float(rope_base), _ptr(q_nope, torch.bfloat16, "q_nope"),
+        _ptr(q_pe, torch.bfloat16, "q_pe"), _ptr(workspace, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "mla_q_proj")
+    return q_nope, q_pe
 
 
 # ------------------------------------------------------------------ decode

@@ -91,6 +91,26 @@ def test_combine_and_append_validation(so):
                             10, fake, 16, None) == -3
 
 
+def test_q_proj_validation(so):
+    d = _dims()
+    ws = so.mla_q_proj_workspace_size(ctypes.byref(d), 64, 7168, 1536)
+    # GEMM 1 partials (fp32 T x q_rank), c_q (bf16), GEMM 2 partials (fp32 T x H * 192)
+    assert ws >= 64 * 1536 * 4 + 64 * 1536 * 2 + 64 * 128 * 192 * 4 and ws % 256 == 0
+    assert so.mla_q_proj_workspace_size(ctypes.byref(d), 64, 7000, 1536) == 0  # hidden not a multiple of 64
+    assert so.mla_q_proj_workspace_size(ctypes.byref(d), 0, 7168, 1536) == 0
+    fake = ctypes.c_void_p(1 << 20)
+
+    def call(T=64, hidden=7168, rank=1536, x=fake, ws_bytes=1 << 30, eps=1e-6):
+        return so.mla_q_proj(ctypes.byref(d), x, T, hidden, fake, rank, None, eps, fake, fake, 1e4, fake, fake,
+                             fake, ws_bytes, None)
+
+    assert call(x=None) == -1
+    assert call(T=0) == -1
+    assert call(hidden=7000) == -2
+    assert call(eps=-1.0) == -1
+    assert call(ws_bytes=16) == -3
+
+
 def test_valid_call_without_gpu_reports_no_device(so):
     import torch
 

@@ -148,3 +148,32 @@ def test_append_tiny_dims_uses_the_cuda_core_path():
     ref = O.append_rows(data["append"]["x"], data["append"]["w_kva"], data["append"]["positions"].numpy(),
                         d.kv_lora_rank)
     assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 2e-3)
+
+
+# -------------------------------------------------------- query projection
+@pytest.mark.parametrize("case", [
+    ("small", I.Dims(num_heads=4, kv_lora_rank=64, rope_dim=32, qk_nope_dim=32, v_head_dim=32, block_size=64),
+     5, 256, 128, True),
+    ("v3", I.WORKLOADS["v3_b64_l1k_8k"].dims, 64, 7168, 1536, True),
+    ("v3_ragged_no_gamma", I.WORKLOADS["v3_b64_l1k_8k"].dims, 130, 7168, 1536, False),
+])
+def test_q_proj_matches_oracle(case):
+    """mla_q_proj against the oracle's fp64 query projection, q_nope and q_pe
+    each within the decode tolerance and elementwise within a few bf16 steps."""
+    L = _lib()
+    _, d, T, hidden, rank, with_gamma = case
+    inp = I.q_proj_inputs(d, T, hidden, rank, seed=41 + T, gamma=with_gamma)
+    dev = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    qn, qp = L.q_proj(d, dev["x"], dev["w_qa"], dev["w_qb"], dev["positions"], q_gamma=dev["gamma"])
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    ref_n, ref_p = O.query_projection(inp["x"], inp["w_qa"], inp["w_qb"], inp["positions"].numpy(), d.num_heads,
+                                      d.qk_nope_dim, d.rope_dim, gamma=inp["gamma"])
+    for got, ref in ((qn, ref_n), (qp, ref_p)):
+        got = got.float().cpu().numpy()
+        assert got.shape == ref.shape
+        ok, err, bound = tolerance_ok(got, ref)
+        assert ok, (err, bound)
+        # c_q is rounded to bf16 before the second product and the result once more
+        scale = np.abs(ref).max()
+        assert np.all(np.abs(got - ref) <= 2.0 ** -6 * np.abs(ref) + 2.0 ** -8 * scale)
