@@ -93,6 +93,14 @@ def load_peaks():
         return dict(FALLBACK_PEAKS)
 
 
+def workload_config(w, cached_tokens):
+    """The workload's identity, the same in both arms' lines."""
+    return {"workload": w.name, "batch_per_gpu": w.batch, "q_len": w.q_len,
+            "context": f"U[{w.length_range[0]},{w.length_range[1]}]", "cached_tokens_per_gpu": cached_tokens,
+            "heads": w.dims.num_heads, "latent": w.dims.kv_lora_rank, "rope": w.dims.rope_dim,
+            "page": w.dims.block_size, "paged": "shuffled" if w.paged else "contiguous"}
+
+
 def workload_totals(w, lengths):
     """Algorithmic units of one decode step. Attention: every cached token's
     576 bf16 values read once plus the absorbed queries; FLOPs 2 H (576 + 512)
@@ -545,13 +553,10 @@ def run_ours(args, w):
         "metric": METRIC, "value": round(t_step * 1e3, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "batch_per_gpu": w.batch, "q_len": w.q_len,
-                   "context": f"U[{w.length_range[0]},{w.length_range[1]}]", "cached_tokens_per_gpu": tot["T"],
-                   "heads": w.dims.num_heads, "latent": w.dims.kv_lora_rank, "rope": w.dims.rope_dim,
-                   "page": w.dims.block_size, "paged": "shuffled", "l2": "flushed (256 MB write) before each step",
-                   "step": "append of the batch's new tokens + absorbed decode" +
-                           (" (append on a side stream; the attention waits for it)" if args.overlap else ""),
-                   "launch": "CUDA graph replay" if args.graph else "direct launches"},
+        "config": dict(workload_config(w, tot["T"]), l2="flushed (256 MB write) before each step",
+                       step="append of the batch's new tokens + absorbed decode" +
+                            (" (append on a side stream; the attention waits for it)" if args.overlap else ""),
+                       launch="CUDA graph replay" if args.graph else "direct launches"),
         "roofline": roof,
         "attn_us": round(t_attn * 1e3, 2),
         "attn_timing": "CUDA events around the attention launch, in a second pass of K steps "
@@ -623,8 +628,7 @@ def run_reference(args, w):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v / 1e3, 3),
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": w.name, "batch_per_gpu": w.batch, "q_len": w.q_len,
-                       "context": f"U[{w.length_range[0]},{w.length_range[1]}]"},
+            "config": dict(workload_config(w, T), step="append of the batch's new tokens + absorbed decode"),
             "cpu_baseline": {"value": round(v, 1), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
