@@ -1,16 +1,19 @@
-// tcgen05 versions of the per-head GEMMs around the attention, for DeepSeek-V3
-// like dims (their weights are read once per step, so they are bandwidth
-// bound: operands arrive by TMA in 128-byte-swizzled boxes, one CTA of four
-// warps per head and block of up to 128 new tokens, accumulators in TMEM):
-//   absorb: Q[g, h, 0:d_c] = bf16(q_nope[g, h] W_UK[h]),  Q[g, h, d_c:] = q_pe[g, h]
-//           (query absorption, "MLA架构：低秩注意力机制优化LLM显存与计算效率" 3.1)
-//   UV:     out[g, h] = bf16(W_UV[h] o_lat[g, h])
-// and the log-sum-exp merge of the split-KV partials into bf16 o_lat that
-// feeds the UV GEMM.
+// tcgen05 versions of the GEMMs around the attention, for DeepSeek-V3 like
+// dims (their weights are read once per step, so they are bandwidth bound:
+// operands arrive by TMA in 128-byte-swizzled boxes, accumulators in TMEM):
+//   absorb:     Q[g, h, 0:d_c] = bf16(q_nope[g, h] W_UK[h]),  Q[g, h, d_c:] = q_pe[g, h]
+//               (query absorption, "MLA架构：低秩注意力机制优化LLM显存与计算效率" 3.1)
+//   merge + UV: out[g, h] = bf16(W_UV[h] o_lat[g, h]) with o_lat the
+//               log-sum-exp merge of the split-KV partials, merged on chip
+//               (merge_uv_kernel), or merged into memory (merge_kernel) and
+//               then multiplied (uv_kernel)
+//   row GEMM:   y = x W (fp32) for x [T, K] and W [K, N], the K range split
+//               over a cluster (append_kernel): the cache append's x W_kva and
+//               the query projection's x W_qa and c_q W_qb.
 //
-// Roles (128 threads): lane 0 of warp 0 issues the TMA loads, lane 0 of
-// warp 1 the MMAs (M = 128 token rows, cta_group::1), warp 2 owns the TMEM
-// allocation, and all four warps (thread t = TMEM lane t = token row g0 + t)
+// Roles of the 128-thread kernels: lane 0 of warp 0 issues the TMA loads,
+// lane 0 of warp 1 the MMAs (M = 128, cta_group::1), warp 2 owns the TMEM
+// allocation, and all four warps (thread t = TMEM lane t = row t of the MMA)
 // run the epilogue. Every mbarrier wait is bounded (ptx::mbar_wait).
 #pragma once
 
