@@ -95,6 +95,18 @@ typedef struct mla_decode_opts {
                                absorption, which do not read the cache.
                                Under stream capture it joins the two
                                streams' work into one graph. */
+    /* Test hooks of the failure detection, 0 in normal use. Every wait of
+     * the tensor-core attention kernel (an mbarrier that a copy, a
+     * tensor-core operation or another warp completes) gives up after a
+     * time limit, records MLA_ERR_DEVICE_TIMEOUT in the device error word
+     * and lets the kernel drain and exit, so that the context stays usable.
+     * debug_wait_limit_us replaces the default limit of 2 s (0 = default).
+     * debug_starve != 0 makes that kernel's load warps issue nothing, so that
+     * no copy or tensor-core operation is ever in flight and every consumer
+     * wait runs out; the call then reports MLA_ERR_DEVICE_TIMEOUT through
+     * mla_get_device_error() and its output is undefined. */
+    uint32_t debug_wait_limit_us;
+    int32_t debug_starve;
 } mla_decode_opts_t;
 
 /* Paged latent cache ("pool"), [MLA-arch] 3.2 kept as one row per token:
@@ -192,10 +204,12 @@ MLA_API size_t mla_q_proj_workspace_size(const mla_dims_t* dims, int32_t n_token
  *   workspace >= mla_decode_workspace_size(...) bytes, 256-byte aligned,
  *           contents need not be initialised
  *   opts    NULL or kernel / split overrides
- * Alignment: q_nope, w_uk, w_uv and out 16-byte aligned select the
- * tensor-core GEMMs around the attention; the tcgen05 attention kernel
- * (opts->kernel = 1, the default for DeepSeek-V3 dims) requires them and
- * returns MLA_ERR_INVALID_ARG otherwise.
+ * Alignment: q_nope, q_pe, w_uk, w_uv and out 16-byte aligned (with d_n a
+ * multiple of 64, d_c of 256, d_r of 8, d_v of 16) select the tcgen05
+ * absorption, merge and up-projection kernels; otherwise CUDA-core kernels
+ * run them. The tcgen05 attention kernel (opts->kernel = 1, the default for
+ * DeepSeek-V3 dims) needs the tcgen05 kernels around it and returns
+ * MLA_ERR_INVALID_ARG when they do not apply.
  * Rounding: q_lat is rounded to bf16 before the score product and the
  * softmax weights to bf16 before the value product; accumulation and the
  * combine are fp32; split partials are fp32 (CUDA-core kernel) or rounded
@@ -233,9 +247,12 @@ MLA_API size_t mla_decode_workspace_size(const mla_dims_t* dims, int32_t batch, 
  * problem needs more scratch than the buffer holds (for DeepSeek-V3 dims
  * the default schedule fits batch * q_len up to 64).
  *
- * Set-up: the first call on each device looks up the buffer's device
- * address (cudaGetSymbolAddress, with that device current) and caches it;
- * make that first call before any stream capture on that device.
+ * Set-up: the first call in each CUDA context (the device's primary
+ * context for runtime users) looks up the buffer's device address
+ * (cudaGetSymbolAddress, with that context current) and caches it under the
+ * context's unique id, so a new context -- another device, a driver-API
+ * context, the primary context re-created after cudaDeviceReset -- gets its
+ * own look-up. Make that first call before any stream capture.
  * Sharing: every call on a device uses the same buffer and leaves its
  * contents behind. Nothing in it needs to start at zero (each call writes
  * every scratch byte it later reads), but calls whose work overlaps on the

@@ -21,25 +21,35 @@
 //          CTA r supplies latent columns 256r + 128n .. +127 for all tokens.
 // The tile's latent values therefore reach each CTA twice (once as keys,
 // once as values), so shared-memory fills are ~1.9x the HBM bytes, while
-// HBM reads stay ~1x because the second read of a page hits L2.
+// HBM reads stay ~1x because the second read of a page hits L2 (each CTA
+// also asks L2 for its page of the next tile ahead of the key loads).
 //
-// Warp roles per CTA (288 threads): one thread of warp 0 streams the queries
+// Warp roles per CTA (256 threads): one thread of warp 0 streams the queries
 // and the key stages (column blocks 0-2, 3-4, 5-6 and 7-8 of the CTA's page,
 // one TMA operation each) into a one-tile key ring; warp 2 streams the value
-// stages (32 tokens x 256 columns, 16 KB) into a three-stage value ring (one
-// thread issues, the warp zeroes the tail rows of partial stages); warp 1
-// allocates tensor memory (both CTAs). In the leader, three threads issue
-// the MMAs: lanes 0 of warps 1 and 3 the score MMAs of every tile (column
-// blocks 0-4 and 5-8, into two half-accumulators that the softmax adds),
-// lane 0 of warp 8 the value MMAs (one thread cannot issue tcgen05.mma fast
-// enough for the M 128 x N 128 score instructions).
+// stages (32 tokens x 256 columns, 16 KB) into a four-stage value ring that
+// holds a whole tile (one thread issues, the warp zeroes the tail rows of
+// partial stages); warp 1 allocates tensor memory (both CTAs). In the leader,
+// two threads (lanes 0 of warps 1 and 3) issue the MMAs, each the same
+// program over the pair's tiles n = 0, 1, ...: its half of the score MMAs of
+// tile n (column blocks 0-4 or 5-8, into two half-accumulators that the
+// softmax adds), then its half of the value MMAs of tile n - 1 (latent
+// columns 0-255 or 256-511 of the CTA pair's O). The tensor pipe therefore
+// runs S(n), PV(n-1), S(n+1), PV(n), ...: the score of the next tile covers
+// the softmax of the current one, and no issuer runs further ahead, so the
+// MMA queue stays short and the key and value stages are released promptly
+// (two threads are needed: one cannot issue the M 128 x N 128 score
+// instructions as fast as the tensor cores run them).
 // Warps 4-7 (thread t = TMEM lane t) run the softmax, rescale O when the
-// running max grows by more than 2^8, write P to shared memory (two buffers,
-// by tile parity, so that the P of tile j is written while the value MMAs of
-// tile j-1 still run) and, at the end of a segment, normalise O and write
-// the partial.
-// Every mbarrier wait is bounded (see ptx::mbar_wait): on expiry the kernel
-// records MLA_ERR_DEVICE_TIMEOUT and every role drains to the common exit.
+// running max grows by more than 2^8, write P to shared memory (one buffer:
+// the value MMAs of tile n - 1 have finished by the time the softmax of tile
+// n has its weights) and, at the end of a segment, normalise O and write the
+// partial.
+// Every mbarrier wait is bounded (see ptx::mbar_wait; the limit is a kernel
+// parameter so that a test can shorten it): on expiry the kernel records
+// MLA_ERR_DEVICE_TIMEOUT and every role drains to the common exit. With the
+// test hook `starve` the load warps issue nothing at all, so no copy or
+// tensor-core operation is in flight when the consumers' waits run out.
 #pragma once
 
 #include "common.cuh"
@@ -64,8 +74,8 @@ __host__ __device__ constexpr int kstage_blocks(int s) { return s == 0 ? 3 : 2; 
 constexpr int kKTile = kQBoxes * kBox;  // 72 KB
 constexpr int kVStage = 2 * kBox;    // value stage: 32 tokens x 256 latent columns (4 x 4 KB)
 constexpr int kVPerTile = 4;         // 4 value stages per tile
-constexpr int kVStages = 3;          // value ring: three stages
-constexpr int kThreads = 288;  // 9 warps; the softmax warps 4-7 own TMEM lanes 0-127
+constexpr int kVStages = 4;          // value ring: four stages (a whole tile)
+constexpr int kThreads = 256;  // 8 warps; the softmax warps 4-7 own TMEM lanes 0-127
 constexpr int kTmemCols = 512;
 constexpr int kTmS = 0;          // two S buffers (tile parity), each lo and hi halves of 64 columns
 constexpr int kTmO = 256;        // O: 256 columns (after the two S buffers of 128)
@@ -74,7 +84,7 @@ constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQBoxes * kBox;
 constexpr int kOffV = kOffK + kKTile;
 constexpr int kOffP = kOffV + kVStages * kVStage;
-constexpr int kOffBar = kOffP + 4 * kBox;  // two P buffers (tile parity) of 2 boxes
+constexpr int kOffBar = kOffP + 2 * kBox;  // one P buffer of 2 boxes
 
 enum Bar {
     B_QFULL = 0, B_QEMPTY, B_SFULL0, B_SFULL1, B_SEMPTY0, B_SEMPTY1, B_PFULL0, B_PFULL1, B_PVDONE0, B_PVDONE1,
@@ -96,11 +106,14 @@ struct Params {
     const int32_t* part_offsets;
     const int32_t* context_lens;
     const int32_t* block_table;
+    const uint8_t* pool;  // the cache rows (for the L2 prefetch of upcoming pages)
     uint16_t* o_part;  // [n_parts, 128, 512] bf16 (normalised partial outputs)
     float* lse_part;  // [n_parts, 128]
     int64_t num_blocks;
     int32_t batch, max_blocks_per_seq, block_size, q_len;
     float scale_log2;  // softmax_scale * log2(e)
+    uint64_t wait_ns;  // limit of every bounded wait (ptx::kWaitLimitNs unless a test shortens it)
+    int32_t starve;    // test hook: the load warps issue nothing, so every consumer wait runs out
 };
 
 struct Ctx {
@@ -110,6 +123,7 @@ struct Ctx {
     uint32_t pair;
     uint32_t tmem;
     volatile int* abort;
+    uint64_t wait_ns;  // limit of every mbarrier wait
     __device__ uint32_t bar(int i) const { return sbase + kOffBar + 8 * i; }
     __device__ uint32_t leader_bar(int i) const { return ptx::mapa(bar(i), 0); }
 };
@@ -122,19 +136,35 @@ __device__ __forceinline__ void ring_next(uint32_t& stage, uint32_t& phase) {
     if (++stage == N) { stage = 0; phase ^= 1; }
 }
 
+// Starts pulling this CTA's 64-token page of tile j of `seg` (73,728
+// contiguous bytes: the 64 rows lie in one pool block because block_size is a
+// multiple of 64) from HBM into L2, so that its key loads a tile later hit L2.
+__device__ __forceinline__ void prefetch_page(const Params& P, const Ctx& c, const Segment& seg, int j) {
+    const int32_t th = seg.tok_begin + j * kTile + 64 * static_cast<int32_t>(c.rank);
+    if (th >= seg.tok_end) return;
+    const int64_t row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks, P.block_size,
+                                    seg.group / P.q_len, th);
+    if (row >= 0) ptx::prefetch_l2(P.pool + row * (kD * 2), 64 * kD * 2);
+}
+
 // Queries and key stages; one thread (lane 0 of warp 0). tm_q, tm_k3 and
 // tm_k2 are 3-D maps {64 columns, rows, 9 column blocks} with boxes
 // {64, 64, 9}, {64, 64, 3} and {64, 64, 2}: one TMA operation fills the whole
-// query block or a key stage.
+// query block or a key stage. Before the loads of tile j it asks L2 for the
+// page of the tile after it (in this segment or the next).
 __device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUtensorMap* tm_k3,
                              const CUtensorMap* tm_k2, const Ctx& c) {
     uint32_t phase = 0;  // parity of the pair's running tile count
     int seg_i = 0;
     SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
     Segment seg;
+    {
+        SegmentIter peek = it;
+        if (peek.next(seg)) prefetch_page(P, c, seg, 0);
+    }
     while (it.next(seg)) {
         const int32_t g = seg.group, b = g / P.q_len;
-        if (seg_i > 0 && !ptx::mbar_wait(c.bar(B_QEMPTY), (seg_i - 1) & 1, c.abort)) return;
+        if (seg_i > 0 && !ptx::mbar_wait(c.bar(B_QEMPTY), (seg_i - 1) & 1, c.abort, c.wait_ns)) return;
         {
             const uint32_t full = c.leader_bar(B_QFULL);
             ptx::mbar_arrive_expect_tx_cluster(full, kQBoxes * kBox);
@@ -152,8 +182,15 @@ __device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUt
                 record_status(MLA_ERR_DEVICE_FAULT);
                 row = 0;
             }
+            if (j + 1 < n_tiles) {
+                prefetch_page(P, c, seg, j + 1);
+            } else {
+                SegmentIter peek = it;
+                Segment nx;
+                if (peek.next(nx)) prefetch_page(P, c, nx, 0);
+            }
             for (int ks = 0; ks < kKStages; ++ks) {
-                if (!ptx::mbar_wait(c.bar(B_KEMPTY0 + ks), phase ^ 1, c.abort)) return;
+                if (!ptx::mbar_wait(c.bar(B_KEMPTY0 + ks), phase ^ 1, c.abort, c.wait_ns)) return;
                 const uint32_t full = c.leader_bar(B_KFULL0 + ks);
                 const int blk = kstage_first_block(ks);
                 ptx::mbar_arrive_expect_tx_cluster(full, kstage_blocks(ks) * kBox);
@@ -169,8 +206,8 @@ __device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUt
     // reach this CTA's shared memory after it exits -- it would land in the
     // barriers of whatever CTA runs here next.
     for (int ks = 0; ks < kKStages; ++ks)
-        if (!ptx::mbar_wait(c.bar(B_KEMPTY0 + ks), phase ^ 1, c.abort)) return;
-    if (seg_i > 0) ptx::mbar_wait(c.bar(B_QEMPTY), (seg_i - 1) & 1, c.abort);
+        if (!ptx::mbar_wait(c.bar(B_KEMPTY0 + ks), phase ^ 1, c.abort, c.wait_ns)) return;
+    if (seg_i > 0) ptx::mbar_wait(c.bar(B_QEMPTY), (seg_i - 1) & 1, c.abort, c.wait_ns);
 }
 
 // Value stages; warp 2 (lane 0 issues and waits, the whole warp zeroes the
@@ -186,7 +223,7 @@ __device__ void value_producer(const Params& P, const CUtensorMap* tm_v, const C
     // a wait by lane 0, its outcome shared so that the warp stays converged
     auto wait0 = [&](uint32_t bar, uint32_t parity) -> bool {
         int ok = 1;
-        if (lane == 0) ok = ptx::mbar_wait(bar, parity, c.abort) ? 1 : 0;
+        if (lane == 0) ok = ptx::mbar_wait(bar, parity, c.abort, c.wait_ns) ? 1 : 0;
         return __shfl_sync(0xffffffffu, ok, 0) != 0;
     };
     SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
@@ -245,13 +282,10 @@ __device__ void value_producer(const Params& P, const CUtensorMap* tm_v, const C
 }
 
 // ------------------------------------------------------------------- MMA
-// Three issuing threads in the leader CTA: two for the score MMAs (one per
-// half of the contraction, each with its own half-accumulator) and one for the
-// value MMAs. A single thread
-// issues at most about one tcgen05.mma every ~47 cycles, while an
-// M 128 x N 128 x K 16 pair instruction takes the tensor cores 32 cycles, and
-// the three streams are independent (different TMEM accumulators, operands
-// and barriers).
+// Two issuing threads in the leader CTA (half 0: lane 0 of warp 1, half 1:
+// lane 0 of warp 3). A single thread issues at most about one tcgen05.mma every
+// ~47 cycles, while an M 128 x N 128 x K 16 pair instruction takes the tensor
+// cores 32 cycles; two threads with independent accumulators keep up.
 struct Descs {
     uint64_t dq, dk, dp, dv;
     __device__ explicit Descs(const Ctx& c)
@@ -262,33 +296,44 @@ struct Descs {
           dv(ptx::smem_desc_sw128(c.sbase + kOffV, kBox / 2, 1024)) {}
 };
 
-// Partial scores S_half = Q[:, blocks] K[:, blocks]^T of every tile, into the
-// half-accumulator `half` of S buffer (tile & 1); one thread per half (lane 0
-// of warp 1: blocks 0-4, key stages 0-1; lane 0 of warp 3: blocks 5-8, key
-// stages 2-3), so that the two threads issue the 36 score instructions of a
-// tile concurrently. Each key stage is consumed by one thread only, once per
-// tile (phase = tile parity). Both threads commit QEMPTY once per segment (the
-// barrier counts 2) and SFULL once per tile (it counts 2).
-__device__ void mma_s_issuer(const Params& P, const Ctx& c, uint32_t half) {
+// Both threads run the same program over the pair's tiles n (counted across
+// segments): the score MMAs of tile n, then the value MMAs of tile n - 1.
+//   score, half h: S_h = Q[:, blocks] K[:, blocks]^T over column blocks 0-4
+//     (h = 0: key stages 0-1) or 5-8 (h = 1: stages 2-3) into half-accumulator
+//     h of S buffer (n & 1); each key stage is consumed by one thread, once
+//     per tile (phase = tile parity). QEMPTY (count 2) is committed once per
+//     segment by each thread, SFULL (count 2) once per tile.
+//   value, half h: O[:, 256h .. 256h + 255] += P V over the tile's visible
+//     32-token value stages (stage q: tokens 32q..32q+31); both threads read
+//     every value stage and commit its VEMPTY (count 2), and PVDONE (count 2)
+//     once per tile. The first value MMA of a segment overwrites O, after the
+//     softmax has read out the previous segment (OEMPTY).
+__device__ void mma_issuer(const Params& P, const Ctx& c, uint32_t half) {
     constexpr uint32_t kIdS = ptx::idesc_bf16(128, 128, false, false);
+    constexpr uint32_t kIdPV = ptx::idesc_bf16(128, 256, false, true);
     const Descs D(c);
-    uint32_t tile_cnt = 0;
-    int seg_i = 0;
-    SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
-    Segment seg;
-    while (it.next(seg)) {
-        if (!ptx::mbar_wait(c.bar(B_QFULL), seg_i & 1, c.abort)) return;
-        ptx::tc_fence_after();
-        const int n_tiles = tiles_of(seg);
-        for (int j = 0; j < n_tiles; ++j, ++tile_cnt) {
-            const uint32_t sb = tile_cnt & 1;
-            const uint32_t d_s = c.tmem + kTmS + 128 * sb + 64 * half;
-            if (!ptx::mbar_wait(c.bar(B_SEMPTY0 + sb), ((tile_cnt >> 1) & 1) ^ 1, c.abort)) return;
-#pragma unroll 1
-            for (int ks = 2 * static_cast<int>(half); ks < 2 * static_cast<int>(half) + 2; ++ks) {
-                if (!ptx::mbar_wait(c.bar(B_KFULL0 + ks), tile_cnt & 1, c.abort)) return;
+    const int ks0 = 2 * static_cast<int>(half);
+    const int k_first = kstage_first_block(ks0);
+    SegmentIter its(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    SegmentIter itv = its;
+    Segment ss, sv;
+    bool have_s = its.next(ss), have_v = itv.next(sv);
+    int s_seg = 0, s_j = 0, v_seg = 0, v_j = 0;
+    uint32_t s_cnt = 0, v_cnt = 0, vst = 0, vph = 0;
+    while (have_s || have_v) {
+        if (have_s) {
+            // ---- score MMAs of tile s_cnt
+            if (s_j == 0) {
+                if (!ptx::mbar_wait(c.bar(B_QFULL), s_seg & 1, c.abort, c.wait_ns)) return;
                 ptx::tc_fence_after();
-                const int k_first = kstage_first_block(0 + 2 * static_cast<int>(half));
+            }
+            const uint32_t sb = s_cnt & 1;
+            const uint32_t d_s = c.tmem + kTmS + 128 * sb + 64 * half;
+            if (!ptx::mbar_wait(c.bar(B_SEMPTY0 + sb), ((s_cnt >> 1) & 1) ^ 1, c.abort, c.wait_ns)) return;
+#pragma unroll 1
+            for (int ks = ks0; ks < ks0 + 2; ++ks) {
+                if (!ptx::mbar_wait(c.bar(B_KFULL0 + ks), s_cnt & 1, c.abort, c.wait_ns)) return;
+                ptx::tc_fence_after();
                 for (int k = kstage_first_block(ks); k < kstage_first_block(ks) + kstage_blocks(ks); ++k) {
                     const uint64_t a0 = D.dq + static_cast<uint64_t>((k * kBox) >> 4);
                     const uint64_t b0 = D.dk + static_cast<uint64_t>((k * kBox) >> 4);
@@ -299,63 +344,66 @@ __device__ void mma_s_issuer(const Params& P, const Ctx& c, uint32_t half) {
                 ptx::mma_commit_pair(c.bar(B_KEMPTY0 + ks), 0x3);
             }
             ptx::mma_commit_pair(c.bar(B_SFULL0 + sb), 0x3);
+            ++s_cnt;
+            if (++s_j == tiles_of(ss)) {
+                ptx::mma_commit_pair(c.bar(B_QEMPTY), 0x3);
+                ++s_seg;
+                s_j = 0;
+                have_s = its.next(ss);
+            }
         }
-        ptx::mma_commit_pair(c.bar(B_QEMPTY), 0x3);
-        ++seg_i;
-    }
-}
-
-// O += P V for every tile; one thread (lane 0 of warp 8 of the leader CTA).
-__device__ void mma_pv_issuer(const Params& P, const Ctx& c) {
-    constexpr uint32_t kIdPV = ptx::idesc_bf16(128, 256, false, true);
-    const Descs D(c);
-    uint32_t vst = 0, vph = 0, pv_cnt = 0;
-    int seg_i = 0;
-    SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
-    Segment seg;
-    while (it.next(seg)) {
-        const int n_tiles = tiles_of(seg);
-        for (int j = 0; j < n_tiles; ++j) {
-            const bool first = (j == 0);
-            const uint32_t pb = pv_cnt & 1;  // P buffer of this tile
-            if (!ptx::mbar_wait(c.bar(B_PFULL0 + pb), (pv_cnt >> 1) & 1, c.abort)) return;
-            if (first && !ptx::mbar_wait(c.bar(B_OEMPTY), (seg_i & 1) ^ 1, c.abort)) return;
-            const int32_t tv = seg.tok_begin + j * kTile;
+        if (have_v && (v_cnt + 1 < s_cnt || !have_s)) {
+            // ---- value MMAs of tile v_cnt (its weights are in the P buffer)
+            const bool first = (v_j == 0);
+            if (!ptx::mbar_wait(c.bar(B_PFULL0 + (v_cnt & 1)), (v_cnt >> 1) & 1, c.abort, c.wait_ns)) return;
+            if (first && !ptx::mbar_wait(c.bar(B_OEMPTY), (v_seg & 1) ^ 1, c.abort, c.wait_ns)) return;
+            const int32_t tv = sv.tok_begin + v_j * kTile;
             for (int q = 0; q < kVPerTile; ++q) {
-                if (seg.tok_end - (tv + 32 * q) <= 0) break;  // no visible token: skipped by the producer too
-                if (!ptx::mbar_wait(c.bar(B_VFULL0 + vst), vph, c.abort)) return;
+                if (sv.tok_end - (tv + 32 * q) <= 0) break;  // no visible token: skipped by the producer too
+                if (!ptx::mbar_wait(c.bar(B_VFULL0 + vst), vph, c.abort, c.wait_ns)) return;
                 ptx::tc_fence_after();
                 // A: P tokens 32q + 16kk .. +15 (box q/2, byte 64 (q&1) + 32 kk of each 128-byte row)
-                const uint64_t a0 = D.dp + static_cast<uint64_t>(((2 * pb + (q >> 1)) * kBox + 64 * (q & 1)) >> 4);
-                const uint64_t b0 = D.dv + static_cast<uint64_t>((vst * kVStage) >> 4);
+                const uint64_t a0 = D.dp + static_cast<uint64_t>(((q >> 1) * kBox + 64 * (q & 1)) >> 4);
+                const uint64_t b0 = D.dv + static_cast<uint64_t>((vst * kVStage + half * kBox) >> 4);
 #pragma unroll
-                for (int n = 0; n < 2; ++n)
-#pragma unroll
-                    for (int kk = 0; kk < 2; ++kk)
-                        ptx::mma_bf16_pair(c.tmem + kTmO + 128 * n, a0 + 2 * kk,
-                                           b0 + static_cast<uint64_t>((n * kBox + 2048 * kk) >> 4), kIdPV,
-                                           !(first && q == 0 && kk == 0));
+                for (int kk = 0; kk < 2; ++kk)
+                    ptx::mma_bf16_pair(c.tmem + kTmO + 128 * half, a0 + 2 * kk,
+                                       b0 + static_cast<uint64_t>((2048 * kk) >> 4), kIdPV,
+                                       !(first && q == 0 && kk == 0));
                 ptx::mma_commit_pair(c.bar(B_VEMPTY0 + vst), 0x3);
                 ring_next<kVStages>(vst, vph);
             }
-            ptx::mma_commit_pair(c.bar(B_PVDONE0 + pb), 0x3);
-            ++pv_cnt;
+            ptx::mma_commit_pair(c.bar(B_PVDONE0 + (v_cnt & 1)), 0x3);
+            ++v_cnt;
+            if (++v_j == tiles_of(sv)) {
+                ++v_seg;
+                v_j = 0;
+                have_v = itv.next(sv);
+            }
         }
-        ++seg_i;
     }
 }
 
 // --------------------------------------------------------------- softmax
+// The softmax warps execute warp-collective tensor-memory instructions
+// (tcgen05.ld / st .sync.aligned), so every branch they take must be
+// warp-uniform: a wait succeeds for the whole warp or for none of it (a lane
+// that gave up makes its warp give up), and the O rescale runs for the whole
+// warp when any of its rows needs it.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
+    return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, limit_ns));
+}
+
 struct Exchanger {  // swaps one float between thread t and thread t ^ 64 of the softmax warps
     float* red;
     uint32_t bar;
     uint32_t n = 0;
-    __device__ bool swap(float v, float& partner, int t, volatile int* abort) {
+    __device__ bool swap(float v, float& partner, int t, volatile int* abort, uint64_t limit_ns) {
         float* buf = red + (n & 1) * 128;
         buf[t] = v;
         __syncwarp();
         if (ptx::lane_id() == 0) ptx::mbar_arrive_local(bar);
-        if (!ptx::mbar_wait(bar, n & 1, abort)) return false;
+        if (!warp_wait(bar, n & 1, abort, limit_ns)) return false;
         partner = buf[t ^ 64];
         ++n;
         return true;
@@ -376,12 +424,12 @@ __device__ void softmax(const Params& P, const Ctx& c) {
     uint32_t tile_cnt = 0;
     // Value MMAs of the pair's tile k signal PVDONE[k & 1] (phase k >> 1). pv_done is the
     // highest k known complete (a completion implies every earlier one). Each wait is at
-    // most one phase behind its barrier: tile k + 2's value MMAs need the P this thread
+    // most one phase behind its barrier: tile k + 1's value MMAs need the P this thread
     // writes after the wait.
     int32_t pv_done = -1;
     auto wait_pv = [&](int32_t k) -> bool {
         if (k <= pv_done) return true;
-        if (!ptx::mbar_wait(c.bar(B_PVDONE0 + (k & 1)), (static_cast<uint32_t>(k) >> 1) & 1, c.abort)) return false;
+        if (!warp_wait(c.bar(B_PVDONE0 + (k & 1)), (static_cast<uint32_t>(k) >> 1) & 1, c.abort, c.wait_ns)) return false;
         pv_done = k;
         return true;
     };
@@ -393,7 +441,7 @@ __device__ void softmax(const Params& P, const Ctx& c) {
         for (int j = 0; j < n_tiles; ++j) {
             const int32_t tc = static_cast<int32_t>(tile_cnt);
             const uint32_t sb = tile_cnt & 1;
-            if (!ptx::mbar_wait(c.bar(B_SFULL0 + sb), (tile_cnt >> 1) & 1, c.abort)) return;
+            if (!warp_wait(c.bar(B_SFULL0 + sb), (tile_cnt >> 1) & 1, c.abort, c.wait_ns)) return;
             ptx::tc_fence_after();
             float s[64];
             {
@@ -429,7 +477,7 @@ __device__ void softmax(const Params& P, const Ctx& c) {
             // the scale is positive, so the max of the raw scores gives the max of the scaled ones
             const float mloc = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale_log2;
             float mpart;
-            if (!xc.swap(mloc, mpart, t, c.abort)) return;
+            if (!xc.swap(mloc, mpart, t, c.abort, c.wait_ns)) return;
             const float m_tile = fmaxf(mloc, mpart);
             const float m_new = fmaxf(m_run, m_tile);
             const bool rescale = m_new > m_run + 8.f;  // keep a stale max unless it grows by > 2^8
@@ -443,7 +491,9 @@ __device__ void softmax(const Params& P, const Ctx& c) {
                 ps[i & 3] += s[i];
             }
             l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-            if (j > 0 && rescale) {  // O is rescaled once the previous tile's value MMAs are done
+            // O is rescaled once the previous tile's value MMAs are done, by the whole warp
+            // (alpha = 1 in the rows that keep their max)
+            if (j > 0 && __any_sync(0xffffffffu, rescale)) {
                 if (!wait_pv(tc - 1)) return;
                 ptx::tc_fence_after();
 #pragma unroll 1
@@ -457,10 +507,10 @@ __device__ void softmax(const Params& P, const Ctx& c) {
                 }
                 ptx::tmem_wait_st();
             }
-            // this tile's P buffer was last read by the value MMAs of tile tc - 2
-            if (tc >= 2 && !wait_pv(tc - 2)) return;
+            // the P buffer was last read by the value MMAs of tile tc - 1
+            if (tc >= 1 && !wait_pv(tc - 1)) return;
             ptx::tc_fence_after();
-            uint8_t* const prow = c.smem + kOffP + (2 * sb + half) * kBox + hrow * 128;
+            uint8_t* const prow = c.smem + kOffP + half * kBox + hrow * 128;
             // P row (bf16) into the K-major 128B-swizzled A operand of the PV MMA
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8) {
@@ -481,7 +531,7 @@ __device__ void softmax(const Params& P, const Ctx& c) {
         if (!wait_pv(static_cast<int32_t>(tile_cnt) - 1)) return;
         ptx::tc_fence_after();
         float lpart;
-        if (!xc.swap(l_run, lpart, t, c.abort)) return;
+        if (!xc.swap(l_run, lpart, t, c.abort, c.wait_ns)) return;
         const float l_tot = l_run + lpart;
         const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
         // O rows go out, rounded to bf16, through the (now idle) P buffers: each thread
@@ -531,7 +581,7 @@ __device__ void softmax(const Params& P, const Ctx& c) {
 }
 
 // ------------------------------------------------------------------ kernel
-// grid: 2 * workers CTAs (clusters of 2); block 256; dynamic smem kSmemBytes.
+// grid: 2 * workers CTAs (clusters of 2); block kThreads; dynamic smem kSmemBytes.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     pair_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k3,
                        const __grid_constant__ CUtensorMap tm_k2, const __grid_constant__ CUtensorMap tm_v,
@@ -546,6 +596,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     c.rank = ptx::cluster_ctarank();
     c.pair = ptx::cluster_id_x();
     c.abort = reinterpret_cast<volatile int*>(smem + kOffMisc);
+    c.wait_ns = P.wait_ns;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc + 16);
 
     if (threadIdx.x == 0) {
@@ -558,8 +609,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ptx::mbar_init(c.bar(B_SEMPTY1), 8);
         ptx::mbar_init(c.bar(B_PFULL0), 8);
         ptx::mbar_init(c.bar(B_PFULL1), 8);
-        ptx::mbar_init(c.bar(B_PVDONE0), 1);
-        ptx::mbar_init(c.bar(B_PVDONE1), 1);
+        ptx::mbar_init(c.bar(B_PVDONE0), 2);
+        ptx::mbar_init(c.bar(B_PVDONE1), 2);
         ptx::mbar_init(c.bar(B_OEMPTY), 8);
         ptx::mbar_init(c.bar(B_PATCH), 1);
         ptx::mbar_init(c.bar(B_XCHG), 4);
@@ -569,7 +620,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < kVStages; ++s) {
             ptx::mbar_init(c.bar(B_VFULL0 + s), 2);
-            ptx::mbar_init(c.bar(B_VEMPTY0 + s), 1);
+            ptx::mbar_init(c.bar(B_VEMPTY0 + s), 2);
         }
         ptx::fence_mbar_init();
     }
@@ -592,13 +643,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     pdl_trigger();
 
     if (warp == 0) {
-        if (ptx::lane_id() == 0) key_producer(P, &tm_q, &tm_k3, &tm_k2, c);
+        if (ptx::lane_id() == 0 && !P.starve) key_producer(P, &tm_q, &tm_k3, &tm_k2, c);
     } else if (warp == 2) {
-        value_producer(P, &tm_v, c);
+        if (!P.starve) value_producer(P, &tm_v, c);
     } else if (warp == 1 || warp == 3) {
-        if (c.rank == 0 && ptx::lane_id() == 0) mma_s_issuer(P, c, static_cast<uint32_t>(warp >> 1));
-    } else if (warp == 8) {
-        if (c.rank == 0 && ptx::lane_id() == 0) mma_pv_issuer(P, c);
+        if (c.rank == 0 && ptx::lane_id() == 0) mma_issuer(P, c, static_cast<uint32_t>(warp >> 1));
     } else if (warp >= 4) {
         softmax(P, c);
     }

@@ -193,7 +193,8 @@ __global__ void __launch_bounds__(kThreads, 1) uv_kernel(const __grid_constant__
         ptx::mma_commit_1(bar_addr(smem, off_bar, 2 * kUvStages));
     }
     // epilogue: thread t = TMEM lane t = token row g0 + t
-    const bool ok = ptx::mbar_wait(bar_addr(smem, off_bar, 2 * kUvStages), 0, abort);
+    // warp-uniform (the tensor-memory loads below are warp-collective)
+    const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_addr(smem, off_bar, 2 * kUvStages), 0, abort));
     ptx::tc_fence_after();
     if (ok) {
         const int g = g0 + static_cast<int>(threadIdx.x);
@@ -438,7 +439,8 @@ __global__ void __launch_bounds__(kMuvThreads, 1) merge_uv_kernel(const __grid_c
     // ---- epilogue: thread t < 128 = TMEM lane t = output column d; TMEM column j = group g0 + j.
     // D goes through shared memory (stage 0, free once every MMA is done) as bf16 [64 groups][128]
     // so that the stores are whole 16-byte pieces of the output rows.
-    const bool done = ptx::mbar_wait(bar_addr(smem, off_bar, 2 * kMuvStages), 0, abort) && !*abort;
+    const bool done =
+        __all_sync(0xffffffffu, ptx::mbar_wait(bar_addr(smem, off_bar, 2 * kMuvStages), 0, abort) && !*abort);
     ptx::tc_fence_after();
     uint16_t* stg = reinterpret_cast<uint16_t*>(smem);
     if (warp < 4) {
@@ -552,7 +554,7 @@ __global__ void __launch_bounds__(kThreads) absorb_kernel(const __grid_constant_
         for (int i = 0; i < kPe; ++i)
             if (i < dr / 8) pe[i] = src[i];
     }
-    const bool ok = ptx::mbar_wait(done, 0, abort);
+    const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(done, 0, abort));  // warp-uniform
     ptx::tc_fence_after();
     if (ok) {
         const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
@@ -681,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 1) append_kernel(const __grid_consta
     // thread t = TMEM lane t = token row m0 + t: the CTA's partial tile into shared memory
     // (row t: 64 floats = 16 chunks of 16 B, chunk c at (c ^ (t & 15)) to spread the banks);
     // the ring is free once every MMA is done
-    const bool ok = ptx::mbar_wait(bar_addr(smem, off_bar, 2 * kApStages), 0, abort);
+    const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_addr(smem, off_bar, 2 * kApStages), 0, abort));
     ptx::tc_fence_after();
     const int t = static_cast<int>(threadIdx.x);
     float* red = reinterpret_cast<float*>(smem);

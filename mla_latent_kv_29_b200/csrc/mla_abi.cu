@@ -16,7 +16,6 @@
 #include "decode_generic.cuh"
 #include "append.cuh"
 #include "decode_pair.cuh"
-#include "gemm_small.cuh"
 #include "gemm_tc05.cuh"
 #include "qproj.cuh"
 
@@ -250,14 +249,6 @@ int ensure_smem(K kernel, size_t bytes) {
         return MLA_ERR_CUDA;
     }
     return MLA_OK;
-}
-
-// ---- tensor-core GEMM eligibility ------------------------------------
-// absorb: d_n multiple of 16 (<= 256), d_c multiple of 128; up-projection:
-// d_v multiple of 64 and the [64 + d_v, d_c + 8] bf16 tiles within 227 KB.
-bool tc_gemm_dims_ok(const mla_dims_t* d) {
-    return d->qk_nope_dim % 16 == 0 && d->qk_nope_dim <= 256 && d->kv_lora_rank % 128 == 0 &&
-           d->v_head_dim % 64 == 0 && uv_tc_smem(d->kv_lora_rank, d->v_head_dim) <= 227 * 1024 && d->kv_lora_rank <= 512;
 }
 
 // ---- append split-K plan ----------------------------------------------
@@ -528,10 +519,13 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     const int32_t G = batch * q_len;
     const int H = dims->num_heads, dc = dims->kv_lora_rank, dr = dims->rope_dim;
 
-    const bool tc = tc_gemm_dims_ok(dims) && aligned(q_nope, 16) && aligned(w_uk, 16) && aligned(w_uv, 16) &&
-                    aligned(out, 16);
-    // the tensor-core kernel writes bf16 partials, which only the tensor-core merge reads
-    if (L.kernel == kKernelPair && !tc) return MLA_ERR_INVALID_ARG;
+    // The tcgen05 absorption, merge and up-projection kernels take their
+    // operands through TMA (16-byte aligned); other dims or alignments use the
+    // CUDA-core kernels. The tensor-core attention writes bf16 partials, which
+    // only the tcgen05 merge reads, so it needs the tcgen05 kernels around it.
+    const bool tc05 = tc05_dims_ok(dims) && aligned(q_nope, 16) && aligned(q_pe, 16) && aligned(w_uk, 16) &&
+                      aligned(w_uv, 16) && aligned(out, 16);
+    if (L.kernel == kKernelPair && !tc05) return MLA_ERR_INVALID_ARG;
 
     const size_t plan_smem = sizeof(int32_t) * (static_cast<size_t>(G) + 1);
     const int32_t prefix_in_smem = plan_smem <= 48 * 1024 ? 1 : 0;
@@ -539,7 +533,6 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
                         L.workers, hdr, tile_prefix, part_offsets, worker_group, prefix_in_smem)) return rc;
     if (int rc = launch_status()) return rc;
 
-    const bool tc05 = tc && tc05_dims_ok(dims) && aligned(q_pe, 16);
     if (tc05) {
         CUtensorMap tm_qn, tm_wuk;
         if (int rc = encode_2d(&tm_qn, q_nope, static_cast<uint64_t>(H) * dims->qk_nope_dim, G, tc05::kRows)) return rc;
@@ -549,12 +542,6 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         if (int rc = ensure_smem(tc05::absorb_kernel, smem)) return rc;
         if (int rc = launch(tc05::absorb_kernel, dim3(H, (G + tc05::kRows - 1) / tc05::kRows, dc / 256), tc05::kThreads, smem, st,
             tm_qn, tm_wuk, static_cast<const uint16_t*>(q_pe), G, H, dims->qk_nope_dim, dc, dr, q)) return rc;
-    } else if (tc) {
-        const size_t smem = absorb_tc_smem(dims->qk_nope_dim);
-        if (int rc = ensure_smem(absorb_tc_kernel, smem)) return rc;
-        if (int rc = launch(absorb_tc_kernel, dim3(H, dc / 128, (G + kTcRows - 1) / kTcRows), kTcThreads, smem, st,
-            static_cast<const uint16_t*>(q_nope), static_cast<const uint16_t*>(q_pe),
-            static_cast<const uint16_t*>(w_uk), q, G, H, dims->qk_nope_dim, dc, dr)) return rc;
     } else {
         const size_t absorb_smem = sizeof(float) * kAbsorbGroups * dims->qk_nope_dim;
         if (int rc = ensure_smem(absorb_q_kernel, absorb_smem)) return rc;
@@ -578,6 +565,7 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         PP.part_offsets = part_offsets;
         PP.context_lens = context_lens;
         PP.block_table = block_table;
+        PP.pool = static_cast<const uint8_t*>(pool);
         PP.o_part = reinterpret_cast<uint16_t*>(o_part);  // bf16 partials (the slot layout keeps fp32 size)
         PP.lse_part = lse_part;
         PP.num_blocks = num_blocks;
@@ -586,6 +574,8 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         PP.block_size = dims->block_size;
         PP.q_len = q_len;
         PP.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
+        PP.wait_ns = (opts && opts->debug_wait_limit_us) ? 1000ull * opts->debug_wait_limit_us : ptx::kWaitLimitNs;
+        PP.starve = (opts && opts->debug_starve) ? 1 : 0;
         if (int rc = ensure_smem(pair::pair_decode_kernel, pair::kSmemBytes)) return rc;
         if (int rc = wait_hook(opts ? opts->cache_ready : nullptr, st)) return rc;
         record_hook(opts ? opts->event_attn_begin : nullptr, st);
@@ -658,20 +648,6 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         if (int rc = ensure_smem(tc05::uv_kernel, smem)) return rc;
         if (int rc = launch(tc05::uv_kernel, dim3(H, (G + tc05::kRows - 1) / tc05::kRows), tc05::kThreads, smem, st,
             tm_ol, tm_wuv, G, H, dc, dims->v_head_dim, static_cast<uint16_t*>(out))) return rc;
-    } else if (tc) {
-        const size_t smem = uv_tc_smem(dc, dims->v_head_dim);
-        const dim3 grid(H, (G + kTcRows - 1) / kTcRows);
-        uint16_t* o = static_cast<uint16_t*>(out);
-        const uint16_t* wv = static_cast<const uint16_t*>(w_uv);
-        if (L.kernel == kKernelPair) {  // bf16 partials
-            if (int rc = ensure_smem(merge_uv_tc_kernel<uint16_t>, smem)) return rc;
-            if (int rc = launch(merge_uv_tc_kernel<uint16_t>, grid, kTcThreads, smem, st,
-                reinterpret_cast<const uint16_t*>(o_part), lse_part, part_offsets, wv, G, H, dc, dims->v_head_dim, o)) return rc;
-        } else {
-            if (int rc = ensure_smem(merge_uv_tc_kernel<float>, smem)) return rc;
-            if (int rc = launch(merge_uv_tc_kernel<float>, grid, kTcThreads, smem, st, o_part, lse_part, part_offsets, wv, G, H, dc,
-                                                                     dims->v_head_dim, o)) return rc;
-        }
     } else {
         const size_t uv_smem = sizeof(float) * kUvGroups * dc;
         if (int rc = ensure_smem(combine_uv_kernel, uv_smem)) return rc;
@@ -713,29 +689,66 @@ int mla_debug_resolve_slots(const mla_dims_t* dims, const int32_t* block_table, 
 // that cannot allocate device memory themselves (see mla_b200.h). Host code
 // must not pass `g_no_alloc_scratch` itself to a kernel: on the host that
 // name is only a stand-in for the symbol. The device address is looked up
-// with cudaGetSymbolAddress once per device, with that device current.
+// with cudaGetSymbolAddress once per CUDA context, with that context current,
+// and cached under the context's process-unique id (cuCtxGetId), so that a
+// context created later (another device, a driver-API context, the primary
+// context re-created after cudaDeviceReset) never sees a stale address.
 namespace mla {
 namespace {
 
 static __device__ __align__(256) unsigned char g_no_alloc_scratch[MLA_NO_ALLOC_SCRATCH_BYTES];
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename F>
+F driver_fn(const char* name) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return reinterpret_cast<F>(p);
+}
+
+// Process-unique id of the current context; false if none is current.
+bool current_context_id(unsigned long long* id) {
+    static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    CUcontext ctx = nullptr;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+struct ScratchEntry {
+    unsigned long long ctx_id;
+    void* ptr;
+};
 std::mutex g_no_alloc_mutex;
-void* g_no_alloc_ptr[64] = {nullptr};
+ScratchEntry g_no_alloc_cache[64] = {};
+int g_no_alloc_next = 0;
 
 int no_alloc_scratch(void** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return MLA_ERR_NO_DEVICE; }
-    if (dev < 0 || dev >= 64) return MLA_ERR_NO_DEVICE;
     std::lock_guard<std::mutex> lock(g_no_alloc_mutex);
-    if (!g_no_alloc_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_no_alloc_scratch) != cudaSuccess || p == nullptr) {
-            cudaGetLastError();
-            return MLA_ERR_CUDA;
-        }
-        g_no_alloc_ptr[dev] = p;
+    unsigned long long id = 0;
+    const bool have_id = current_context_id(&id);
+    if (have_id)
+        for (const ScratchEntry& e : g_no_alloc_cache)
+            if (e.ptr && e.ctx_id == id) {
+                *out = e.ptr;
+                return MLA_OK;
+            }
+    void* p = nullptr;  // first call in this context (the look-up makes the runtime's context current)
+    if (cudaGetSymbolAddress(&p, g_no_alloc_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
     }
-    *out = g_no_alloc_ptr[dev];
+    if (have_id || current_context_id(&id)) {
+        g_no_alloc_cache[g_no_alloc_next] = ScratchEntry{id, p};
+        g_no_alloc_next = (g_no_alloc_next + 1) % 64;
+    }
+    *out = p;
     return MLA_OK;
 }
 

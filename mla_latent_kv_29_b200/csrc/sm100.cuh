@@ -105,17 +105,18 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with parity `parity` to complete. Gives up after
-// kWaitLimitNs (or at once if *abort is already set), records
-// MLA_ERR_DEVICE_TIMEOUT, sets *abort and returns false.
+// limit_ns (default kWaitLimitNs; or at once if *abort is already set),
+// records MLA_ERR_DEVICE_TIMEOUT, sets *abort and returns false.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             *abort = 1;
             record_status(MLA_ERR_DEVICE_TIMEOUT);
             return false;

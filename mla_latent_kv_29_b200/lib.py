@@ -48,7 +48,8 @@ class CDims(ctypes.Structure):
 class CDecodeOpts(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("num_workers", ctypes.c_int32),
                 ("event_attn_begin", ctypes.c_void_p), ("event_attn_end", ctypes.c_void_p),
-                ("cache_ready", ctypes.c_void_p)]
+                ("cache_ready", ctypes.c_void_p), ("debug_wait_limit_us", ctypes.c_uint32),
+                ("debug_starve", ctypes.c_int32)]
 
 
 _lib = None
@@ -103,10 +104,11 @@ def _event_handle(ev) -> Optional[int]:
     return ev.cuda_event
 
 
-def c_opts(kernel: int = KERNEL_AUTO, num_workers: int = 0, events=None, cache_ready=None) -> CDecodeOpts:
+def c_opts(kernel: int = KERNEL_AUTO, num_workers: int = 0, events=None, cache_ready=None,
+           debug_wait_limit_us: int = 0, debug_starve: bool = False) -> CDecodeOpts:
     b, e = (None, None) if events is None else (_event_handle(events[0]), _event_handle(events[1]))
     r = None if cache_ready is None else _event_handle(cache_ready)
-    return CDecodeOpts(int(kernel), int(num_workers), b, e, r)
+    return CDecodeOpts(int(kernel), int(num_workers), b, e, r, int(debug_wait_limit_us), int(bool(debug_starve)))
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -201,14 +203,17 @@ def decode_workspace_size(dims: Dims, softmax_scale: float, batch: int, q_len: i
 
 def decode(dims: Dims, softmax_scale: float, q_nope, q_pe, pool, block_table, context_lens,
            max_context_len: int, w_uk, w_uv, out=None, workspace=None, kernel: int = KERNEL_AUTO,
-           num_workers: int = 0, stream=None, attn_events=None, cache_ready=None):
+           num_workers: int = 0, stream=None, attn_events=None, cache_ready=None, debug_wait_limit_us: int = 0,
+           debug_starve: bool = False):
     """attn_events: optional (begin, end) torch.cuda.Event pair recorded around the
     attention kernel on the launch stream. cache_ready: optional torch.cuda.Event
     (already recorded once, so that it has a handle) that the attention launch
-    waits for, e.g. recorded after an append_kv on another stream."""
+    waits for, e.g. recorded after an append_kv on another stream.
+    debug_wait_limit_us / debug_starve: the failure-detection test hooks of
+    mla_decode_opts_t (leave at 0 / False)."""
     lib = load()
     cd = c_dims(dims, softmax_scale)
-    o = c_opts(kernel, num_workers, attn_events, cache_ready)
+    o = c_opts(kernel, num_workers, attn_events, cache_ready, debug_wait_limit_us, debug_starve)
     B, Sq = q_nope.shape[0], q_nope.shape[1]
     if out is None:
         out = torch.empty(B, Sq, dims.num_heads, dims.v_head_dim, dtype=torch.bfloat16, device=q_nope.device)

@@ -241,6 +241,105 @@ def test_append_on_a_side_stream_with_cache_ready():
     np.testing.assert_array_equal(out.float().cpu().numpy(), serial)
 
 
+# --------------------------------------------------- online-softmax rescale
+# The kernels keep a running max per (query, head) and rescale the value
+# accumulator when a later tile's max exceeds it (the tensor-core kernel only
+# when it grows by more than 2^8 in the exp2 domain). N(0,1) data never makes
+# the max grow that much after the first tile, so these cases plant scores
+# that do: every head of a sequence gets the same RoPE query u (head 0's), and
+# chosen cache rows get k_pe += a * u, which adds scale * a * |u|^2 (= delta
+# natural-log units) to that token's score in every head. The pool and the
+# queries are modified on the host before the copy, so the oracle and the GPU
+# read the same bf16 values. Softmax of the absorbed scores: "一次讲透MHA、GQA、
+# MQA、MLA", section "MLA的实现" (forward_inference_absorbed).
+RESCALE_CASES = {
+    # name: (batch, q_len, lengths, spikes [(b, t, delta)], ramp delta per 128 tokens or None)
+    "late_dominant_key": (2, 1, [1000, 700], [(0, 700, 40.0), (1, 450, 20.0)], None),
+    "rising_ramp": (2, 1, [1200, 900], [], 7.0),
+    "slow_ramp": (1, 1, [1500], [], 3.0),
+    "spike_in_partial_last_page": (2, 1, [1000, 333], [(0, 990, 30.0), (1, 330, 25.0)], None),
+    "spike_seen_by_last_new_token_only": (2, 4, [700, 520], [(0, 699, 40.0), (1, 517, 30.0)], None),
+    "dominant_first_tile_then_low": (1, 1, [900], [(0, 5, 40.0)], None),
+}
+
+
+def planted_scores(name):
+    B, sq, lens, spikes, ramp = RESCALE_CASES[name]
+    w, lengths = small_v3("rescale_" + name, B, sq, lens)
+    data = build(w, lengths=lengths)
+    d = w.dims
+    qp = data["q_pe"]
+    qp[:] = qp[:, :1, :1, :]  # one RoPE query per sequence, shared by its new tokens and heads
+    u = qp[:, 0, 0, :].double()  # [B, d_r]
+    unit = 1.0 / (w.softmax_scale * (u * u).sum(-1))  # k_pe += delta * unit * u adds delta to the score
+    flat = data["pool"].view(-1, d.row_width)
+    tab = data["table"].numpy()
+    for b, L in enumerate(lens):
+        if ramp is not None:
+            t = np.arange(L)
+            rows = torch.from_numpy(tab[b, t // d.block_size].astype(np.int64) * d.block_size + t % d.block_size)
+            add = torch.from_numpy(ramp * t / 128.0)[:, None] * unit[b] * u[b][None, :]
+            flat[rows, d.kv_lora_rank:] = (flat[rows, d.kv_lora_rank:].double() + add).to(torch.bfloat16)
+    for b, t, delta in spikes:
+        row = O.resolve_slot(tab, b, t, d.block_size)
+        flat[row, d.kv_lora_rank:] = (flat[row, d.kv_lora_rank:].double() + delta * unit[b] * u[b]).to(torch.bfloat16)
+    return w, data
+
+
+def lazy_rescales(w, data, tile=128, threshold=8.0, margin=1.0):
+    """Tiles (after the first of a group) at which a max kept stale until it
+    is exceeded by more than 2^threshold would be raised, over every (group,
+    head), counting only growths that clear the threshold by `margin` (so
+    that the bf16 rounding of the absorbed query cannot move them below it)."""
+    d = w.dims
+    q_lat = O.absorb_query(data["q_nope"], data["w_uk"])  # [B, Sq, H, d_c]
+    qpe = data["q_pe"].double().numpy()
+    events = 0
+    for b, L in enumerate(data["lengths"].tolist()):
+        c, kpe = O.gather_sequence(data["pool"], data["table"].numpy(), b, L, d)
+        for s in range(w.q_len):
+            n = O.visible_count(L, w.q_len, s)
+            z = w.softmax_scale * (c[:n] @ q_lat[b, s].T + kpe[:n] @ qpe[b, s].T) / math.log(2.0)  # [n, H]
+            m_use = z[:tile].max(0)
+            for j in range(tile, n, tile):
+                m = z[j:j + tile].max(0)
+                events += int(np.sum(m > m_use + threshold + margin))
+                m_use = np.where(m > m_use + threshold, m, m_use)
+    return events
+
+
+@pytest.mark.parametrize("kernel", list(KERNELS))
+@pytest.mark.parametrize("name", list(RESCALE_CASES))
+@pytest.mark.parametrize("workers", [1, 3])
+def test_online_softmax_rescale_matches_oracle(kernel, name, workers):
+    w, data = planted_scores(name)
+    if name != "dominant_first_tile_then_low":
+        assert lazy_rescales(w, data) > 0  # the case does reach the rescale branch
+    got = run_decode(w, to_device(data), kernel=KERNELS[kernel], num_workers=workers)
+    check(got, oracle_out(w, data))
+
+
+# ------------------------------------------------------ failure detection
+def test_bounded_wait_expiry_reports_timeout_and_context_survives():
+    """The tensor-core attention's waits are bounded. With the starve test hook
+    its load warps issue nothing (no copy or tensor-core operation is ever in
+    flight), so every consumer wait runs out after the shortened 1 ms limit;
+    the call must report MLA_ERR_DEVICE_TIMEOUT through the device error word,
+    and an ordinary decode afterwards in the same context must still match the
+    oracle."""
+    L = _lib()
+    w, lengths = small_v3("wait_expiry", 1, 1, [100])
+    data = build(w, lengths=lengths)
+    dd = to_device(data)
+    L.device_error()  # clear
+    L.decode(w.dims, w.softmax_scale, dd["q_nope"], dd["q_pe"], dd["pool"], dd["table"], dd["lengths"], 100,
+             dd["w_uk"], dd["w_uv"], kernel=KERNELS["pair"], debug_wait_limit_us=1000, debug_starve=True)
+    assert L.device_error() == -6
+    assert L.device_error() == 0  # read and cleared
+    got = run_decode(w, dd, kernel=KERNELS["pair"])
+    check(got, oracle_out(w, data))
+
+
 # ---------------------------------------------------------------- full size
 def _sample(w, k):
     g = torch.Generator().manual_seed(w.seed + 77)

@@ -49,14 +49,32 @@ def test_no_alloc_matches_decode_on_two_calls_in_a_row():
 
 
 def test_no_alloc_refuses_problems_beyond_its_buffer():
+    """Batch 128 with one-token contexts needs more scratch than the buffer
+    holds (the absorbed queries and the split partials grow with the batch):
+    the call returns MLA_ERR_SCRATCH_LIMIT and leaves the output untouched.
+    Every argument is a real device tensor of the stated shape."""
     from mla_latent_kv_29_b200 import lib as L
 
     lib = L.load()
     w = I.WORKLOADS["v3_b64_l1k_8k"]
-    cd = L.c_dims(w.dims, w.softmax_scale)
+    d = w.dims
+    cd = L.c_dims(d, w.softmax_scale)
+    B = 128
     assert lib.mla_decode_workspace_size(ctypes.byref(cd), 64, 1, 8192, None) <= L.NO_ALLOC_SCRATCH_BYTES
-    fake = ctypes.c_void_p(1 << 20)  # never touched: the size check comes first
-    rc = lib.mla_decode_no_alloc(ctypes.byref(cd), fake, fake, 4096, 1, fake, 100, fake, 128, fake, 8192, fake,
-                                 fake, fake, None, None)
-    assert rc == -8
-    assert "scratch" in L.error_string(rc)
+    assert lib.mla_decode_workspace_size(ctypes.byref(cd), B, 1, 1, None) > L.NO_ALLOC_SCRATCH_BYTES
+    dev = "cuda"
+    q_nope = torch.zeros(B, 1, d.num_heads, d.qk_nope_dim, dtype=torch.bfloat16, device=dev)
+    q_pe = torch.zeros(B, 1, d.num_heads, d.rope_dim, dtype=torch.bfloat16, device=dev)
+    pool = torch.zeros(B, d.block_size, d.row_width, dtype=torch.bfloat16, device=dev)
+    table = torch.arange(B, dtype=torch.int32, device=dev).view(B, 1)
+    lengths = torch.ones(B, dtype=torch.int32, device=dev)
+    w_uk = torch.zeros(d.num_heads, d.qk_nope_dim, d.kv_lora_rank, dtype=torch.bfloat16, device=dev)
+    w_uv = torch.zeros(d.num_heads, d.v_head_dim, d.kv_lora_rank, dtype=torch.bfloat16, device=dev)
+    out = torch.full((B, 1, d.num_heads, d.v_head_dim), 7.0, dtype=torch.bfloat16, device=dev)
+    with pytest.raises(L.MLAError) as e:
+        L.decode_no_alloc(d, w.softmax_scale, q_nope, q_pe, pool, table, lengths, 1, w_uk, w_uv, out=out)
+    assert e.value.status == -8
+    assert "scratch" in L.error_string(e.value.status)
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    assert bool(torch.all(out == 7.0))  # nothing was enqueued
