@@ -93,12 +93,24 @@ def load_peaks():
         return dict(FALLBACK_PEAKS)
 
 
+STEP_TEXT = "append of the batch's new tokens + absorbed decode"
+
+
 def workload_config(w, cached_tokens):
-    """The workload's identity, the same in both arms' lines."""
+    """The workload's identity: the same object in both arms' lines (how each
+    arm times it goes in its own `timing` entry)."""
     return {"workload": w.name, "batch_per_gpu": w.batch, "q_len": w.q_len,
             "context": f"U[{w.length_range[0]},{w.length_range[1]}]", "cached_tokens_per_gpu": cached_tokens,
             "heads": w.dims.num_heads, "latent": w.dims.kv_lora_rank, "rope": w.dims.rope_dim,
-            "page": w.dims.block_size, "paged": "shuffled" if w.paged else "contiguous"}
+            "page": w.dims.block_size, "paged": "shuffled" if w.paged else "contiguous", "step": STEP_TEXT}
+
+
+def spread(values_ms):
+    """median / p10 / p90 (µs) of per-step times given in ms."""
+    v = sorted(values_ms)
+    q = lambda f: v[min(len(v) - 1, max(0, int(round(f * (len(v) - 1)))))]
+    return {"reps": len(v), "median_us": round(statistics.median(v) * 1e3, 2), "p10_us": round(q(0.1) * 1e3, 2),
+            "p90_us": round(q(0.9) * 1e3, 2), "mean_us": round(statistics.mean(v) * 1e3, 2)}
 
 
 def workload_totals(w, lengths):
@@ -143,15 +155,20 @@ def q_proj_line(w, ms, peaks):
 
 
 def roofline(bytes_, flops, seconds, peaks):
+    """The bound whose time is larger, against the given peaks; `frac_nominal`
+    is the same achieved figure against the nominal B200 peaks (8 TB/s HBM,
+    2.25 PFLOP/s dense bf16), the roofline the target is stated on."""
     gbs = bytes_ / seconds / 1e9
     tfs = flops / seconds / 1e12
     t_hbm = bytes_ / (peaks["hbm_gbs"] * 1e9)
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)
     if t_hbm >= t_tc:
         return dict(bound="hbm", achieved=round(gbs, 1), peak=peaks["hbm_gbs"], unit="GB/s",
-                    frac=round(gbs / peaks["hbm_gbs"], 4)), gbs, tfs
+                    frac=round(gbs / peaks["hbm_gbs"], 4),
+                    frac_nominal=round(gbs / NOMINAL["hbm_gbs"], 4), peak_nominal=NOMINAL["hbm_gbs"]), gbs, tfs
     return dict(bound="tensor", achieved=round(tfs, 2), peak=peaks["bf16_tflops"], unit="TFLOP/s",
-                frac=round(tfs / peaks["bf16_tflops"], 4)), gbs, tfs
+                frac=round(tfs / peaks["bf16_tflops"], 4),
+                frac_nominal=round(tfs / NOMINAL["bf16_tflops"], 4), peak_nominal=NOMINAL["bf16_tflops"]), gbs, tfs
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
@@ -163,10 +180,9 @@ KERNEL_SOURCES = ("decode_pair.cuh", "plan.cuh", "sm100.cuh", "common.cuh")
 TRAFFIC = {
     # profiles/pair_decode_kernel_v3_b64_l1k_8k.md (ncu launch list of one step, the attention launch:
     # dram__bytes_read.sum + dram__bytes_write.sum)
-    "v3_b64_l1k_8k": {"bytes": 356330496 + 6199552,
-                      "sources_sha256": "4aa3b05c0112b687b2e42b853cb84ab7862955e617074b06f879e28b79ec3953"},
+    "v3_b64_l1k_8k": {"bytes": 362545664 + 6273792,
+                      "sources_sha256": "22d86e39818b42247981432c84e3a295238f61a271b743e5641bb3de9301dc56"},
 }
-
 
 def kernel_sources_sha256() -> str:
     import hashlib
@@ -553,10 +569,12 @@ def run_ours(args, w):
         "metric": METRIC, "value": round(t_step * 1e3, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(w, tot["T"]), l2="flushed (256 MB write) before each step",
-                       step="append of the batch's new tokens + absorbed decode" +
-                            (" (append on a side stream; the attention waits for it)" if args.overlap else ""),
-                       launch="CUDA graph replay" if args.graph else "direct launches"),
+        "config": workload_config(w, tot["T"]),
+        "timing": {"l2": "flushed (256 MB write) before each step",
+                   "append": "on a side stream; the attention waits for it" if args.overlap else "in stream order",
+                   "launch": "CUDA graph replay" if args.graph else "direct launches",
+                   "value": "mean of the K device-timed steps (CUDA events on the launch stream), max over ranks",
+                   "step_spread": spread(step_ms), "attn_spread": spread(attn_ms)},
         "roofline": roof,
         "attn_us": round(t_attn * 1e3, 2),
         "attn_timing": "CUDA events around the attention launch, in a second pass of K steps "
@@ -605,7 +623,10 @@ def profile_step(args, w):
 
 
 def run_reference(args, w):
-    """The oracle timed on the host cores (the reference arm)."""
+    """The oracle timed on the host cores (the reference arm). Each step times
+    the fp64 oracle on one sequence and a quarter of the heads (plus that
+    sequence's append rows) and scales by tokens and heads to the whole
+    workload; the line states the seconds actually timed and the factor."""
     from mla_latent_kv_29_b200 import inputs as I
 
     rank, world, _ = dist_env()
@@ -615,20 +636,28 @@ def run_reference(args, w):
     H = w.dims.num_heads
     heads = list(range(0, H, 4))
     T = sum(lengths)
-    per_step = []
+    per_step, timed_s, factors = [], 0.0, []
     for k in range(args.warmup + args.steps):
         b = k % w.batch
         s, tok = oracle_sample_seconds(w, lengths, [b], heads)
         if k >= args.warmup:
-            per_step.append(s * (T / tok) * (H / len(heads)))
+            f = (T / tok) * (H / len(heads))
+            per_step.append(s * f)
+            timed_s += s
+            factors.append(f)
     v = statistics.mean(per_step) * 1e6
-    sample = (f"each step: fp64 explicit oracle on 1 of {w.batch} sequences and {len(heads)} of {H} heads "
-              f"plus its append rows, scaled by tokens and heads to the full step")
+    sample = (f"each of the {args.steps} timed steps: the fp64 explicit oracle on 1 of {w.batch} sequences and "
+              f"{len(heads)} of {H} heads plus its append rows ({timed_s:.2f} s of oracle time in all), scaled by "
+              f"tokens and heads to the whole step (factor {statistics.mean(factors):.0f} on average)")
     return {"impl": "reference", "metric": METRIC, "value": round(v, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v / 1e3, 3),
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": dict(workload_config(w, T), step="append of the batch's new tokens + absorbed decode"),
+            "config": workload_config(w, T),
+            "timing": {"value": "mean over the timed steps of (oracle seconds on the sample x scale factor)",
+                       "timed_seconds": round(timed_s, 3), "samples": args.steps,
+                       "scale_factor_mean": round(statistics.mean(factors), 1),
+                       "step_spread": spread([x * 1e3 for x in per_step])},
             "cpu_baseline": {"value": round(v, 1), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -637,7 +666,7 @@ def run_reference(args, w):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="v3_b64_l1k_8k")

@@ -24,27 +24,23 @@
 // HBM reads stay ~1x because the second read of a page hits L2 (each CTA
 // also asks L2 for its page of the next tile ahead of the key loads).
 //
-// Warp roles per CTA (256 threads): one thread of warp 0 streams the queries
+// Warp roles per CTA (320 threads): one thread of warp 0 streams the queries
 // and the key stages (column blocks 0-2, 3-4, 5-6 and 7-8 of the CTA's page,
 // one TMA operation each) into a one-tile key ring; warp 2 streams the value
 // stages (32 tokens x 256 columns, 16 KB) into a four-stage value ring that
 // holds a whole tile (one thread issues, the warp zeroes the tail rows of
 // partial stages); warp 1 allocates tensor memory (both CTAs). In the leader,
-// two threads (lanes 0 of warps 1 and 3) issue the MMAs, each the same
-// program over the pair's tiles n = 0, 1, ...: its half of the score MMAs of
-// tile n (column blocks 0-4 or 5-8, into two half-accumulators that the
-// softmax adds), then its half of the value MMAs of tile n - 1 (latent
-// columns 0-255 or 256-511 of the CTA pair's O). The tensor pipe therefore
-// runs S(n), PV(n-1), S(n+1), PV(n), ...: the score of the next tile covers
-// the softmax of the current one, and no issuer runs further ahead, so the
-// MMA queue stays short and the key and value stages are released promptly
-// (two threads are needed: one cannot issue the M 128 x N 128 score
-// instructions as fast as the tensor cores run them).
+// four threads issue the MMAs, each its own independent stream: lanes 0 of
+// warps 1 and 3 the score MMAs of every tile (column blocks 0-4 and 5-8,
+// into two half-accumulators that the softmax adds), lanes 0 of warps 8 and 9
+// the value MMAs (latent columns 0-255 and 256-511 of the pair's O). One
+// thread cannot issue the M 128 x N 128 score instructions as fast as the
+// tensor cores run them, and a thread stalls at each wait for its operands,
+// so independent streams keep the tensor pipe fed while any one of them waits.
 // Warps 4-7 (thread t = TMEM lane t) run the softmax, rescale O when the
-// running max grows by more than 2^8, write P to shared memory (one buffer:
-// the value MMAs of tile n - 1 have finished by the time the softmax of tile
-// n has its weights) and, at the end of a segment, normalise O and write the
-// partial.
+// running max grows by more than 2^8, write P to shared memory (one buffer,
+// rewritten once the value MMAs of the previous tile are done) and, at the
+// end of a segment, normalise O and write the partial.
 // Every mbarrier wait is bounded (see ptx::mbar_wait; the limit is a kernel
 // parameter so that a test can shorten it): on expiry the kernel records
 // MLA_ERR_DEVICE_TIMEOUT and every role drains to the common exit. With the
@@ -75,7 +71,7 @@ constexpr int kKTile = kQBoxes * kBox;  // 72 KB
 constexpr int kVStage = 2 * kBox;    // value stage: 32 tokens x 256 latent columns (4 x 4 KB)
 constexpr int kVPerTile = 4;         // 4 value stages per tile
 constexpr int kVStages = 4;          // value ring: four stages (a whole tile)
-constexpr int kThreads = 256;  // 8 warps; the softmax warps 4-7 own TMEM lanes 0-127
+constexpr int kThreads = 320;  // 10 warps; the softmax warps 4-7 own TMEM lanes 0-127
 constexpr int kTmemCols = 512;
 constexpr int kTmS = 0;          // two S buffers (tile parity), each lo and hi halves of 64 columns
 constexpr int kTmO = 256;        // O: 256 columns (after the two S buffers of 128)
@@ -282,10 +278,10 @@ __device__ void value_producer(const Params& P, const CUtensorMap* tm_v, const C
 }
 
 // ------------------------------------------------------------------- MMA
-// Two issuing threads in the leader CTA (half 0: lane 0 of warp 1, half 1:
-// lane 0 of warp 3). A single thread issues at most about one tcgen05.mma every
-// ~47 cycles, while an M 128 x N 128 x K 16 pair instruction takes the tensor
-// cores 32 cycles; two threads with independent accumulators keep up.
+// Four issuing threads in the leader CTA: two for the score MMAs, two for the
+// value MMAs. A single thread issues at most about one tcgen05.mma every ~47
+// cycles, while an M 128 x N 128 x K 16 pair instruction takes the tensor
+// cores 32 cycles; streams with their own accumulators keep up together.
 struct Descs {
     uint64_t dq, dk, dp, dv;
     __device__ explicit Descs(const Ctx& c)
@@ -296,43 +292,32 @@ struct Descs {
           dv(ptx::smem_desc_sw128(c.sbase + kOffV, kBox / 2, 1024)) {}
 };
 
-// Both threads run the same program over the pair's tiles n (counted across
-// segments): the score MMAs of tile n, then the value MMAs of tile n - 1.
-//   score, half h: S_h = Q[:, blocks] K[:, blocks]^T over column blocks 0-4
-//     (h = 0: key stages 0-1) or 5-8 (h = 1: stages 2-3) into half-accumulator
-//     h of S buffer (n & 1); each key stage is consumed by one thread, once
-//     per tile (phase = tile parity). QEMPTY (count 2) is committed once per
-//     segment by each thread, SFULL (count 2) once per tile.
-//   value, half h: O[:, 256h .. 256h + 255] += P V over the tile's visible
-//     32-token value stages (stage q: tokens 32q..32q+31); both threads read
-//     every value stage and commit its VEMPTY (count 2), and PVDONE (count 2)
-//     once per tile. The first value MMA of a segment overwrites O, after the
-//     softmax has read out the previous segment (OEMPTY).
-__device__ void mma_issuer(const Params& P, const Ctx& c, uint32_t half) {
+// Score MMAs, half h (lane 0 of warp 1: h = 0; lane 0 of warp 3: h = 1):
+// S_h = Q[:, blocks] K[:, blocks]^T over column blocks 0-4 (key stages 0-1) or
+// 5-8 (stages 2-3) into half-accumulator h of S buffer (tile & 1), up to two
+// tiles ahead of the softmax (the S buffers). Each key stage is consumed by
+// one thread, once per tile (phase = tile parity); both threads commit QEMPTY
+// (count 2) once per segment and SFULL (count 2) once per tile.
+__device__ void mma_s_issuer(const Params& P, const Ctx& c, uint32_t half) {
     constexpr uint32_t kIdS = ptx::idesc_bf16(128, 128, false, false);
-    constexpr uint32_t kIdPV = ptx::idesc_bf16(128, 256, false, true);
     const Descs D(c);
+    uint32_t tile_cnt = 0;
+    int seg_i = 0;
     const int ks0 = 2 * static_cast<int>(half);
     const int k_first = kstage_first_block(ks0);
-    SegmentIter its(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
-    SegmentIter itv = its;
-    Segment ss, sv;
-    bool have_s = its.next(ss), have_v = itv.next(sv);
-    int s_seg = 0, s_j = 0, v_seg = 0, v_j = 0;
-    uint32_t s_cnt = 0, v_cnt = 0, vst = 0, vph = 0;
-    while (have_s || have_v) {
-        if (have_s) {
-            // ---- score MMAs of tile s_cnt
-            if (s_j == 0) {
-                if (!ptx::mbar_wait(c.bar(B_QFULL), s_seg & 1, c.abort, c.wait_ns)) return;
-                ptx::tc_fence_after();
-            }
-            const uint32_t sb = s_cnt & 1;
+    SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    Segment seg;
+    while (it.next(seg)) {
+        if (!ptx::mbar_wait(c.bar(B_QFULL), seg_i & 1, c.abort, c.wait_ns)) return;
+        ptx::tc_fence_after();
+        const int n_tiles = tiles_of(seg);
+        for (int j = 0; j < n_tiles; ++j, ++tile_cnt) {
+            const uint32_t sb = tile_cnt & 1;
             const uint32_t d_s = c.tmem + kTmS + 128 * sb + 64 * half;
-            if (!ptx::mbar_wait(c.bar(B_SEMPTY0 + sb), ((s_cnt >> 1) & 1) ^ 1, c.abort, c.wait_ns)) return;
+            if (!ptx::mbar_wait(c.bar(B_SEMPTY0 + sb), ((tile_cnt >> 1) & 1) ^ 1, c.abort, c.wait_ns)) return;
 #pragma unroll 1
             for (int ks = ks0; ks < ks0 + 2; ++ks) {
-                if (!ptx::mbar_wait(c.bar(B_KFULL0 + ks), s_cnt & 1, c.abort, c.wait_ns)) return;
+                if (!ptx::mbar_wait(c.bar(B_KFULL0 + ks), tile_cnt & 1, c.abort, c.wait_ns)) return;
                 ptx::tc_fence_after();
                 for (int k = kstage_first_block(ks); k < kstage_first_block(ks) + kstage_blocks(ks); ++k) {
                     const uint64_t a0 = D.dq + static_cast<uint64_t>((k * kBox) >> 4);
@@ -344,25 +329,36 @@ __device__ void mma_issuer(const Params& P, const Ctx& c, uint32_t half) {
                 ptx::mma_commit_pair(c.bar(B_KEMPTY0 + ks), 0x3);
             }
             ptx::mma_commit_pair(c.bar(B_SFULL0 + sb), 0x3);
-            ++s_cnt;
-            if (++s_j == tiles_of(ss)) {
-                ptx::mma_commit_pair(c.bar(B_QEMPTY), 0x3);
-                ++s_seg;
-                s_j = 0;
-                have_s = its.next(ss);
-            }
         }
-        if (have_v && (v_cnt + 1 < s_cnt || !have_s)) {
-            // ---- value MMAs of tile v_cnt (its weights are in the P buffer)
-            const bool first = (v_j == 0);
-            if (!ptx::mbar_wait(c.bar(B_PFULL0 + (v_cnt & 1)), (v_cnt >> 1) & 1, c.abort, c.wait_ns)) return;
-            if (first && !ptx::mbar_wait(c.bar(B_OEMPTY), (v_seg & 1) ^ 1, c.abort, c.wait_ns)) return;
-            const int32_t tv = sv.tok_begin + v_j * kTile;
+        ptx::mma_commit_pair(c.bar(B_QEMPTY), 0x3);
+        ++seg_i;
+    }
+}
+
+// Value MMAs, half h (lane 0 of warp 8 + h): O[:, 256h .. 256h + 255] += P V
+// over the tile's visible 32-token value stages (stage q: tokens 32q..32q+31,
+// stages without a visible token skipped here and by the producer alike).
+// Both threads read every value stage and commit its VEMPTY (count 2), and
+// PVDONE (count 2) once per tile. The first value MMA of a segment overwrites
+// O, after the softmax has read out the previous segment (OEMPTY).
+__device__ void mma_pv_issuer(const Params& P, const Ctx& c, uint32_t half) {
+    constexpr uint32_t kIdPV = ptx::idesc_bf16(128, 256, false, true);
+    const Descs D(c);
+    uint32_t vst = 0, vph = 0, pv_cnt = 0;
+    int seg_i = 0;
+    SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    Segment seg;
+    while (it.next(seg)) {
+        const int n_tiles = tiles_of(seg);
+        for (int j = 0; j < n_tiles; ++j) {
+            const bool first = (j == 0);
+            if (!ptx::mbar_wait(c.bar(B_PFULL0 + (pv_cnt & 1)), (pv_cnt >> 1) & 1, c.abort, c.wait_ns)) return;
+            if (first && !ptx::mbar_wait(c.bar(B_OEMPTY), (seg_i & 1) ^ 1, c.abort, c.wait_ns)) return;
+            const int32_t tv = seg.tok_begin + j * kTile;
             for (int q = 0; q < kVPerTile; ++q) {
-                if (sv.tok_end - (tv + 32 * q) <= 0) break;  // no visible token: skipped by the producer too
+                if (seg.tok_end - (tv + 32 * q) <= 0) break;
                 if (!ptx::mbar_wait(c.bar(B_VFULL0 + vst), vph, c.abort, c.wait_ns)) return;
                 ptx::tc_fence_after();
-                // A: P tokens 32q + 16kk .. +15 (box q/2, byte 64 (q&1) + 32 kk of each 128-byte row)
                 const uint64_t a0 = D.dp + static_cast<uint64_t>(((q >> 1) * kBox + 64 * (q & 1)) >> 4);
                 const uint64_t b0 = D.dv + static_cast<uint64_t>((vst * kVStage + half * kBox) >> 4);
 #pragma unroll
@@ -373,14 +369,10 @@ __device__ void mma_issuer(const Params& P, const Ctx& c, uint32_t half) {
                 ptx::mma_commit_pair(c.bar(B_VEMPTY0 + vst), 0x3);
                 ring_next<kVStages>(vst, vph);
             }
-            ptx::mma_commit_pair(c.bar(B_PVDONE0 + (v_cnt & 1)), 0x3);
-            ++v_cnt;
-            if (++v_j == tiles_of(sv)) {
-                ++v_seg;
-                v_j = 0;
-                have_v = itv.next(sv);
-            }
+            ptx::mma_commit_pair(c.bar(B_PVDONE0 + (pv_cnt & 1)), 0x3);
+            ++pv_cnt;
         }
+        ++seg_i;
     }
 }
 
@@ -647,7 +639,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else if (warp == 2) {
         if (!P.starve) value_producer(P, &tm_v, c);
     } else if (warp == 1 || warp == 3) {
-        if (c.rank == 0 && ptx::lane_id() == 0) mma_issuer(P, c, static_cast<uint32_t>(warp >> 1));
+        if (c.rank == 0 && ptx::lane_id() == 0) mma_s_issuer(P, c, static_cast<uint32_t>(warp >> 1));
+    } else if (warp >= 8) {
+        if (c.rank == 0 && ptx::lane_id() == 0) mma_pv_issuer(P, c, static_cast<uint32_t>(warp - 8));
     } else if (warp >= 4) {
         softmax(P, c);
     }
