@@ -411,6 +411,107 @@ def count_library_launches(step, device):
     return len(names), sorted(set(n.split("(")[0].replace("void ", "") for n in names))
 
 
+def timed_calls(fn, flush, K, warmup, device):
+    """Device times (ms) of K calls of fn, each after an L2 flush, CUDA events
+    on the current stream."""
+    import torch
+
+    for _ in range(warmup):
+        fn()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    torch.cuda.synchronize(device)
+    for k in range(K):
+        flush.zero_()
+        ev[k][0].record()
+        fn()
+        ev[k][1].record()
+    torch.cuda.synchronize(device)
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def o_proj_lines(w, st, flush, K, warmup, device, peaks):
+    """The output projection of the step's G tokens, two ways (mla_o_proj):
+    unfused, out [G, H d_v] times W_O [H d_v, 7168] after the per-head W_UV;
+    absorbed, o_lat [G, H d_c] times W_UV^T W_O [H d_c, 7168] (the decode with
+    output_latent). Weights are random of those shapes (the product's values
+    do not change the traffic); bytes = weights + activations in + out."""
+    import torch
+
+    from mla_latent_kv_29_b200 import lib
+
+    d = st["d"]
+    G = w.batch * w.q_len
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed + 77)
+    res = {}
+    for name, k in (("unfused", d.num_heads * d.v_head_dim), ("absorbed", d.num_heads * d.kv_lora_rank)):
+        wt = (torch.randn(k, HIDDEN, generator=gen, device=device) * k ** -0.5).to(torch.bfloat16)
+        x = torch.randn(G, k, generator=gen, device=device).to(torch.bfloat16)
+        y = torch.empty(G, HIDDEN, dtype=torch.bfloat16, device=device)
+        ws = torch.empty(lib.o_proj_workspace_size(G, k, HIDDEN), dtype=torch.uint8, device=device)
+        ms = timed_calls(lambda: lib.o_proj(x, wt, y=y, workspace=ws), flush, K, warmup, device)
+        t = statistics.median(ms)
+        bytes_ = 2 * (k * HIDDEN + G * k + G * HIDDEN)
+        gbs = bytes_ / (t * 1e-3) / 1e9
+        res[name] = {"us": round(t * 1e3, 2), "k": k, "n": HIDDEN, "tokens": G, "bytes": bytes_,
+                     "achieved_gbs": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4)}
+        del wt, x, y, ws
+    res["absorbed_over_unfused_time"] = round(res["absorbed"]["us"] / res["unfused"]["us"], 3)
+    res["timing"] = "median of K calls, CUDA events around each, L2 flushed before each"
+    return res
+
+
+def workload_summary(name, args, device, peaks, flush, K=10):
+    """Step and attention times of another workload (same step as the headline:
+    append of the new tokens + decode, CUDA graph replay, L2 flushed before
+    each step), for the summary of every configuration."""
+    import dataclasses
+
+    import torch
+
+    from mla_latent_kv_29_b200 import inputs as I
+
+    rank, _, _ = dist_env()
+    w = I.WORKLOADS[name]
+    w = dataclasses.replace(w, seed=rank_seed(w.seed, rank))
+    st = setup_gpu(w, device, rank)
+    step = make_step(w, st, args.kernel, overlap=args.overlap)
+    ea = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    ea[0].record()
+    ea[1].record()
+    graphs = []
+
+    def capture(events):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(events=events)
+        g.replay()
+        torch.cuda.synchronize(device)
+        graphs.append(g)
+        return g.replay
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(device)
+    run, run_attn = capture(None), capture(ea)
+    step_ms = timed_calls(run, flush, K, 2, device)
+    attn_ms = []
+    for _ in range(K):
+        flush.zero_()
+        run_attn()
+        torch.cuda.synchronize(device)
+        attn_ms.append(ea[0].elapsed_time(ea[1]))
+    tot = workload_totals(w, st["lengths"].tolist())
+    t_attn = statistics.median(attn_ms) / 1e3
+    roof, gbs, tfs = roofline(tot["attn_bytes"], tot["attn_flops"], t_attn, peaks)
+    del graphs, st
+    torch.cuda.synchronize(device)
+    return {"step_us_median": round(statistics.median(step_ms) * 1e3, 2),
+            "attn_us_median": round(t_attn * 1e6, 2), "attn_bound": roof["bound"], "attn_frac": roof["frac"],
+            "attn_frac_nominal": roof["frac_nominal"], "attn_gbs": round(gbs, 1), "attn_tflops": round(tfs, 2),
+            "cached_tokens": tot["T"], "new_tokens": tot["G"], "steps": K}
+
+
 def run_ours(args, w):
     import torch
 
@@ -589,9 +690,17 @@ def run_ours(args, w):
                 "d2h_bytes_per_step": h_out.numel() * 2},
         "gpu_launches": launches_per_step * K,
         "q_proj": q_proj_line(w, t_q, peaks),
+        "o_proj": o_proj_lines(w, st, flush, min(K, 20), args.warmup, device, peaks),
         "kernels": kernel_names,
         "clocks": clocks,
     }
+    if args.all_workloads:
+        from mla_latent_kv_29_b200 import inputs as I
+
+        line["workloads"] = {n: workload_summary(n, args, device, peaks, flush)
+                             for n in I.WORKLOADS if n not in (w.name, "tiny_b1_l128")}
+        line["workloads"]["_note"] = ("the other configurations, each timed the same way as the headline "
+                                      "(median of 10 steps); tiny_b1_l128 is a correctness case only")
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, st["lengths"].tolist(), args.cpu_seconds)
     return line
@@ -620,6 +729,46 @@ def profile_step(args, w):
     torch.cuda.synchronize(device)
     torch.cuda.profiler.stop()
     assert lib.device_error() == 0, "device fault in the profiled step"
+
+
+def profile_ops(args, w):
+    """One step, one query projection and the two output projections (unfused
+    and absorbed) of the workload's new tokens between cudaProfilerStart and
+    cudaProfilerStop (for `ncu --profile-from-start off`), each after an L2
+    flush, warm-ups outside. Prints nothing."""
+    import torch
+
+    from mla_latent_kv_29_b200 import inputs as I
+    from mla_latent_kv_29_b200 import lib
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    lib.load()
+    st = setup_gpu(w, device, 0)
+    step = make_step(w, st, args.kernel, overlap=args.overlap)
+    d = st["d"]
+    G = w.batch * w.q_len
+    qin = I.q_proj_inputs(d, G, HIDDEN, Q_RANK, seed=w.seed)
+    qd = {k: (v.to(device) if v is not None else None) for k, v in qin.items()}
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed + 77)
+    ops = [step, lambda: lib.q_proj(d, qd["x"], qd["w_qa"], qd["w_qb"], qd["positions"], q_gamma=qd["gamma"])]
+    for k in (d.num_heads * d.v_head_dim, d.num_heads * d.kv_lora_rank):
+        wt = (torch.randn(k, HIDDEN, generator=gen, device=device) * k ** -0.5).to(torch.bfloat16)
+        x = torch.randn(G, k, generator=gen, device=device).to(torch.bfloat16)
+        ops.append(lambda x=x, wt=wt: lib.o_proj(x, wt))
+    for f in ops:
+        for _ in range(args.warmup):
+            f()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    torch.cuda.synchronize(device)
+    torch.cuda.profiler.start()
+    for f in ops:
+        flush.zero_()
+        f()
+    torch.cuda.synchronize(device)
+    torch.cuda.profiler.stop()
+    assert lib.device_error() == 0, "device fault in the profiled operations"
 
 
 def run_reference(args, w):
@@ -674,12 +823,17 @@ def main(argv=None):
     ap.add_argument("--soak", type=float, default=1.5, help="seconds of untimed steps while clocks are sampled")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--all-workloads", action=argparse.BooleanOptionalAction, default=True,
+                    help="add a summary of every other configuration to the line")
     ap.add_argument("--overlap", action=argparse.BooleanOptionalAction, default=True,
                     help="run the append on a side stream beside the decode's query-side launches")
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="replay each step from a captured CUDA graph")
     ap.add_argument("--profile-step", action="store_true",
                     help="run one step between profiler start/stop (for ncu --profile-from-start off) and exit")
+    ap.add_argument("--profile-ops", action="store_true",
+                    help="run one step, one query projection and the two output projections between profiler "
+                         "start/stop (for ncu --profile-from-start off) and exit")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -692,6 +846,9 @@ def main(argv=None):
     w = dataclasses.replace(w, seed=rank_seed(w.seed, rank))
     if args.profile_step:
         profile_step(args, w)
+        return
+    if args.profile_ops:
+        profile_ops(args, w)
         return
     line = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
     if line is not None:

@@ -107,6 +107,14 @@ typedef struct mla_decode_opts {
      * mla_get_device_error() and its output is undefined. */
     uint32_t debug_wait_limit_us;
     int32_t debug_starve;
+    /* 0: out = W_UV o_lat per head (bf16 [batch, q_len, H, v_head_dim]).
+     * 1: out receives o_lat itself (bf16 [batch, q_len, H, kv_lora_rank]) and
+     * w_uv is not read: the input of the full absorption of W_UV into the
+     * output projection ([MQA-MLA] "MLA的实现", forward_inference_absorbed,
+     * W_o_absorbed = W_UV^T W_O; [MLA-arch] 3.1), applied with mla_o_proj.
+     * Needs the tensor-core merge (kv_lora_rank 256 or 512, the alignment
+     * below), else MLA_ERR_UNSUPPORTED_DIMS before anything is enqueued. */
+    int32_t output_latent;
 } mla_decode_opts_t;
 
 /* Paged latent cache ("pool"), [MLA-arch] 3.2 kept as one row per token:
@@ -167,8 +175,8 @@ MLA_API size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t n_token
  *   q_pe     bf16 [n_tokens, H, rope_dim] (output)
  *   workspace >= mla_q_proj_workspace_size(dims, n_tokens, hidden, q_rank)
  *            bytes, 256-byte aligned, contents need not be initialised.
- * hidden, q_rank and H * (qk_nope_dim + rope_dim) must be multiples of 64 and
- * rope_dim even and <= 128 (else MLA_ERR_UNSUPPORTED_DIMS). Accumulation is
+ * hidden, q_rank and H * (qk_nope_dim + rope_dim) must be multiples of 64,
+ * q_rank <= 2048 and rope_dim even and <= 128 (else MLA_ERR_UNSUPPORTED_DIMS). Accumulation is
  * fp32; c_q is rounded to bf16 before the second product. */
 MLA_API int mla_q_proj(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t hidden,
                        const void* w_qa, int32_t q_rank, const void* q_gamma, float rms_eps,
@@ -267,6 +275,31 @@ MLA_API int mla_decode_no_alloc(const mla_dims_t* dims, const void* q_nope, cons
                                 const int32_t* context_lens, int32_t max_context_len,
                                 const void* w_uk, const void* w_uv, void* out,
                                 const mla_decode_opts_t* opts, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* Output projection: y = x W for a few token rows, the step after the
+ * attention ([MQA-MLA] "MLA的实现": the W_O of forward_training and the
+ * W_o_absorbed of forward_inference_absorbed; [MLA-arch] 3.1, W_V absorbed
+ * into the O projection). Two uses:
+ *   x = out viewed as [n_tokens, H * v_head_dim], w = W_O [H * v_head_dim,
+ *       hidden] (row h * v_head_dim + d holds head h's value index d): the
+ *       output projection after the per-head up-projection;
+ *   x = o_lat viewed as [n_tokens, H * kv_lora_rank] (mla_decode with
+ *       output_latent = 1), w = W_UV^T W_O stacked per head [H * kv_lora_rank,
+ *       hidden]: the full absorption, which reads kv_lora_rank / v_head_dim
+ *       times the weight bytes.
+ *   y[t, n] = bf16(sum_k x[t, k] w[k, n]), fp32 accumulation.
+ * Arguments:
+ *   x  bf16 [n_tokens, k], 16-byte aligned;  w  bf16 [k, n], 16-byte aligned
+ *   y  bf16 [n_tokens, n], 8-byte aligned
+ *   workspace >= mla_o_proj_workspace_size(n_tokens, k, n) bytes, 256-byte
+ *            aligned, contents need not be initialised.
+ * k and n must be multiples of 64 (else MLA_ERR_UNSUPPORTED_DIMS). */
+MLA_API int mla_o_proj(const void* x, int32_t n_tokens, int32_t k, const void* w, int32_t n, void* y,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace mla_o_proj needs; 0 if the sizes are invalid. */
+MLA_API size_t mla_o_proj_workspace_size(int32_t n_tokens, int32_t k, int32_t n);
 
 /* ------------------------------------------------------------------ */
 /* Log-sum-exp combine of split-KV partials (the merge the split decode

@@ -7,9 +7,10 @@
 //               log-sum-exp merge of the split-KV partials, merged on chip
 //               (merge_uv_kernel), or merged into memory (merge_kernel) and
 //               then multiplied (uv_kernel)
-//   row GEMM:   y = x W (fp32) for x [T, K] and W [K, N], the K range split
-//               over a cluster (append_kernel): the cache append's x W_kva and
-//               the query projection's x W_qa and c_q W_qb.
+//   row GEMM:   y = x W (fp32 partials over K ranges) for x [T, K] and W
+//               [K, N] (row_gemm_kernel): the cache append's x W_kva, the
+//               query projection's x W_qa and c_q W_qb, and the output
+//               projection (sum_partials_kernel adds its partials into bf16).
 //
 // Roles of the 128-thread kernels: lane 0 of warp 0 issues the TMA loads,
 // lane 0 of warp 1 the MMAs (M = 128, cta_group::1), warp 2 owns the TMEM
@@ -589,154 +590,163 @@ __global__ void __launch_bounds__(kThreads) absorb_kernel(const __grid_constant_
     pdl_wait();
 }
 
-// --------------------------------------------------------------- append
-// kv[t, n0 .. n0 + 63] = x[t, :] W_kva[:, n0 .. n0 + 63] (fp32) for t in
-// [m0, m0 + 128): the joint down-projection of the cache append
-// (kv_a_proj_with_mqa, "MLA架构：低秩注意力机制优化LLM显存与计算效率" 2.2).
-// The hidden dimension is split over the S * Z CTAs along grid z, in Z
-// clusters of S (cluster (1, 1, S)); each CTA streams its K-blocks of 64
-// through a ring of (x box {64, 128 rows}, W box {64 columns, 64 rows})
-// stages into a M 128 x N 64 TMEM accumulator, the S partial tiles of a
-// cluster meet in shared memory and CTA r of the cluster sums rows
-// [r 128 / S, (r + 1) 128 / S) over the cluster (distributed shared memory)
-// and stores them into partial z / S of kv ([Z][T][N]; the epilogue adds the
-// Z partials). S = 1 stores directly.
-// tm_x: x as 2-D [T rows, hidden columns]; tm_w: W_kva as 2-D [hidden rows,
-// N columns], box {64, 64} (MN-major B). grid (N / 64, ceil(T / 128), S Z);
-// block 128; dynamic smem append_smem().
-constexpr int kApStages = 6;
-constexpr int kApStageBytes = kRows * kBoxBytes + 64 * kBoxBytes;  // 24 KB
-__host__ __device__ inline size_t append_smem() { return static_cast<size_t>(kApStages) * kApStageBytes + 256 + 1024; }
-
-__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t cluster_addr) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(cluster_addr)
-                 : "memory");
-    return v;
+// --------------------------------------------------------------- row GEMM
+// part[z][t][n0 .. n0 + 64 nb - 1] = x[t, K-range z] W[K-range z, n0 .. n0 + 64 nb - 1]
+// (fp32) for t in [m0, m0 + 128): a GEMM with few rows (new tokens) whose cost
+// is streaming the weight W once. Used for the joint down-projection of the
+// cache append (kv_a_proj_with_mqa, "MLA架构：低秩注意力机制优化LLM显存与计算效率"
+// 2.2), the query projections (2.1) and the output projection. The grid covers
+// the weight with (column tile of 64 nb, K-range of k_per_cta blocks of 64)
+// work units sized so that whole waves of CTAs stream it; the consumer (the
+// append or query epilogue, or sum_partials_kernel) sums the Z partials of a
+// column tile, requesting four at a time.
+// Each CTA streams its K-blocks through a ring of stages (x box {64, 128 rows}
+// plus nb W boxes {64 columns, 64 rows}) into an M 128 x N 64 nb TMEM
+// accumulator and stores its rows of the partial tile.
+// tm_x: x as 2-D [T rows, K columns]; tm_w: W as 2-D [K rows, N columns], box
+// {64, 64} (MN-major B). grid (N / (64 nb), ceil(T / 128), Z); block 128;
+// dynamic smem row_gemm_smem(nb).
+constexpr int kRgSmemBudget = 200 * 1024;
+__host__ __device__ inline int row_gemm_stage_bytes(int nb) { return kRows * kBoxBytes + nb * 64 * kBoxBytes; }
+__host__ __device__ inline int row_gemm_stages(int nb) { return kRgSmemBudget / row_gemm_stage_bytes(nb); }
+__host__ __device__ inline size_t row_gemm_smem(int nb) {
+    return static_cast<size_t>(row_gemm_stages(nb)) * row_gemm_stage_bytes(nb) + 256 + 1024;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) append_kernel(const __grid_constant__ CUtensorMap tm_x,
-                                                            const __grid_constant__ CUtensorMap tm_w, int32_t T,
-                                                            int32_t N, int32_t k_blocks, int32_t k_blocks_per_cta,
-                                                            int32_t S, float* __restrict__ kv) {
+__global__ void __launch_bounds__(kThreads, 1) row_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
+                                                              const __grid_constant__ CUtensorMap tm_w, int32_t T,
+                                                              int32_t N, int32_t k_blocks, int32_t k_per_cta,
+                                                              int32_t nb, float* __restrict__ part) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
-    const int off_bar = kApStages * kApStageBytes;  // full[s], empty[s], done
-    volatile int* abort = reinterpret_cast<volatile int*>(smem + off_bar + 8 * (2 * kApStages + 1));
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + 8 * (2 * kApStages + 1) + 16);
+    const int stage_bytes = row_gemm_stage_bytes(nb), n_stages = row_gemm_stages(nb);
+    const int off_bar = n_stages * stage_bytes;  // full[s], empty[s], done
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + off_bar + 8 * (2 * n_stages + 1));
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + 8 * (2 * n_stages + 1) + 16);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * 64, m0 = blockIdx.y * kRows, z = blockIdx.z;
-    kv += static_cast<int64_t>(z / S) * T * N;  // this cluster's partial
-    const int kb0 = z * k_blocks_per_cta;
-    const int nk = max(0, min(k_blocks_per_cta, k_blocks - kb0));  // this CTA's K-blocks of 64
+    const int ncols = 64 * nb;
+    const int n0 = blockIdx.x * ncols, m0 = blockIdx.y * kRows, z = blockIdx.z;
+    part += static_cast<int64_t>(z) * T * N;
+    const int kb0 = z * k_per_cta;
+    const int nk = max(0, min(k_per_cta, k_blocks - kb0));  // this CTA's K-blocks of 64
     if (threadIdx.x == 0) {
         *abort = 0;
-        for (int i = 0; i < kApStages; ++i) {
+        for (int i = 0; i < n_stages; ++i) {
             ptx::mbar_init(bar_addr(smem, off_bar, i), 1);
-            ptx::mbar_init(bar_addr(smem, off_bar, kApStages + i), 1);
+            ptx::mbar_init(bar_addr(smem, off_bar, n_stages + i), 1);
         }
-        ptx::mbar_init(bar_addr(smem, off_bar, 2 * kApStages), 1);
+        ptx::mbar_init(bar_addr(smem, off_bar, 2 * n_stages), 1);
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tm_x);
         ptx::prefetch_tmap(&tm_w);
     }
     if (warp == 2) {
-        ptx::tmem_alloc_1(ptx::smem_u32(tmem_slot), 64);
+        ptx::tmem_alloc_1(ptx::smem_u32(tmem_slot), ncols);
         ptx::tmem_relinquish_1();
     }
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    pdl_wait();
-    pdl_trigger();
 
     if (warp == 0 && lane == 0) {  // producer
-        for (int i = 0; i < nk; ++i) {
-            const int st = i % kApStages;
-            if (!ptx::mbar_wait(bar_addr(smem, off_bar, kApStages + st), ((i / kApStages) & 1) ^ 1, abort)) break;
+        // The weights are not written by earlier launches: the first stages' weight
+        // boxes are requested before the dependency wait, the activations after it.
+        const int pre = min(nk, n_stages);
+        for (int i = 0; i < pre; ++i) {
+            const uint32_t full = bar_addr(smem, off_bar, i);
+            const uint32_t dst = ptx::smem_u32(smem + i * stage_bytes);
+            ptx::mbar_arrive_expect_tx_local(full, stage_bytes);
+            for (int b = 0; b < nb; ++b)
+                ptx::tma_load_2d(dst + (kRows + 64 * b) * kBoxBytes, &tm_w, n0 + 64 * b, 64 * (kb0 + i), full);
+        }
+        pdl_wait();
+        pdl_trigger();
+        for (int i = 0; i < pre; ++i)
+            ptx::tma_load_2d(ptx::smem_u32(smem + i * stage_bytes), &tm_x, 64 * (kb0 + i), m0,
+                             bar_addr(smem, off_bar, i));
+        for (int i = pre; i < nk; ++i) {
+            const int st = i % n_stages;
+            if (!ptx::mbar_wait(bar_addr(smem, off_bar, n_stages + st), ((i / n_stages) & 1) ^ 1, abort)) break;
             const uint32_t full = bar_addr(smem, off_bar, st);
-            const uint32_t dst = ptx::smem_u32(smem + st * kApStageBytes);
-            ptx::mbar_arrive_expect_tx_local(full, kApStageBytes);
+            const uint32_t dst = ptx::smem_u32(smem + st * stage_bytes);
+            ptx::mbar_arrive_expect_tx_local(full, stage_bytes);
             ptx::tma_load_2d(dst, &tm_x, 64 * (kb0 + i), m0, full);
-            ptx::tma_load_2d(dst + kRows * kBoxBytes, &tm_w, n0, 64 * (kb0 + i), full);
+            for (int b = 0; b < nb; ++b)
+                ptx::tma_load_2d(dst + (kRows + 64 * b) * kBoxBytes, &tm_w, n0 + 64 * b, 64 * (kb0 + i), full);
         }
-    } else if (warp == 1 && lane == 0) {  // MMA issuer
-        constexpr uint32_t idesc = ptx::idesc_bf16(kRows, 64, false, true);
-        for (int i = 0; i < nk; ++i) {
-            const int st = i % kApStages;
-            if (!ptx::mbar_wait(bar_addr(smem, off_bar, st), (i / kApStages) & 1, abort)) break;
-            ptx::tc_fence_after();
-            const uint32_t base = ptx::smem_u32(smem + st * kApStageBytes);
-            const uint64_t da = ptx::smem_desc_sw128(base, 16, 1024);
-            const uint64_t db = ptx::smem_desc_sw128(base + kRows * kBoxBytes, 64 * kBoxBytes, 1024);
+    } else {
+        pdl_wait();
+        pdl_trigger();
+        if (warp == 1 && lane == 0) {  // MMA issuer
+            const uint32_t idesc = ptx::idesc_bf16(kRows, ncols, false, true);
+            for (int i = 0; i < nk; ++i) {
+                const int st = i % n_stages;
+                if (!ptx::mbar_wait(bar_addr(smem, off_bar, st), (i / n_stages) & 1, abort)) break;
+                ptx::tc_fence_after();
+                const uint32_t base = ptx::smem_u32(smem + st * stage_bytes);
+                const uint64_t da = ptx::smem_desc_sw128(base, 16, 1024);
+                // B: the nb boxes of 64 columns are 8 KB apart (LBO); 8-row atoms 1 KB apart (SBO)
+                const uint64_t db = ptx::smem_desc_sw128(base + kRows * kBoxBytes, 64 * kBoxBytes, 1024);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                ptx::mma_bf16_1(tmem, da + 2 * kk, db + static_cast<uint64_t>((2048 * kk) >> 4), idesc,
-                                (i | kk) != 0);
-            ptx::mma_commit_1(bar_addr(smem, off_bar, kApStages + st));
+                for (int kk = 0; kk < 4; ++kk)
+                    ptx::mma_bf16_1(tmem, da + 2 * kk, db + static_cast<uint64_t>((2048 * kk) >> 4), idesc,
+                                    (i | kk) != 0);
+                ptx::mma_commit_1(bar_addr(smem, off_bar, n_stages + st));
+            }
+            ptx::mma_commit_1(bar_addr(smem, off_bar, 2 * n_stages));
         }
-        ptx::mma_commit_1(bar_addr(smem, off_bar, 2 * kApStages));
     }
-    // thread t = TMEM lane t = token row m0 + t: the CTA's partial tile into shared memory
-    // (row t: 64 floats = 16 chunks of 16 B, chunk c at (c ^ (t & 15)) to spread the banks);
-    // the ring is free once every MMA is done
-    const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_addr(smem, off_bar, 2 * kApStages), 0, abort));
+    // epilogue: thread t = TMEM lane t = token row m0 + t, 32 columns at a time
+    const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_addr(smem, off_bar, 2 * n_stages), 0, abort));
     ptx::tc_fence_after();
     const int t = static_cast<int>(threadIdx.x);
-    float* red = reinterpret_cast<float*>(smem);
-    {
-        float v[64];
-        float (&v0)[32] = *reinterpret_cast<float(*)[32]>(&v[0]);
-        float (&v1)[32] = *reinterpret_cast<float(*)[32]>(&v[32]);
-        const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        ptx::tmem_ld32(tl, v0);
-        ptx::tmem_ld32(tl + 32, v1);
+    const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+#pragma unroll 1
+    for (int c0 = 0; c0 < ncols; c0 += 32) {
+        float v[32];
+        ptx::tmem_ld32(tl + c0, v);
         ptx::tmem_wait_ld();
         if (!ok || nk == 0) {  // nothing accumulated (or a wait gave up): contribute zeros
 #pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] = 0.f;
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
         }
-        if (S == 1) {
-            if (m0 + t < T) {
-                float4* dst = reinterpret_cast<float4*>(kv + static_cast<int64_t>(m0 + t) * N + n0);
+        if (m0 + t < T) {
+            float4* dst = reinterpret_cast<float4*>(part + static_cast<int64_t>(m0 + t) * N + n0 + c0);
 #pragma unroll
-                for (int c = 0; c < 16; ++c) dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-            }
-        } else {
-#pragma unroll
-            for (int c = 0; c < 16; ++c)
-                *reinterpret_cast<float4*>(red + t * 64 + ((c ^ (t & 15)) << 2)) =
-                    make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            for (int c = 0; c < 8; ++c) dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
         }
-    }
-    if (S > 1) {
-        ptx::cluster_sync();  // every partial tile of the cluster is in shared memory
-        const int rows = kRows / S, r0 = static_cast<int>(ptx::cluster_ctarank()) * rows;  // this CTA's rows
-        const uint32_t red_s = ptx::smem_u32(red);
-        for (int idx = t; idx < rows * 16; idx += kThreads) {
-            const int row = r0 + idx / 16, c = idx % 16;
-            const uint32_t off = static_cast<uint32_t>(row * 64 + ((c ^ (row & 15)) << 2)) * 4;
-            float4 b[8];  // every peer's chunk is requested before any is summed
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                if (q < S) b[q] = ld_dsmem_v4(ptx::mapa(red_s + off, static_cast<uint32_t>(q)));
-            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                if (q < S) { a.x += b[q].x; a.y += b[q].y; a.z += b[q].z; a.w += b[q].w; }
-            if (m0 + row < T) *reinterpret_cast<float4*>(kv + static_cast<int64_t>(m0 + row) * N + n0 + 4 * c) = a;
-        }
-        ptx::cluster_sync();  // peers stay resident until every read of their tile is done
     }
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 2) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc_1(tmem, 64);
+        ptx::tmem_dealloc_1(tmem, ncols);
     }
+}
+
+// y[t, :] = bf16(sum_z part[z][t][:]) for the row GEMM's Z partials ([Z][T][N]
+// fp32, N a multiple of 4). Thread = 4 consecutive columns of one row; up to
+// four partials are requested before any is summed. grid ceil(T N / 512);
+// block 128.
+__global__ void __launch_bounds__(128) sum_partials_kernel(const float* __restrict__ part, int32_t Z, int32_t T,
+                                                           int32_t N, uint16_t* __restrict__ y) {
+    pdl_wait();
+    pdl_trigger();
+    const int64_t i4 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+    const int64_t zs = static_cast<int64_t>(T) * N;
+    if (i4 >= zs) return;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int z0 = 0; z0 < Z; z0 += 4) {
+        float4 b[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            b[u] = z0 + u < Z ? __ldg(reinterpret_cast<const float4*>(part + (z0 + u) * zs + i4))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) { a.x += b[u].x; a.y += b[u].y; a.z += b[u].z; a.w += b[u].w; }
+    }
+    *reinterpret_cast<uint2*>(y + i4) = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
 }
 
 }  // namespace tc05

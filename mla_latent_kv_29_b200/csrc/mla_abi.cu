@@ -251,33 +251,48 @@ int ensure_smem(K kernel, size_t bytes) {
     return MLA_OK;
 }
 
-// ---- append split-K plan ----------------------------------------------
-// tc: the tcgen05 GEMM (N and hidden multiples of 64), its K split over
-// `cluster` * `splits` CTAs: `splits` clusters of `cluster` CTAs that reduce
-// on chip, so the epilogue sums `splits` partials; otherwise the CUDA-core
-// GEMM writes `splits` partials.
+// ---- row GEMM plan ------------------------------------------------------
+// tc: the tcgen05 row GEMM (N and the inner dimension multiples of 64): column
+// tiles of 64 nb, the K-blocks of 64 split into `splits` ranges of
+// k_per_split, one CTA per (column tile, row tile, range); the consumer sums
+// the `splits` partials, four per memory round trip. The split is chosen to
+// cover the weight in whole waves of CTAs (one per SM) at the least bytes per
+// SM: weights, activations (from L2) and the partials' round trip, with the
+// consumer's round trips counted as the bytes an SM streams in that time.
+// Otherwise the CUDA-core GEMM writes `splits` partials.
 struct AppendPlan {
     bool tc;
-    int splits, k_per_split, cluster;
+    int splits, k_per_split, nb;
 };
 
 AppendPlan append_plan(int32_t n_tokens, int32_t hidden, int32_t N) {
     AppendPlan a;
     a.tc = (N % 64 == 0) && (hidden % 64 == 0);
-    a.cluster = 1;
+    a.nb = 1;
     if (a.tc) {
-        const int64_t tiles = static_cast<int64_t>(N / 64) * ((n_tokens + tc05::kRows - 1) / tc05::kRows);
-        const int k_blocks = hidden / 64;
-        const int sms = num_sms();
-        int s = 8;  // a portable cluster; it must divide the 128 rows of a tile
-        while (s > 1 && (tiles * s > sms || s > k_blocks)) s /= 2;
-        // One cluster along K: two clusters of 8 per column tile (144 CTAs for 64
-        // tokens) measured slower than one (15.3 against 10.2 us), so the kernel's
-        // support for several clusters along K is not used here.
-        const int z = 1;
-        a.cluster = s;
-        a.splits = z;
-        a.k_per_split = (k_blocks + s * z - 1) / (s * z);  // in K-blocks of 64 per CTA
+        const int64_t kb = hidden / 64, mt = (n_tokens + tc05::kRows - 1) / tc05::kRows, sms = num_sms();
+        double best = -1.0;
+        for (int nb = 4; nb >= 1; nb /= 2) {
+            if (N % (64 * nb)) continue;
+            const int64_t nt = N / (64 * nb);
+            for (int64_t kpc = 1; kpc <= kb; ++kpc) {
+                const int64_t z = (kb + kpc - 1) / kpc;
+                if (kpc > 1 && (kb + kpc - 2) / (kpc - 1) == z) continue;  // a smaller kpc does the same
+                const int64_t ctas = nt * mt * z, waves = (ctas + sms - 1) / sms;
+                // bytes per SM: weights (HBM), activations (L2, a quarter of the cost), the
+                // partials written and read back, and the consumer's memory round trips (one
+                // per four partials, ~0.7 us, the bytes an SM streams meanwhile at ~44 GB/s)
+                const double per_sm = static_cast<double>(waves) * kpc *
+                                          (nb * 64.0 * tc05::kBoxBytes + 0.25 * tc05::kRows * tc05::kBoxBytes) +
+                                      2.0 * 4.0 * z * n_tokens * N / sms + 31e3 * static_cast<double>((z + 3) / 4);
+                if (best < 0 || per_sm < best) {
+                    best = per_sm;
+                    a.nb = nb;
+                    a.k_per_split = static_cast<int>(kpc);
+                    a.splits = static_cast<int>(z);
+                }
+            }
+        }
         return a;
     }
     const int tile_n = kApTileN, tile_t = kApTileT, tile_k = kApTileK;
@@ -295,7 +310,7 @@ AppendPlan append_plan(int32_t n_tokens, int32_t hidden, int32_t N) {
 }
 
 // part[z][t][n] (fp32 [ap.splits][T][N]) = the K-range z of x . w on the
-// tcgen05 GEMM: x bf16 [T, K], w bf16 [K, N], K and N multiples of 64,
+// tcgen05 row GEMM: x bf16 [T, K], w bf16 [K, N], K and N multiples of 64,
 // x and w 16-byte aligned.
 int launch_row_gemm(const void* x, int32_t T, int32_t K, const void* w, int32_t N, const AppendPlan& ap,
                     float* part, cudaStream_t st) {
@@ -303,11 +318,11 @@ int launch_row_gemm(const void* x, int32_t T, int32_t K, const void* w, int32_t 
     CUtensorMap tm_x, tm_w;
     if (int rc = encode_2d(&tm_x, x, K, T, tc05::kRows)) return rc;
     if (int rc = encode_2d(&tm_w, w, N, K, 64)) return rc;
-    const size_t smem = tc05::append_smem();
-    if (int rc = ensure_smem(tc05::append_kernel, smem)) return rc;
-    const dim3 grid(N / 64, (T + tc05::kRows - 1) / tc05::kRows, ap.cluster * ap.splits);
-    return launch_cluster(tc05::append_kernel, grid, tc05::kThreads, smem, st, dim3(1, 1, ap.cluster), tm_x, tm_w, T,
-                          N, K / 64, ap.k_per_split, ap.cluster, part);
+    const size_t smem = tc05::row_gemm_smem(ap.nb);
+    if (int rc = ensure_smem(tc05::row_gemm_kernel, smem)) return rc;
+    const dim3 grid(N / (64 * ap.nb), (T + tc05::kRows - 1) / tc05::kRows, ap.splits);
+    return launch(tc05::row_gemm_kernel, grid, tc05::kThreads, smem, st, tm_x, tm_w, T, N, K / 64, ap.k_per_split,
+                  ap.nb, part);
 }
 
 // ---- query projection workspace: GEMM 1 partials | c_q bf16 | GEMM 2 partials
@@ -320,7 +335,8 @@ int q_proj_layout(const mla_dims_t* d, int32_t T, int32_t hidden, int32_t R, QPr
     if (int rc = check_dims(d)) return rc;
     if (T < 1 || hidden < 1 || R < 1) return MLA_ERR_INVALID_ARG;
     const int64_t N2 = static_cast<int64_t>(d->num_heads) * (d->qk_nope_dim + d->rope_dim);
-    if (hidden % 64 || R % 64 || N2 % 64 || N2 >= (int64_t(1) << 30) || d->rope_dim % 2 ||
+    if (hidden % 64 || R % 64 || R > kQNormThreads * kQNormCols || N2 % 64 || N2 >= (int64_t(1) << 30) ||
+        d->rope_dim % 2 ||
         d->rope_dim > 2 * kQMaxRopePairs || d->qk_nope_dim + d->rope_dim / 2 > 1024)
         return MLA_ERR_UNSUPPORTED_DIMS;
     L->g1 = append_plan(T, hidden, R);
@@ -526,6 +542,8 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     const bool tc05 = tc05_dims_ok(dims) && aligned(q_nope, 16) && aligned(q_pe, 16) && aligned(w_uk, 16) &&
                       aligned(w_uv, 16) && aligned(out, 16);
     if (L.kernel == kKernelPair && !tc05) return MLA_ERR_INVALID_ARG;
+    const bool latent_out = opts && opts->output_latent;
+    if (latent_out && !tc05) return MLA_ERR_UNSUPPORTED_DIMS;  // o_lat comes from the tensor-core merge
 
     const size_t plan_smem = sizeof(int32_t) * (static_cast<size_t>(G) + 1);
     const int32_t prefix_in_smem = plan_smem <= 48 * 1024 ? 1 : 0;
@@ -615,7 +633,20 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     // the fused merge + up-projection takes bf16 partials, d_v = 128 and at most
     // 64 * kMuvMaxBox partial slots per block of 64 groups (<= 64 + workers - 1)
     const int muv_box = static_cast<int>((std::min<int64_t>(G, tc05::kMuvRows) + L.workers - 1 + 63) / 64);
-    if (tc05 && L.kernel == kKernelPair && dims->v_head_dim == tc05::kMuvDv && muv_box <= tc05::kMuvMaxBox) {
+    if (latent_out) {
+        // out = o_lat (bf16 [G, H, d_c]): the merge only; W_UV is applied later, absorbed into W_O
+        uint16_t* o_lat = static_cast<uint16_t*>(out);
+        const dim3 mgrid(G, (H + 3) / 4);
+        if (L.kernel == kKernelPair) {
+            if (int rc = launch(tc05::merge_kernel<uint16_t>, mgrid, 128, 0, st,
+                                reinterpret_cast<const uint16_t*>(o_part), lse_part, part_offsets, G, H, dc, o_lat))
+                return rc;
+        } else {
+            if (int rc = launch(tc05::merge_kernel<float>, mgrid, 128, 0, st, o_part, lse_part, part_offsets, G, H, dc,
+                                o_lat))
+                return rc;
+        }
+    } else if (tc05 && L.kernel == kKernelPair && dims->v_head_dim == tc05::kMuvDv && muv_box <= tc05::kMuvMaxBox) {
         CUtensorMap tm_wuv, tm_p;
         if (int rc = encode_2d(&tm_wuv, w_uv, dc, static_cast<uint64_t>(H) * tc05::kMuvDv, tc05::kMuvDv)) return rc;
         if (int rc = encode_parts(&tm_p, o_part, dc, H, L.max_parts)) return rc;
@@ -655,6 +686,30 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
             o_part, lse_part, part_offsets, static_cast<const uint16_t*>(w_uv), G, H, dc, dims->v_head_dim,
             static_cast<uint16_t*>(out))) return rc;
     }
+    return launch_status();
+}
+
+size_t mla_o_proj_workspace_size(int32_t n_tokens, int32_t k, int32_t n) {
+    if (n_tokens < 1 || k < 64 || n < 64 || k % 64 || n % 64) return 0;
+    const AppendPlan a = append_plan(n_tokens, k, n);
+    return align_up(sizeof(float) * static_cast<size_t>(a.splits) * n_tokens * n);
+}
+
+int mla_o_proj(const void* x, int32_t n_tokens, int32_t k, const void* w, int32_t n, void* y, void* workspace,
+               size_t workspace_bytes, void* stream) {
+    if (!x || !w || !y || !workspace || n_tokens < 1 || k < 1 || n < 1) return MLA_ERR_INVALID_ARG;
+    if (k % 64 || n % 64) return MLA_ERR_UNSUPPORTED_DIMS;
+    if (!aligned(workspace, kAlign) || !aligned(x, 16) || !aligned(w, 16) || !aligned(y, 8)) return MLA_ERR_INVALID_ARG;
+    if (workspace_bytes < mla_o_proj_workspace_size(n_tokens, k, n)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+    if (int rc = device_ok()) return rc;
+    cudaStream_t st = as_stream(stream);
+    const AppendPlan ap = append_plan(n_tokens, k, n);
+    float* part = static_cast<float*>(workspace);
+    if (int rc = launch_row_gemm(x, n_tokens, k, w, n, ap, part, st)) return rc;
+    const int64_t quads = static_cast<int64_t>(n_tokens) * n / 4;
+    if (int rc = launch(tc05::sum_partials_kernel, static_cast<unsigned>((quads + 127) / 128), 128, 0, st,
+                        static_cast<const float*>(part), ap.splits, n_tokens, n, static_cast<uint16_t*>(y)))
+        return rc;
     return launch_status();
 }
 

@@ -3,7 +3,7 @@
 // (q_b_proj), each head's qk_head_dim values split into the d_n non-RoPE part
 // and the d_r RoPE part, the latter rotated (rotate-half RoPE of
 // "一次讲透MHA、GQA、MQA、MLA", "MLA的实现") at the token's position.
-// The two GEMMs run on tc05::append_kernel (fp32 partials); the kernels here
+// The two GEMMs run on tc05::row_gemm_kernel (fp32 partials); the kernels here
 // are the row normalisation between them and the split + RoPE after them.
 // Both run once per CTA, so their loops stay rolled.
 #pragma once
@@ -13,6 +13,7 @@
 namespace mla {
 
 constexpr int kQNormThreads = 256;
+constexpr int kQNormCols = 8;  // q_rank <= 256 * 8
 
 // out[t, :] = bf16(c / sqrt(mean(c^2) + eps) * gamma), c = sum over the
 // `splits` partials part[z][t][:] (fp32, [splits][T][R]). grid T; block 256;
@@ -26,14 +27,36 @@ __global__ void __launch_bounds__(kQNormThreads) q_norm_kernel(const float* __re
     extern __shared__ float row[];
     __shared__ float red[kQNormThreads / 32];
     const int t = blockIdx.x;
+    // thread j owns columns j + 256 i (i < kQNormCols); the columns of four
+    // splits are requested together, so four splits cost one memory round trip
+    float acc[kQNormCols];
+#pragma unroll
+    for (int i = 0; i < kQNormCols; ++i) acc[i] = 0.f;
+    const int64_t zs = static_cast<int64_t>(T) * R;
+    const float* src = part + static_cast<int64_t>(t) * R + threadIdx.x;
+#pragma unroll 1
+    for (int z0 = 0; z0 < splits; z0 += 4) {
+        float v[4][kQNormCols];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int i = 0; i < kQNormCols; ++i)
+                v[u][i] = (z0 + u < splits && static_cast<int>(threadIdx.x) + kQNormThreads * i < R)
+                              ? __ldg(src + (z0 + u) * zs + kQNormThreads * i)
+                              : 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int i = 0; i < kQNormCols; ++i) acc[i] += v[u][i];
+    }
     float ss = 0.f;
-#pragma unroll 1
-    for (int n = threadIdx.x; n < R; n += kQNormThreads) {
-        float v = 0.f;
-#pragma unroll 1
-        for (int z = 0; z < splits; ++z) v += part[(static_cast<int64_t>(z) * T + t) * R + n];
-        row[n] = v;
-        ss = fmaf(v, v, ss);
+#pragma unroll
+    for (int i = 0; i < kQNormCols; ++i) {
+        const int n = static_cast<int>(threadIdx.x) + kQNormThreads * i;
+        if (n < R) {
+            row[n] = acc[i];
+            ss = fmaf(acc[i], acc[i], ss);
+        }
     }
     ss = warp_sum(ss);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;

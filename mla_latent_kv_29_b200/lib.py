@@ -30,7 +30,8 @@ KERNEL_AUTO, KERNEL_SM100, KERNEL_GENERIC = 0, 1, 2
 
 EXPORTED = ("mla_append_kv", "mla_append_workspace_size", "mla_decode", "mla_decode_workspace_size",
             "mla_combine", "mla_debug_resolve_slots", "mla_get_device_error", "mla_error_string",
-            "mla_version", "mla_decode_no_alloc", "mla_q_proj", "mla_q_proj_workspace_size")
+            "mla_version", "mla_decode_no_alloc", "mla_q_proj", "mla_q_proj_workspace_size", "mla_o_proj",
+            "mla_o_proj_workspace_size")
 
 
 class MLAError(RuntimeError):
@@ -49,7 +50,7 @@ class CDecodeOpts(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("num_workers", ctypes.c_int32),
                 ("event_attn_begin", ctypes.c_void_p), ("event_attn_end", ctypes.c_void_p),
                 ("cache_ready", ctypes.c_void_p), ("debug_wait_limit_us", ctypes.c_uint32),
-                ("debug_starve", ctypes.c_int32)]
+                ("debug_starve", ctypes.c_int32), ("output_latent", ctypes.c_int32)]
 
 
 _lib = None
@@ -79,6 +80,8 @@ def load():
         "mla_decode_no_alloc": (_I32, [D, _P, _P, _I32, _I32, _P, _I64, _P, _I32, _P, _I32, _P, _P, _P, O, _P]),
         "mla_q_proj": (_I32, [D, _P, _I32, _I32, _P, _I32, _P, _F, _P, _P, _F, _P, _P, _P, _SZ, _P]),
         "mla_q_proj_workspace_size": (_SZ, [D, _I32, _I32, _I32]),
+        "mla_o_proj": (_I32, [_P, _I32, _I32, _P, _I32, _P, _P, _SZ, _P]),
+        "mla_o_proj_workspace_size": (_SZ, [_I32, _I32, _I32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -105,10 +108,11 @@ def _event_handle(ev) -> Optional[int]:
 
 
 def c_opts(kernel: int = KERNEL_AUTO, num_workers: int = 0, events=None, cache_ready=None,
-           debug_wait_limit_us: int = 0, debug_starve: bool = False) -> CDecodeOpts:
+           debug_wait_limit_us: int = 0, debug_starve: bool = False, output_latent: bool = False) -> CDecodeOpts:
     b, e = (None, None) if events is None else (_event_handle(events[0]), _event_handle(events[1]))
     r = None if cache_ready is None else _event_handle(cache_ready)
-    return CDecodeOpts(int(kernel), int(num_workers), b, e, r, int(debug_wait_limit_us), int(bool(debug_starve)))
+    return CDecodeOpts(int(kernel), int(num_workers), b, e, r, int(debug_wait_limit_us), int(bool(debug_starve)),
+                       int(bool(output_latent)))
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -193,6 +197,32 @@ def q_proj(dims: Dims, x, w_qa, w_qb, positions, q_gamma=None, rms_eps: float = 
     return q_nope, q_pe
 
 
+# ------------------------------------------------------- output projection
+def o_proj_workspace_size(n_tokens: int, k: int, n: int) -> int:
+    return int(load().mla_o_proj_workspace_size(n_tokens, k, n))
+
+
+def o_proj(x, w, y=None, workspace=None, stream=None):
+    """mla_o_proj: y [T, n] = bf16(x [T, k] . w [k, n]); x may be any contiguous
+    tensor whose trailing dims flatten to k (e.g. the decode output [B, Sq, H, d_v])."""
+    lib = load()
+    x2 = x.reshape(-1, w.shape[0]) if x.dim() != 2 else x
+    T, k = x2.shape
+    n = w.shape[1]
+    need = lib.mla_o_proj_workspace_size(T, k, n)
+    if need == 0:
+        raise MLAError(-2, "mla_o_proj_workspace_size")
+    if workspace is None:
+        workspace = _workspace(need, x.device)
+    if y is None:
+        y = torch.empty(T, n, dtype=torch.bfloat16, device=x.device)
+    st = lib.mla_o_proj(_ptr(x2, torch.bfloat16, "x"), T, k, _ptr(w, torch.bfloat16, "w"), n,
+                        _ptr(y, torch.bfloat16, "y"), _ptr(workspace, None, "workspace"),
+                        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "mla_o_proj")
+    return y
+
+
 # ------------------------------------------------------------------ decode
 def decode_workspace_size(dims: Dims, softmax_scale: float, batch: int, q_len: int, max_context_len: int,
                           kernel: int = KERNEL_AUTO, num_workers: int = 0) -> int:
@@ -204,19 +234,21 @@ def decode_workspace_size(dims: Dims, softmax_scale: float, batch: int, q_len: i
 def decode(dims: Dims, softmax_scale: float, q_nope, q_pe, pool, block_table, context_lens,
            max_context_len: int, w_uk, w_uv, out=None, workspace=None, kernel: int = KERNEL_AUTO,
            num_workers: int = 0, stream=None, attn_events=None, cache_ready=None, debug_wait_limit_us: int = 0,
-           debug_starve: bool = False):
+           debug_starve: bool = False, output_latent: bool = False):
     """attn_events: optional (begin, end) torch.cuda.Event pair recorded around the
     attention kernel on the launch stream. cache_ready: optional torch.cuda.Event
     (already recorded once, so that it has a handle) that the attention launch
     waits for, e.g. recorded after an append_kv on another stream.
     debug_wait_limit_us / debug_starve: the failure-detection test hooks of
-    mla_decode_opts_t (leave at 0 / False)."""
+    mla_decode_opts_t (leave at 0 / False). output_latent: return o_lat
+    [B, Sq, H, d_c] instead of the up-projected output (w_uv is not read)."""
     lib = load()
     cd = c_dims(dims, softmax_scale)
-    o = c_opts(kernel, num_workers, attn_events, cache_ready, debug_wait_limit_us, debug_starve)
+    o = c_opts(kernel, num_workers, attn_events, cache_ready, debug_wait_limit_us, debug_starve, output_latent)
     B, Sq = q_nope.shape[0], q_nope.shape[1]
     if out is None:
-        out = torch.empty(B, Sq, dims.num_heads, dims.v_head_dim, dtype=torch.bfloat16, device=q_nope.device)
+        width = dims.kv_lora_rank if output_latent else dims.v_head_dim
+        out = torch.empty(B, Sq, dims.num_heads, width, dtype=torch.bfloat16, device=q_nope.device)
     need = lib.mla_decode_workspace_size(ctypes.byref(cd), B, Sq, int(max_context_len), ctypes.byref(o))
     if need == 0:
         raise MLAError(-2, "mla_decode_workspace_size")

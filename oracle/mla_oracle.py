@@ -259,3 +259,52 @@ def absorb_query(q_nope, w_uk) -> np.ndarray:
 def up_project(o_lat, w_uv) -> np.ndarray:
     """out[..., h, :] = W_UV[h] o_lat[..., h, :] (the value up-projection)."""
     return np.einsum("...hc,hvc->...hv", _f64(o_lat), _f64(w_uv))
+
+
+# --------------------------------------------------- output projection ----
+def output_projection(out, w_o) -> np.ndarray:
+    """y = concat_h(out[..., h, :]) . W_O, the projection after the per-head
+    up-projection ([MQA-MLA] "MLA的实现": forward_training ends with w_o over
+    the heads' outputs laid side by side; [MLA-arch] 3.1).
+
+    out [..., H, d_v]; w_o [H * d_v, hidden], row h * d_v + d holding head h's
+    value index d (the page's linear weight viewed as [D_model, N_h, D_h],
+    transposed). Returns float64 [..., hidden].
+    """
+    o = _f64(out)
+    return o.reshape(o.shape[:-2] + (-1,)) @ _f64(w_o)
+
+
+def absorbed_output_weight(w_uv, w_o) -> np.ndarray:
+    """W_UV absorbed into the output projection, stacked per head.
+
+    Block h (rows h * d_c .. (h + 1) * d_c - 1) is W_UV[h]^T . W_O[h * d_v ..
+    (h + 1) * d_v - 1] ([MQA-MLA] forward_inference_absorbed, the einsum that
+    fuses w_uv into w_o; [MLA-arch] 3.1, W_V absorbed into the O projection),
+    so that o_lat[..., H, d_c] flattened times this weight is the output
+    projection of the up-projected heads. Returns float64 [H * d_c, hidden].
+    """
+    wv, wo = _f64(w_uv), _f64(w_o)
+    H, dv, _ = wv.shape
+    return np.concatenate([wv[h].T @ wo[h * dv:(h + 1) * dv] for h in range(H)], axis=0)
+
+
+def decode_latent_paged(q_nope, q_pe, pool, block_table, lengths, w_uk, dims, scale: float,
+                        batch_ids=None) -> np.ndarray:
+    """o_lat [B, Sq, H, d_c] float64: the attention output in the latent space
+    (softmax of the absorbed scores applied to c, [MQA-MLA]
+    forward_inference_absorbed before its output einsum), per new token with
+    the causal rule above. Rows of sequences outside ``batch_ids`` are NaN."""
+    q_lat = absorb_query(q_nope, w_uk)
+    qp = _f64(q_pe)
+    B, sq, H = q_lat.shape[:3]
+    out = np.full((B, sq, H, dims.kv_lora_rank), np.nan)
+    ids = range(B) if batch_ids is None else batch_ids
+    lengths = [int(v) for v in (lengths.tolist() if hasattr(lengths, "tolist") else lengths)]
+    for b in ids:
+        c, kpe = gather_sequence(pool, block_table, b, lengths[b], dims)
+        for s in range(sq):
+            n = visible_count(lengths[b], sq, s)
+            for h in range(H):
+                out[b, s, h], _ = latent_partial(q_lat[b, s, h], qp[b, s, h], c[:n], kpe[:n], scale)
+    return out

@@ -177,3 +177,71 @@ def test_q_proj_matches_oracle(case):
         # c_q is rounded to bf16 before the second product and the result once more
         scale = np.abs(ref).max()
         assert np.all(np.abs(got - ref) <= 2.0 ** -6 * np.abs(ref) + 2.0 ** -8 * scale)
+
+
+# ------------------------------------------------------- output projection
+def _check(got, ref):
+    got = got.float().cpu().numpy() if isinstance(got, torch.Tensor) else got
+    assert np.all(np.isfinite(got))
+    ok, err, bound = tolerance_ok(got, ref)
+    assert ok, f"max|err| {err:.3e} > {bound:.3e}"
+
+
+@pytest.mark.parametrize("T,K,N", [(1, 256, 128), (64, 2048, 576), (130, 1024, 320), (64, 16384, 256)])
+def test_o_proj_matches_oracle(T, K, N):
+    """mla_o_proj y = bf16(x W) against the oracle's output projection (x read as
+    heads of 64 values), over row tiles, ragged rows and several K splits."""
+    L = _lib()
+    g = torch.Generator().manual_seed(T * 7 + K + N)
+    x = I.bf16(torch.randn(T, K, generator=g))
+    w = I.bf16(torch.randn(K, N, generator=g) / math.sqrt(K))
+    y = L.o_proj(x.cuda(), w.cuda())
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    _check(y, O.output_projection(x.view(T, K // 64, 64), w))
+
+
+def test_output_projection_after_decode_unfused_and_absorbed():
+    """The decode output through W_O, and the full absorption: the decode's o_lat
+    (output_latent) through W_UV^T W_O; both against the oracle's explicit
+    decode followed by the output projection, and o_lat against the oracle's
+    latent decode."""
+    L = _lib()
+    w = I.scaled(I.WORKLOADS["v3_b64_l1k_8k"], batch=3, q_len=2, name="o_proj_chain")
+    data = build(w, lengths=torch.tensor([300, 77, 129], dtype=torch.int32))
+    dd = to_device(data)
+    d = w.dims
+    hidden = 256
+    g = torch.Generator().manual_seed(31)
+    w_o = I.bf16(torch.randn(d.num_heads * d.v_head_dim, hidden, generator=g) / math.sqrt(d.num_heads * d.v_head_dim))
+    args = (d, w.softmax_scale, dd["q_nope"], dd["q_pe"], dd["pool"], dd["table"], dd["lengths"], 300,
+            dd["w_uk"], dd["w_uv"])
+    explicit = O.decode_paged(data["q_nope"], data["q_pe"], data["pool"], data["table"].numpy(), data["lengths"],
+                              data["w_uk"], data["w_uv"], d, w.softmax_scale)
+    ref_y = O.output_projection(explicit, w_o).reshape(-1, hidden)
+    out = L.decode(*args)
+    y = L.o_proj(out, w_o.cuda())
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    _check(y, ref_y)
+    o_lat = L.decode(*args, output_latent=True)
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    assert tuple(o_lat.shape) == (3, 2, d.num_heads, d.kv_lora_rank)
+    _check(o_lat, O.decode_latent_paged(data["q_nope"], data["q_pe"], data["pool"], data["table"].numpy(),
+                                        data["lengths"], data["w_uk"], d, w.softmax_scale))
+    w_f = torch.from_numpy(O.absorbed_output_weight(data["w_uv"], w_o)).to(torch.bfloat16)
+    y_f = L.o_proj(o_lat, w_f.cuda())
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    _check(y_f, ref_y)
+
+
+def test_output_latent_needs_the_tensor_core_merge():
+    L = _lib()
+    w = I.WORKLOADS["tiny_b1_l128"]
+    dd = to_device(build(w))
+    with pytest.raises(L.MLAError) as e:
+        L.decode(w.dims, w.softmax_scale, dd["q_nope"], dd["q_pe"], dd["pool"], dd["table"], dd["lengths"], 128,
+                 dd["w_uk"], dd["w_uv"], output_latent=True)
+    assert e.value.status == -2

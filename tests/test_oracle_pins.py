@@ -480,3 +480,88 @@ def test_dims_match_printed_sizes():
     assert (2 * d.num_heads * d.qk_nope_dim) // d.kv_lora_rank == g["latent_compression_ratio"]
     assert d.qk_nope_dim + d.rope_dim == g["qk_head_dim"]
     assert d.num_heads * (d.qk_nope_dim + d.rope_dim) == g["q_b_proj_out"]
+
+
+# ------------------------------------------------------------------------
+# output projection and W_UV absorbed into it
+# ([MQA-MLA] "MLA的实现": forward_training's w_o and forward_inference_absorbed's
+# W_o_absorbed = W_UV^T W_O; [MLA-arch] 3.1, W_V absorbed into the O projection)
+# ------------------------------------------------------------------------
+def _brute_output_projection(out, w_o):
+    """y[t][m] = sum over heads h and value indices d of out[t][h][d] W_O[h d_v + d][m]."""
+    T, H, dv = len(out), len(out[0]), len(out[0][0])
+    hidden = len(w_o[0])
+    y = [[0.0] * hidden for _ in range(T)]
+    for t in range(T):
+        for m in range(hidden):
+            acc = 0.0
+            for h in range(H):
+                for d in range(dv):
+                    acc += out[t][h][d] * w_o[h * dv + d][m]
+            y[t][m] = acc
+    return y
+
+
+def test_output_projection_against_brute_force():
+    rng = _rng(21)
+    out = rng.standard_normal((3, 4, 5))
+    w_o = rng.standard_normal((20, 7))
+    np.testing.assert_allclose(O.output_projection(out, w_o), _brute_output_projection(out.tolist(), w_o.tolist()),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_output_projection_with_identity_weight_concatenates_heads():
+    rng = _rng(22)
+    out = rng.standard_normal((2, 3, 4))
+    y = O.output_projection(out, np.eye(12))
+    np.testing.assert_array_equal(y, out.reshape(2, 12))
+    # one head's block alone: y reads that head's values only
+    w = np.zeros((12, 4))
+    w[4:8] = np.eye(4)
+    np.testing.assert_array_equal(O.output_projection(out, w), out[:, 1, :])
+
+
+@pytest.mark.parametrize("H,dc,dv,hidden", [(3, 8, 4, 5), (4, 32, 16, 24)])
+def test_absorbed_output_weight_identity(H, dc, dv, hidden):
+    """o_lat . (W_UV^T W_O) == (W_UV o_lat) . W_O for every head (associativity)."""
+    rng = _rng(23)
+    o_lat = rng.standard_normal((2, 3, H, dc))
+    w_uv = rng.standard_normal((H, dv, dc)) / math.sqrt(dc)
+    w_o = rng.standard_normal((H * dv, hidden))
+    unfused = O.output_projection(O.up_project(o_lat, w_uv), w_o)
+    fused = o_lat.reshape(2, 3, H * dc) @ O.absorbed_output_weight(w_uv, w_o)
+    np.testing.assert_allclose(fused, unfused, rtol=1e-10, atol=1e-12)
+
+
+def test_absorbed_output_weight_detects_head_mixups():
+    """The identity is sharp: pairing head h's W_UV with another head's W_O block,
+    or using W_UV without the transpose, breaks it."""
+    rng = _rng(24)
+    H, dc, dv, hidden = 3, 6, 6, 5
+    o_lat = rng.standard_normal((4, H, dc))
+    w_uv = rng.standard_normal((H, dv, dc))
+    w_o = rng.standard_normal((H * dv, hidden))
+    good = O.output_projection(O.up_project(o_lat, w_uv), w_o)
+    rolled = O.absorbed_output_weight(np.roll(w_uv, 1, axis=0), w_o)
+    untransposed = np.concatenate([w_uv[h] @ w_o[h * dv:(h + 1) * dv] for h in range(H)], axis=0)
+    for bad_w in (rolled, untransposed):
+        assert np.max(np.abs(o_lat.reshape(4, H * dc) @ bad_w - good)) > 1e-3
+
+
+def test_decode_latent_up_projects_to_the_explicit_decode():
+    """W_UV applied to the latent decode output equals the explicit
+    (decompressed) decode, over a paged pool with several new tokens."""
+    rng = _rng(25)
+    d = _small_dims(H=3, dc=8, dr=4, dn=5, dv=4, bs=4)
+    lengths = [9, 4]
+    sq = 2
+    table = np.array([[5, 1, 3], [0, -1, -1]])
+    pool = rng.standard_normal((6, d.block_size, d.row_width))
+    q_nope = rng.standard_normal((2, sq, d.num_heads, d.qk_nope_dim))
+    q_pe = rng.standard_normal((2, sq, d.num_heads, d.rope_dim))
+    w_uk = rng.standard_normal((d.num_heads, d.qk_nope_dim, d.kv_lora_rank))
+    w_uv = rng.standard_normal((d.num_heads, d.v_head_dim, d.kv_lora_rank))
+    scale = 0.4
+    o_lat = O.decode_latent_paged(q_nope, q_pe, pool, table, lengths, w_uk, d, scale)
+    explicit = O.decode_paged(q_nope, q_pe, pool, table, lengths, w_uk, w_uv, d, scale)
+    np.testing.assert_allclose(O.up_project(o_lat, w_uv), explicit, rtol=1e-10, atol=1e-12)
