@@ -92,22 +92,23 @@ __global__ void __launch_bounds__(256) append_epilogue_kernel(AppendEpiloguePara
     const int N = P.dc + P.dr;
     const int64_t split_stride = static_cast<int64_t>(P.T) * N;
     // kv[n] = sum over splits; each thread owns columns threadIdx.x + 256 i (i < 3 for
-    // N = 576) and loads four splits of all its columns before summing them, so the
-    // loads of a thread are independent and few memory round trips are exposed.
+    // N = 576) and requests eight splits of all its columns before summing them, so
+    // the loads of a thread are independent and few memory round trips are exposed.
     constexpr int kCols = 4;  // N <= 1024
+    constexpr int kBatch = 8;
     float acc[kCols] = {0.f, 0.f, 0.f, 0.f};
     const float* src = P.part + static_cast<int64_t>(t) * N + threadIdx.x;
-    for (int k0 = 0; k0 < P.splits; k0 += 4) {
-        float v[4][kCols];
+    for (int k0 = 0; k0 < P.splits; k0 += kBatch) {
+        float v[kBatch][kCols];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < kBatch; ++u)
 #pragma unroll
             for (int i = 0; i < kCols; ++i) {
                 const int n = static_cast<int>(threadIdx.x) + 256 * i;
                 v[u][i] = (k0 + u < P.splits && n < N) ? __ldg(src + (k0 + u) * split_stride + 256 * i) : 0.f;
             }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < kBatch; ++u)
 #pragma unroll
             for (int i = 0; i < kCols; ++i) acc[i] += v[u][i];
     }
