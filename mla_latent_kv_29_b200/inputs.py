@@ -111,6 +111,13 @@ WORKLOADS = {
         name="v3_b64_l8k", dims=V3, batch=64, q_len=1, length_range=(8192, 8192),
         softmax_scale=1.0 / math.sqrt(192.0), w_std=math.sqrt(1.0 / 512.0), paged=True,
         kv_values="rmsnorm_rope", seed=1005),
+    # chunked prefill: 4 sequences each append a chunk of 128 prompt tokens
+    # (positions 3968..4095) and attend causally over their 4096-token context
+    "v3_b4_sq128_l4k_prefill": Workload(
+        name="v3_b4_sq128_l4k_prefill", dims=V3, batch=4, q_len=128,
+        length_range=(4096, 4096), softmax_scale=1.0 / math.sqrt(192.0),
+        w_std=math.sqrt(1.0 / 512.0), paged=True, kv_values="rmsnorm_rope", seed=1006,
+        append_hidden=7168, append_w_std=math.sqrt(1.0 / 7168.0)),
 }
 
 # Salts for independent streams.

@@ -95,6 +95,19 @@ def test_v3_small_cases(kernel, case, workers):
 
 
 @pytest.mark.parametrize("kernel", list(KERNELS))
+@pytest.mark.parametrize("workers", [0, 7])
+def test_prefill_chunk(kernel, workers):
+    """A chunk of 128 prompt tokens per sequence (chunked prefill): query s of
+    sequence b sees tokens 0 .. L_b - 128 + s. The first sequence holds only
+    the chunk (its first query sees one token); the second has 572 older
+    tokens, so its queries span several tiles and a ragged tail."""
+    w, lengths = small_v3("prefill_chunk", 2, 128, [128, 700])
+    data = build(w, lengths=lengths)
+    got = run_decode(w, to_device(data), kernel=KERNELS[kernel], num_workers=workers)
+    check(got, oracle_out(w, data))
+
+
+@pytest.mark.parametrize("kernel", list(KERNELS))
 def test_nan_in_unused_rows_and_blocks(kernel):
     w, lengths = small_v3("nan_fill", 3, 2, [70, 5, 200], spare=3)
     data = build(w, fill=float("nan"), lengths=lengths)
@@ -369,3 +382,19 @@ def test_full_size_sq4_with_append():
     ids = _sample(w, 2)
     ref = oracle_out(w, data, batch_ids=ids, pool=oracle_append_pool(w, data))
     check(got, ref, ids=ids)
+
+
+def test_full_size_prefill_chunk_with_append():
+    """Chunked prefill at full size: 4 sequences append 128 prompt tokens each
+    (512 rows through the append GEMM), then attend over 4096 tokens."""
+    L = _lib()
+    w = I.WORKLOADS["v3_b4_sq128_l4k_prefill"]
+    data = build(w, fill=float("nan"))
+    dd = to_device(data)
+    ap = dd["append"]
+    L.append_kv(w.dims, ap["x"], ap["w_kva"], ap["seq_ids"], ap["positions"], dd["table"], dd["pool"])
+    got = run_decode(w, dd)
+    ids = _sample(w, 1)
+    ref = oracle_out(w, data, batch_ids=ids, pool=oracle_append_pool(w, data))
+    check(got, ref, ids=ids)
+    assert np.all(np.isfinite(got))
