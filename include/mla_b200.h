@@ -115,6 +115,11 @@ typedef struct mla_decode_opts {
      * Needs the tensor-core merge (kv_lora_rank 256 or 512, the alignment
      * below), else MLA_ERR_UNSUPPORTED_DIMS before anything is enqueued. */
     int32_t output_latent;
+    /* 0: `pool` is the bf16 cache. 1: `pool` is the FP8 cache (layout below;
+     * num_blocks blocks of mla_fp8_block_bytes()). The tensor-core kernel
+     * reads it (DeepSeek-V3 dims); anything else returns
+     * MLA_ERR_UNSUPPORTED_DIMS before enqueuing. */
+    int32_t cache_fp8;
 } mla_decode_opts_t;
 
 /* Paged latent cache ("pool"), [MLA-arch] 3.2 kept as one row per token:
@@ -126,6 +131,34 @@ typedef struct mla_decode_opts {
  *               block_table[b][t / block_size] * block_size + t % block_size
  * A contiguous cache is block_size >= context length with block b for
  * sequence b. */
+
+/* FP8 latent cache. [MLA-arch] 4.2 item 3 ("量化的影响") notes that
+ * quantising the cache shrinks it further and warns about numerical
+ * stability; it fixes no format, so this library defines one:
+ *   code   = OCP E4M3 ("fn": bias 7, subnormals, max 448, S.1111.111 NaN) of
+ *            c / s_t, rounded to nearest even, saturated to +-448;
+ *   s_t    = 2^e_t per token, e_t the smallest integer with
+ *            max_i |c_t[i]| <= 448 * 2^e_t, clamped to [-15, 7] (division by
+ *            s_t is exact; code * s_t is exactly an IEEE half);
+ *   k_pe   = IEEE half (f16), rounded to nearest even.
+ * Block layout (block_size tokens, all little-endian):
+ *   block_size rows of (kv_lora_rank + 2 * rope_dim) bytes: the codes, then
+ *   the f16 k_pe; then block_size fp32 scales s_t.
+ * DeepSeek-V3: 41216 bytes per 64-token block (644 per token; bf16: 1152).
+ * Dequantised cache: c~ = value(code) * s_t, k_pe~ = the f16 value; the
+ * decode over an FP8 pool computes the absorbed attention of that cache.
+ * kv_lora_rank must be a multiple of 16, rope_dim of 8, block_size of 4. */
+
+/* Bytes of one FP8 cache block; 0 for unsupported dims. */
+MLA_API size_t mla_fp8_block_bytes(const mla_dims_t* dims);
+
+/* Converts a bf16 pool (num_blocks blocks, layout above) into the FP8 layout:
+ * every row, the unused ones included (rows must hold finite values; a NaN
+ * gives NaN codes). pool bf16 [num_blocks, block_size, d_c + d_r] and
+ * pool_fp8 (num_blocks * mla_fp8_block_bytes bytes), both 16-byte aligned,
+ * not overlapping. */
+MLA_API int mla_cache_to_fp8(const mla_dims_t* dims, const void* pool, int64_t num_blocks, void* pool_fp8,
+                             void* stream);
 
 /* ------------------------------------------------------------------ */
 /* Cache append: [MLA-arch] 2.2 (kv_a_proj_with_mqa, kv_a_layernorm) and
@@ -154,6 +187,17 @@ MLA_API int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_token
                   void* workspace, size_t workspace_bytes, void* stream);
 
 MLA_API size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t n_tokens, int32_t hidden);
+
+/* mla_append_kv into the FP8 cache: the same arguments and checks, pool_fp8
+ * in the FP8 layout. c is rounded to bf16 (the value the bf16 cache would
+ * store) and then quantised with its token's scale; k_pe is rounded to f16
+ * from fp32. The workspace size is mla_append_workspace_size's. */
+MLA_API int mla_append_kv_fp8(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t hidden,
+                              const void* w_kva, const void* rms_gamma, float rms_eps, float rope_base,
+                              const int32_t* seq_ids, const int32_t* positions,
+                              const int32_t* block_table, int32_t num_seqs, int32_t max_blocks_per_seq,
+                              void* pool_fp8, int64_t num_blocks,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------ */
 /* Query projection of new tokens, the step before the absorption:
@@ -222,7 +266,9 @@ MLA_API size_t mla_q_proj_workspace_size(const mla_dims_t* dims, int32_t n_token
  * softmax weights to bf16 before the value product; accumulation and the
  * combine are fp32; split partials are fp32 (CUDA-core kernel) or rounded
  * to bf16 (tcgen05 kernel); o_lat is rounded to bf16 before the
- * up-projection and out to bf16 once. */
+ * up-projection and out to bf16 once. With the FP8 cache (opts->cache_fp8)
+ * q_lat, q_pe and the softmax weights are rounded to f16 instead, and the
+ * cache enters the products as its exact dequantised f16 values. */
 MLA_API int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe,
                int32_t batch, int32_t q_len,
                const void* pool, int64_t num_blocks,

@@ -7,10 +7,14 @@
 //
 // Two launches: a split-K GEMM writing fp32 partial sums, then one CTA per
 // token that reduces the splits and runs the normalise / rotate / scatter
-// epilogue (the RMSNorm needs the whole 512-wide row).
+// epilogue (the RMSNorm needs the whole 512-wide row). The epilogue writes a
+// bf16 row, or (fp8 set) the row of the FP8 cache (fp8.cuh): c rounded to
+// bf16 first, its e4m3 codes under the per-token power-of-two scale, and k_pe
+// as f16.
 #pragma once
 
 #include "common.cuh"
+#include "fp8.cuh"
 
 namespace mla {
 
@@ -75,12 +79,26 @@ struct AppendEpilogueParams {
     const int32_t* seq_ids;
     const int32_t* positions;
     const int32_t* block_table;
-    uint16_t* pool;
+    uint16_t* pool;        // bf16 rows (fp8 = 0)
+    uint8_t* pool8;        // FP8 blocks (fp8 = 1)
+    fp8::Layout layout8;   // row / scale offsets of the FP8 blocks
+    int32_t fp8;
     int64_t num_blocks;
     int32_t splits, T, dc, dr, num_seqs, max_blocks_per_seq, block_size;
     float eps;
     double rope_base;
 };
+
+// RoPE angle of pair i at position pos: pos * base^(-2i/dr), formed in double and
+// reduced to [-pi, pi] with a two-term 2*pi so the float sine/cosine stay on
+// their short-argument path.
+__device__ __forceinline__ void rope_sincos(int32_t pos, int i, int dr, double base, float* s, float* c) {
+    const double inv_freq = exp2(-2.0 * i / static_cast<double>(dr) * log2(base));
+    const double angle = static_cast<double>(pos) * inv_freq;
+    const double k = rint(angle * 0.15915494309189535);  // 1 / (2 pi)
+    const double reduced = fma(-k, 2.4492935982947064e-16, fma(-k, 6.283185307179586, angle));
+    sincosf(static_cast<float>(reduced), s, c);
+}
 
 // grid (T); block 256; dynamic smem (dc + dr) floats.
 __global__ void __launch_bounds__(256) append_epilogue_kernel(AppendEpilogueParams P) {
@@ -137,6 +155,40 @@ __global__ void __launch_bounds__(256) append_epilogue_kernel(AppendEpiloguePara
         if (threadIdx.x == 0) record_status(MLA_ERR_DEVICE_FAULT);
         return;
     }
+    const int half = P.dr / 2;
+    if (P.fp8) {
+        // c as the bf16 cache would hold it, kept in kv[] for the encode pass
+        float amax = 0.f;
+        for (int n = threadIdx.x; n < P.dc; n += blockDim.x) {
+            float c = kv[n] * r;
+            if (P.gamma) c *= bf16_to_f32(P.gamma[n]);
+            c = bf16_to_f32(f32_to_bf16(c));
+            kv[n] = c;
+            amax = fmaxf(amax, fabsf(c));
+        }
+        amax = warp_max(amax);
+        __syncthreads();  // every thread has read red[0]
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+        __syncthreads();
+        amax = 0.f;
+        for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) amax = fmaxf(amax, red[w]);
+        const int e = fp8::scale_exp(amax);
+        const float inv = fp8::pow2(-e);
+        uint8_t* d8 = P.pool8 + P.layout8.row_off(row);
+        uint16_t* codes = reinterpret_cast<uint16_t*>(d8);
+        for (int n2 = threadIdx.x; n2 < P.dc / 2; n2 += blockDim.x)
+            codes[n2] = fp8::e4m3x2(kv[2 * n2] * inv, kv[2 * n2 + 1] * inv);
+        uint16_t* pe = reinterpret_cast<uint16_t*>(d8 + P.dc);
+        for (int i = threadIdx.x; i < half; i += blockDim.x) {
+            float s, c;
+            rope_sincos(pos, i, P.dr, P.rope_base, &s, &c);
+            const float x1 = kv[P.dc + i], x2 = kv[P.dc + i + half];
+            pe[i] = fp8::f16_bits(x1 * c - x2 * s);
+            pe[i + half] = fp8::f16_bits(x2 * c + x1 * s);
+        }
+        if (threadIdx.x == 0) *reinterpret_cast<float*>(P.pool8 + P.layout8.scale_off(row)) = fp8::pow2(e);
+        return;
+    }
     uint16_t* dst = P.pool + row * N;
     for (int n = threadIdx.x; n < P.dc; n += blockDim.x) {
         float c = kv[n] * r;
@@ -144,16 +196,9 @@ __global__ void __launch_bounds__(256) append_epilogue_kernel(AppendEpiloguePara
         dst[n] = f32_to_bf16(c);
     }
     // rotate-half RoPE: pair (i, i + dr/2) rotated by pos * base^(-2i/dr)
-    const int half = P.dr / 2;
     for (int i = threadIdx.x; i < half; i += blockDim.x) {
-        // angle = pos * base^(-2i/dr), formed in double; reduced to [-pi, pi] with a
-        // two-term 2*pi so the float sine/cosine stay on their short-argument path
-        const double inv_freq = exp2(-2.0 * i / static_cast<double>(P.dr) * log2(P.rope_base));
-        const double angle = static_cast<double>(pos) * inv_freq;
-        const double k = rint(angle * 0.15915494309189535);  // 1 / (2 pi)
-        const double reduced = fma(-k, 2.4492935982947064e-16, fma(-k, 6.283185307179586, angle));
         float s, c;
-        sincosf(static_cast<float>(reduced), &s, &c);
+        rope_sincos(pos, i, P.dr, P.rope_base, &s, &c);
         const float x1 = kv[P.dc + i], x2 = kv[P.dc + i + half];
         dst[P.dc + i] = f32_to_bf16(x1 * c - x2 * s);
         dst[P.dc + i + half] = f32_to_bf16(x2 * c + x1 * s);

@@ -46,11 +46,25 @@
 // MLA_ERR_DEVICE_TIMEOUT and every role drains to the common exit. With the
 // test hook `starve` the load warps issue nothing at all, so no copy or
 // tensor-core operation is in flight when the consumers' waits run out.
+//
+// FP8 cache (pair_decode_f8_kernel; the format is in fp8.cuh). The same
+// pipeline with f16 operands: the absorbed queries arrive as f16, the softmax
+// writes P as f16, and every cache box is expanded in place. The load warps
+// copy each [rows x 64] box of e4m3 codes (64 bytes a row, unswizzled) into
+// the upper half of the shared-memory box that will hold its f16 values, and
+// the token scales into the lower half of the stage's first box; two more
+// warps (384 threads) turn them into exactly the 128B-swizzled f16 boxes the
+// bf16 path loads directly (warp 10 the key stages, warp 11 the value stages,
+// zeroing value rows past the visible range), then signal the stage full to
+// the leader. Each warp reads a box's codes and scales into registers before
+// any lane writes it. The f16 RoPE key box is copied as it is. HBM bytes per
+// token: 644 instead of 1152.
 #pragma once
 
 #include "common.cuh"
 #include "plan.cuh"
 #include "sm100.cuh"
+#include "fp8.cuh"
 
 namespace mla {
 namespace pair {
@@ -72,6 +86,10 @@ constexpr int kVStage = 2 * kBox;    // value stage: 32 tokens x 256 latent colu
 constexpr int kVPerTile = 4;         // 4 value stages per tile
 constexpr int kVStages = 4;          // value ring: four stages (a whole tile)
 constexpr int kThreads = 320;  // 10 warps; the softmax warps 4-7 own TMEM lanes 0-127
+constexpr int kF8Threads = 384;  // FP8 cache: + warp 10 (key expansion) and warp 11 (value expansion)
+constexpr int kF8Row = kDc + 2 * kDr;  // 640 bytes: 512 e4m3 codes, then the f16 RoPE key
+constexpr int kF8KSrc = kBox / 2;      // a key box's 64 rows of 64 codes sit in its upper 4 KB
+constexpr int kF8VSrc = kBox / 4;      // a value box's 32 rows of 64 codes sit in its upper 2 KB
 constexpr int kTmemCols = 512;
 constexpr int kTmS = 0;          // two S buffers (tile parity), each lo and hi halves of 64 columns
 constexpr int kTmO = 256;        // O: 256 columns (after the two S buffers of 128)
@@ -86,7 +104,8 @@ enum Bar {
     B_QFULL = 0, B_QEMPTY, B_SFULL0, B_SFULL1, B_SEMPTY0, B_SEMPTY1, B_PFULL0, B_PFULL1, B_PVDONE0, B_PVDONE1,
     B_OEMPTY, B_PATCH, B_XCHG,
     B_KFULL0, B_KEMPTY0 = B_KFULL0 + kKStages, B_VFULL0 = B_KEMPTY0 + kKStages, B_VEMPTY0 = B_VFULL0 + kVStages,
-    B_COUNT = B_VEMPTY0 + kVStages
+    B_KRAW0 = B_VEMPTY0 + kVStages, B_VRAW0 = B_KRAW0 + kKStages,  // FP8: codes landed (this CTA)
+    B_COUNT = B_VRAW0 + kVStages
 };
 constexpr int kOffRed = kOffBar + 8 * 64;          // exchange buffer [2][128] floats
 constexpr int kOffMisc = kOffRed + 2 * 128 * 4;    // abort flag, TMEM base
@@ -110,6 +129,7 @@ struct Params {
     float scale_log2;  // softmax_scale * log2(e)
     uint64_t wait_ns;  // limit of every bounded wait (ptx::kWaitLimitNs unless a test shortens it)
     int32_t starve;    // test hook: the load warps issue nothing, so every consumer wait runs out
+    int64_t f8_block_bytes;  // FP8 cache: bytes of one cache block (rows, then scales)
 };
 
 struct Ctx {
@@ -134,13 +154,23 @@ __device__ __forceinline__ void ring_next(uint32_t& stage, uint32_t& phase) {
 
 // Starts pulling this CTA's 64-token page of tile j of `seg` (73,728
 // contiguous bytes: the 64 rows lie in one pool block because block_size is a
-// multiple of 64) from HBM into L2, so that its key loads a tile later hit L2.
+// multiple of 64; FP8: 40,960 bytes of rows and the page's 256 bytes of
+// scales) from HBM into L2, so that its key loads a tile later hit L2.
+template <bool kF8>
 __device__ __forceinline__ void prefetch_page(const Params& P, const Ctx& c, const Segment& seg, int j) {
     const int32_t th = seg.tok_begin + j * kTile + 64 * static_cast<int32_t>(c.rank);
     if (th >= seg.tok_end) return;
     const int64_t row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks, P.block_size,
                                     seg.group / P.q_len, th);
-    if (row >= 0) ptx::prefetch_l2(P.pool + row * (kD * 2), 64 * kD * 2);
+    if (row < 0) return;
+    if (kF8) {
+        const int64_t blk = row / P.block_size, slot = row % P.block_size;
+        const uint8_t* base = P.pool + blk * P.f8_block_bytes;
+        ptx::prefetch_l2(base + slot * kF8Row, 64 * kF8Row);
+        ptx::prefetch_l2(base + static_cast<int64_t>(P.block_size) * kF8Row + 4 * slot, 64 * 4);
+    } else {
+        ptx::prefetch_l2(P.pool + row * (kD * 2), 64 * kD * 2);
+    }
 }
 
 // Queries and key stages; one thread (lane 0 of warp 0). tm_q, tm_k3 and
@@ -156,7 +186,7 @@ __device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUt
     Segment seg;
     {
         SegmentIter peek = it;
-        if (peek.next(seg)) prefetch_page(P, c, seg, 0);
+        if (peek.next(seg)) prefetch_page<false>(P, c, seg, 0);
     }
     while (it.next(seg)) {
         const int32_t g = seg.group, b = g / P.q_len;
@@ -179,11 +209,11 @@ __device__ void key_producer(const Params& P, const CUtensorMap* tm_q, const CUt
                 row = 0;
             }
             if (j + 1 < n_tiles) {
-                prefetch_page(P, c, seg, j + 1);
+                prefetch_page<false>(P, c, seg, j + 1);
             } else {
                 SegmentIter peek = it;
                 Segment nx;
-                if (peek.next(nx)) prefetch_page(P, c, nx, 0);
+                if (peek.next(nx)) prefetch_page<false>(P, c, nx, 0);
             }
             for (int ks = 0; ks < kKStages; ++ks) {
                 if (!ptx::mbar_wait(c.bar(B_KEMPTY0 + ks), phase ^ 1, c.abort, c.wait_ns)) return;
@@ -277,6 +307,239 @@ __device__ void value_producer(const Params& P, const CUtensorMap* tm_v, const C
     }
 }
 
+// ------------------------------------------------------------ FP8 cache loads
+// Coordinates of pool row `row` (= block * block_size + slot) in the FP8 maps.
+struct F8At {
+    int32_t slot, block;
+};
+__device__ __forceinline__ F8At f8_at(int64_t row, int32_t bs) {
+    return {static_cast<int32_t>(row % bs), static_cast<int32_t>(row / bs)};
+}
+
+// Queries and key stages over the FP8 cache; one thread (lane 0 of warp 0).
+// tm_k8: the codes {640 bytes, block_size rows, blocks} (row pitch 640, block
+// pitch f8_block_bytes), box {64, 64, 1}, unswizzled; tm_ks: the scales
+// {block_size, blocks} fp32, box {64, 1}; tm_kr: the f16 RoPE keys {64,
+// block_size, blocks}, box {64, 64, 1}, 128B-swizzled. Key stage ks receives
+// the codes of its column blocks (all but block 8, the RoPE key) in the upper
+// halves of their boxes, the page's 64 scales at the start of its first box,
+// and (last stage) the RoPE box in place, all on this CTA's KRAW barrier; the
+// key expansion warp then fills the leader's KFULL.
+__device__ void key_producer_f8(const Params& P, const CUtensorMap* tm_q, const CUtensorMap* tm_k8,
+                                const CUtensorMap* tm_ks, const CUtensorMap* tm_kr, const Ctx& c) {
+    uint32_t phase = 0;
+    int seg_i = 0;
+    SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    Segment seg;
+    {
+        SegmentIter peek = it;
+        if (peek.next(seg)) prefetch_page<true>(P, c, seg, 0);
+    }
+    while (it.next(seg)) {
+        const int32_t g = seg.group, b = g / P.q_len;
+        if (seg_i > 0 && !ptx::mbar_wait(c.bar(B_QEMPTY), (seg_i - 1) & 1, c.abort, c.wait_ns)) return;
+        {
+            const uint32_t full = c.leader_bar(B_QFULL);
+            ptx::mbar_arrive_expect_tx_cluster(full, kQBoxes * kBox);
+            ptx::tma_load_3d_pair(c.sbase + kOffQ, tm_q, 0, g * kH + 64 * c.rank, 0, full);
+        }
+        const int n_tiles = tiles_of(seg);
+        for (int j = 0; j < n_tiles; ++j) {
+            const int32_t t0 = seg.tok_begin + j * kTile;
+            int32_t th = t0 + 64 * static_cast<int32_t>(c.rank);
+            if (th >= seg.tok_end) th = t0;  // no visible token in this half: any valid page (masked)
+            int64_t row = resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks, P.block_size,
+                                      b, th);
+            if (row < 0) {
+                record_status(MLA_ERR_DEVICE_FAULT);
+                row = 0;
+            }
+            const F8At at = f8_at(row, P.block_size);
+            if (j + 1 < n_tiles) {
+                prefetch_page<true>(P, c, seg, j + 1);
+            } else {
+                SegmentIter peek = it;
+                Segment nx;
+                if (peek.next(nx)) prefetch_page<true>(P, c, nx, 0);
+            }
+            for (int ks = 0; ks < kKStages; ++ks) {
+                if (!ptx::mbar_wait(c.bar(B_KEMPTY0 + ks), phase ^ 1, c.abort, c.wait_ns)) return;
+                const uint32_t raw = c.bar(B_KRAW0 + ks);
+                const int blk = kstage_first_block(ks);
+                const bool last = ks == kKStages - 1;
+                const int n8 = last ? kstage_blocks(ks) - 1 : kstage_blocks(ks);
+                ptx::mbar_arrive_expect_tx_local(raw, n8 * kF8KSrc + 64 * 4 + (last ? kBox : 0));
+                for (int i = 0; i < n8; ++i)
+                    ptx::tma_load_3d(c.sbase + kOffK + (blk + i) * kBox + kF8KSrc, tm_k8, 64 * (blk + i), at.slot,
+                                     at.block, raw);
+                ptx::tma_load_2d(c.sbase + kOffK + blk * kBox, tm_ks, at.slot, at.block, raw);
+                if (last) ptx::tma_load_3d(c.sbase + kOffK + (kQBoxes - 1) * kBox, tm_kr, 0, at.slot, at.block, raw);
+            }
+            phase ^= 1;
+        }
+        ++seg_i;
+    }
+    for (int ks = 0; ks < kKStages; ++ks)  // tail, as in key_producer
+        if (!ptx::mbar_wait(c.bar(B_KEMPTY0 + ks), phase ^ 1, c.abort, c.wait_ns)) return;
+    if (seg_i > 0) ptx::mbar_wait(c.bar(B_QEMPTY), (seg_i - 1) & 1, c.abort, c.wait_ns);
+}
+
+// Value stages over the FP8 cache; one thread (lane 0 of warp 2). tm_v8: the
+// codes with box {64, 32, 1}; tm_vs: the scales with box {32, 1}. Stage q of a
+// tile (tokens 32q..32q+31; box bx = latent columns 256r + 64bx) receives the
+// codes of its four boxes in their upper halves and the 32 scales at its start,
+// on this CTA's VRAW barrier; rows past the visible range are loaded too and
+// zeroed by the value expansion warp, which then fills the leader's VFULL.
+__device__ void value_producer_f8(const Params& P, const CUtensorMap* tm_v8, const CUtensorMap* tm_vs, const Ctx& c) {
+    uint32_t stage = 0, phase = 0;
+    SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    Segment seg;
+    while (it.next(seg)) {
+        const int32_t b = seg.group / P.q_len;
+        const int n_tiles = tiles_of(seg);
+        for (int j = 0; j < n_tiles; ++j) {
+            const int32_t tv = seg.tok_begin + j * kTile;
+            for (int q = 0; q < kVPerTile; ++q) {
+                const int32_t tq = tv + 32 * q;
+                if (seg.tok_end - tq <= 0) break;
+                const int64_t row =
+                    resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks, P.block_size, b, tq);
+                if (!ptx::mbar_wait(c.bar(B_VEMPTY0 + stage), phase ^ 1, c.abort, c.wait_ns)) return;
+                const uint32_t raw = c.bar(B_VRAW0 + stage);
+                const uint32_t dst = c.sbase + kOffV + stage * kVStage;
+                if (row >= 0) {
+                    const F8At at = f8_at(row, P.block_size);
+                    ptx::mbar_arrive_expect_tx_local(raw, 4 * kF8VSrc + 32 * 4);
+                    for (int bx = 0; bx < 4; ++bx)
+                        ptx::tma_load_3d(dst + bx * (kBox / 2) + kF8VSrc, tm_v8,
+                                         64 * (4 * static_cast<int32_t>(c.rank) + bx), at.slot, at.block, raw);
+                    ptx::tma_load_2d(dst, tm_vs, at.slot, at.block, raw);
+                } else {
+                    record_status(MLA_ERR_DEVICE_FAULT);
+                    ptx::mbar_arrive_local(raw);  // nothing loaded: the expansion writes zeros
+                }
+                ring_next<kVStages>(stage, phase);
+            }
+        }
+    }
+    for (int i = 0; i < kVStages; ++i) {  // tail, as for the key ring
+        if (!ptx::mbar_wait(c.bar(B_VEMPTY0 + stage), phase ^ 1, c.abort, c.wait_ns)) return;
+        ring_next<kVStages>(stage, phase);
+    }
+}
+
+// A wait by every lane of a warp that succeeds for all of them or for none (a
+// lane that gave up makes its warp give up): warp-collective code after it
+// (tensor-memory loads and stores, __syncwarp) stays converged.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
+    return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, limit_ns));
+}
+
+// One box expanded in place by a warp: rows r0 + 8k (k < K; r0 = lane / 4) of
+// 64 codes at `src` (64-byte rows; this lane's 16-byte chunk ch = lane % 4)
+// become f16 rows of 128 bytes at `box` in the TMA's SWIZZLE_128B layout
+// (16-byte chunk i of row r at position i ^ (r % 8); the box is 1 KB aligned),
+// the two chunks of this lane being 2ch and 2ch + 1. Rows >= keep become
+// zeros. s2[k]: the f16x2 scale of row r0 + 8k. Every lane reads its codes
+// before any lane writes, since rows 32.. of the box overlay the codes.
+template <int K>
+__device__ __forceinline__ void expand_box(uint8_t* box, const uint8_t* src, const uint32_t (&s2)[K], int r0,
+                                           int ch, int keep) {
+    uint4 v[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) v[k] = *reinterpret_cast<const uint4*>(src + (r0 + 8 * k) * 64 + 16 * ch);
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        const int r = r0 + 8 * k;
+        uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
+        if (r < keep) {
+            const uint2 a = fp8::dequant4(v[k].x, s2[k]), b = fp8::dequant4(v[k].y, s2[k]);
+            const uint2 d = fp8::dequant4(v[k].z, s2[k]), e = fp8::dequant4(v[k].w, s2[k]);
+            lo = make_uint4(a.x, a.y, b.x, b.y);
+            hi = make_uint4(d.x, d.y, e.x, e.y);
+        }
+        uint8_t* rowp = box + r * 128;
+        *reinterpret_cast<uint4*>(rowp + (((2 * ch) ^ (r & 7)) << 4)) = lo;
+        *reinterpret_cast<uint4*>(rowp + (((2 * ch + 1) ^ (r & 7)) << 4)) = hi;
+    }
+}
+
+// Key expansion (warp 10): per tile and key stage, after KRAW, the stage's
+// code boxes become f16 key boxes (scales read first: they sit in the first
+// box), then the stage is signalled to the leader's KFULL (count 2: both CTAs).
+__device__ void key_expander(const Params& P, const Ctx& c) {
+    const uint32_t lane = ptx::lane_id();
+    const int r0 = static_cast<int>(lane >> 2), ch = static_cast<int>(lane & 3);
+    uint32_t phase = 0;
+    SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    Segment seg;
+    while (it.next(seg)) {
+        const int n_tiles = tiles_of(seg);
+        for (int j = 0; j < n_tiles; ++j) {
+            for (int ks = 0; ks < kKStages; ++ks) {
+                if (!warp_wait(c.bar(B_KRAW0 + ks), phase, c.abort, c.wait_ns)) return;
+                const int blk = kstage_first_block(ks);
+                const int n8 = ks == kKStages - 1 ? kstage_blocks(ks) - 1 : kstage_blocks(ks);
+                const float* sc = reinterpret_cast<const float*>(c.smem + kOffK + blk * kBox);
+                uint32_t s2[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) s2[k] = fp8::scale_f16x2(sc[r0 + 8 * k]);
+#pragma unroll 1
+                for (int i = 0; i < n8; ++i) {
+                    uint8_t* box = c.smem + kOffK + (blk + i) * kBox;
+                    expand_box<8>(box, box + kF8KSrc, s2, r0, ch, 64);
+                }
+                ptx::fence_proxy_async_smem();  // the generic-proxy writes, before the MMAs read them
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive_cluster(c.leader_bar(B_KFULL0 + ks));
+            }
+            phase ^= 1;
+        }
+    }
+}
+
+// Value expansion (warp 11): per visible value stage, after VRAW, its four code
+// boxes become f16 value boxes (rows past the visible range, or all rows if the
+// page is missing, as zeros), then VFULL of the leader (count 2).
+__device__ void value_expander(const Params& P, const Ctx& c) {
+    const uint32_t lane = ptx::lane_id();
+    const int r0 = static_cast<int>(lane >> 2), ch = static_cast<int>(lane & 3);
+    uint32_t stage = 0, phase = 0;
+    SegmentIter it(P.hdr, P.worker_group, P.tile_prefix, P.part_offsets, P.context_lens, P.q_len, kTile, c.pair);
+    Segment seg;
+    while (it.next(seg)) {
+        const int32_t b = seg.group / P.q_len;
+        const int n_tiles = tiles_of(seg);
+        for (int j = 0; j < n_tiles; ++j) {
+            const int32_t tv = seg.tok_begin + j * kTile;
+            for (int q = 0; q < kVPerTile; ++q) {
+                const int32_t tq = tv + 32 * q;
+                const int nv = min(32, seg.tok_end - tq);
+                if (nv <= 0) break;
+                const int64_t row =
+                    resolve_row(P.block_table, P.batch, P.max_blocks_per_seq, P.num_blocks, P.block_size, b, tq);
+                if (!warp_wait(c.bar(B_VRAW0 + stage), phase, c.abort, c.wait_ns)) return;
+                const int keep = row >= 0 ? nv : 0;
+                uint8_t* st = c.smem + kOffV + stage * kVStage;
+                const float* sc = reinterpret_cast<const float*>(st);
+                uint32_t s2[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) s2[k] = fp8::scale_f16x2(sc[r0 + 8 * k]);
+#pragma unroll 1
+                for (int bx = 0; bx < 4; ++bx) {
+                    uint8_t* box = st + bx * (kBox / 2);
+                    expand_box<4>(box, box + kF8VSrc, s2, r0, ch, keep);
+                }
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive_cluster(c.leader_bar(B_VFULL0 + stage));
+                ring_next<kVStages>(stage, phase);
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------- MMA
 // Four issuing threads in the leader CTA: two for the score MMAs, two for the
 // value MMAs. A single thread issues at most about one tcgen05.mma every ~47
@@ -297,9 +560,11 @@ struct Descs {
 // 5-8 (stages 2-3) into half-accumulator h of S buffer (tile & 1), up to two
 // tiles ahead of the softmax (the S buffers). Each key stage is consumed by
 // one thread, once per tile (phase = tile parity); both threads commit QEMPTY
-// (count 2) once per segment and SFULL (count 2) once per tile.
+// (count 2) once per segment and SFULL (count 2) once per tile. kF16: f16
+// operands (FP8 cache) instead of bf16.
+template <bool kF16>
 __device__ void mma_s_issuer(const Params& P, const Ctx& c, uint32_t half) {
-    constexpr uint32_t kIdS = ptx::idesc_bf16(128, 128, false, false);
+    constexpr uint32_t kIdS = kF16 ? ptx::idesc_f16(128, 128, false, false) : ptx::idesc_bf16(128, 128, false, false);
     const Descs D(c);
     uint32_t tile_cnt = 0;
     int seg_i = 0;
@@ -341,8 +606,9 @@ __device__ void mma_s_issuer(const Params& P, const Ctx& c, uint32_t half) {
 // Both threads read every value stage and commit its VEMPTY (count 2), and
 // PVDONE (count 2) once per tile. The first value MMA of a segment overwrites
 // O, after the softmax has read out the previous segment (OEMPTY).
+template <bool kF16>
 __device__ void mma_pv_issuer(const Params& P, const Ctx& c, uint32_t half) {
-    constexpr uint32_t kIdPV = ptx::idesc_bf16(128, 256, false, true);
+    constexpr uint32_t kIdPV = kF16 ? ptx::idesc_f16(128, 256, false, true) : ptx::idesc_bf16(128, 256, false, true);
     const Descs D(c);
     uint32_t vst = 0, vph = 0, pv_cnt = 0;
     int seg_i = 0;
@@ -379,12 +645,8 @@ __device__ void mma_pv_issuer(const Params& P, const Ctx& c, uint32_t half) {
 // --------------------------------------------------------------- softmax
 // The softmax warps execute warp-collective tensor-memory instructions
 // (tcgen05.ld / st .sync.aligned), so every branch they take must be
-// warp-uniform: a wait succeeds for the whole warp or for none of it (a lane
-// that gave up makes its warp give up), and the O rescale runs for the whole
-// warp when any of its rows needs it.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
-    return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, limit_ns));
-}
+// warp-uniform: waits go through warp_wait, and the O rescale runs for the
+// whole warp when any of its rows needs it.
 
 struct Exchanger {  // swaps one float between thread t and thread t ^ 64 of the softmax warps
     float* red;
@@ -402,6 +664,7 @@ struct Exchanger {  // swaps one float between thread t and thread t ^ 64 of the
     }
 };
 
+template <bool kF16>
 __device__ void softmax(const Params& P, const Ctx& c) {
     const int t = static_cast<int>(threadIdx.x) - 128;  // TMEM lane
     const uint32_t lane = ptx::lane_id();
@@ -503,14 +766,16 @@ __device__ void softmax(const Params& P, const Ctx& c) {
             if (tc >= 1 && !wait_pv(tc - 1)) return;
             ptx::tc_fence_after();
             uint8_t* const prow = c.smem + kOffP + half * kBox + hrow * 128;
-            // P row (bf16) into the K-major 128B-swizzled A operand of the PV MMA
+            // P row (bf16, or f16 with the FP8 cache) into the K-major 128B-swizzled A
+            // operand of the PV MMA
+            auto pk = [](float lo, float hi) { return kF16 ? ptx::f16x2(lo, hi) : ptx::bf16x2(lo, hi); };
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8) {
                 uint4 u;
-                u.x = ptx::bf16x2(s[8 * c8 + 0], s[8 * c8 + 1]);
-                u.y = ptx::bf16x2(s[8 * c8 + 2], s[8 * c8 + 3]);
-                u.z = ptx::bf16x2(s[8 * c8 + 4], s[8 * c8 + 5]);
-                u.w = ptx::bf16x2(s[8 * c8 + 6], s[8 * c8 + 7]);
+                u.x = pk(s[8 * c8 + 0], s[8 * c8 + 1]);
+                u.y = pk(s[8 * c8 + 2], s[8 * c8 + 3]);
+                u.z = pk(s[8 * c8 + 4], s[8 * c8 + 5]);
+                u.w = pk(s[8 * c8 + 6], s[8 * c8 + 7]);
                 *reinterpret_cast<uint4*>(prow + ((c8 ^ (hrow & 7)) << 4)) = u;
             }
             ptx::fence_proxy_async_smem();
@@ -639,11 +904,104 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else if (warp == 2) {
         if (!P.starve) value_producer(P, &tm_v, c);
     } else if (warp == 1 || warp == 3) {
-        if (c.rank == 0 && ptx::lane_id() == 0) mma_s_issuer(P, c, static_cast<uint32_t>(warp >> 1));
+        if (c.rank == 0 && ptx::lane_id() == 0) mma_s_issuer<false>(P, c, static_cast<uint32_t>(warp >> 1));
     } else if (warp >= 8) {
-        if (c.rank == 0 && ptx::lane_id() == 0) mma_pv_issuer(P, c, static_cast<uint32_t>(warp - 8));
+        if (c.rank == 0 && ptx::lane_id() == 0) mma_pv_issuer<false>(P, c, static_cast<uint32_t>(warp - 8));
     } else if (warp >= 4) {
-        softmax(P, c);
+        softmax<false>(P, c);
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync();  // no MMA or remote arrive targets this CTA any more
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc_pair(c.tmem, kTmemCols);
+    }
+}
+
+// The same kernel over the FP8 cache: f16 queries and softmax weights, the
+// cache boxes expanded in place by warps 10 and 11 (see the header). grid: 2 *
+// workers CTAs (clusters of 2); block kF8Threads; dynamic smem kSmemBytes.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF8Threads, 1)
+    pair_decode_f8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k8,
+                          const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_kr,
+                          const __grid_constant__ CUtensorMap tm_v8, const __grid_constant__ CUtensorMap tm_vs,
+                          const Params P) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw = ptx::smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    const int warp = threadIdx.x >> 5;
+    Ctx c;
+    c.smem = smem;
+    c.sbase = ptx::smem_u32(smem);
+    c.rank = ptx::cluster_ctarank();
+    c.pair = ptx::cluster_id_x();
+    c.abort = reinterpret_cast<volatile int*>(smem + kOffMisc);
+    c.wait_ns = P.wait_ns;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc + 16);
+
+    if (threadIdx.x == 0) {
+        *c.abort = 0;
+        ptx::mbar_init(c.bar(B_QFULL), 2);
+        ptx::mbar_init(c.bar(B_QEMPTY), 2);
+        ptx::mbar_init(c.bar(B_SFULL0), 2);
+        ptx::mbar_init(c.bar(B_SFULL1), 2);
+        ptx::mbar_init(c.bar(B_SEMPTY0), 8);
+        ptx::mbar_init(c.bar(B_SEMPTY1), 8);
+        ptx::mbar_init(c.bar(B_PFULL0), 8);
+        ptx::mbar_init(c.bar(B_PFULL1), 8);
+        ptx::mbar_init(c.bar(B_PVDONE0), 2);
+        ptx::mbar_init(c.bar(B_PVDONE1), 2);
+        ptx::mbar_init(c.bar(B_OEMPTY), 8);
+        ptx::mbar_init(c.bar(B_PATCH), 1);
+        ptx::mbar_init(c.bar(B_XCHG), 4);
+        for (int s = 0; s < kKStages; ++s) {
+            ptx::mbar_init(c.bar(B_KFULL0 + s), 2);   // the key expansion warps of both CTAs
+            ptx::mbar_init(c.bar(B_KEMPTY0 + s), 1);
+            ptx::mbar_init(c.bar(B_KRAW0 + s), 1);    // this CTA's producer (+ its copies' bytes)
+        }
+        for (int s = 0; s < kVStages; ++s) {
+            ptx::mbar_init(c.bar(B_VFULL0 + s), 2);   // the value expansion warps of both CTAs
+            ptx::mbar_init(c.bar(B_VEMPTY0 + s), 2);
+            ptx::mbar_init(c.bar(B_VRAW0 + s), 1);
+        }
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && ptx::lane_id() == 0) {
+        ptx::prefetch_tmap(&tm_q);
+        ptx::prefetch_tmap(&tm_k8);
+        ptx::prefetch_tmap(&tm_ks);
+        ptx::prefetch_tmap(&tm_kr);
+        ptx::prefetch_tmap(&tm_v8);
+        ptx::prefetch_tmap(&tm_vs);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc_pair(ptx::smem_u32(tmem_slot), kTmemCols);
+        ptx::tmem_relinquish_pair();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync();  // the peer's barriers exist before anyone arrives on them
+    ptx::tc_fence_after();
+    c.tmem = *tmem_slot;
+    pdl_wait();  // the schedule and the absorbed queries come from the preceding kernels
+    pdl_trigger();
+
+    if (warp == 0) {
+        if (ptx::lane_id() == 0 && !P.starve) key_producer_f8(P, &tm_q, &tm_k8, &tm_ks, &tm_kr, c);
+    } else if (warp == 2) {
+        if (ptx::lane_id() == 0 && !P.starve) value_producer_f8(P, &tm_v8, &tm_vs, c);
+    } else if (warp == 1 || warp == 3) {
+        if (c.rank == 0 && ptx::lane_id() == 0) mma_s_issuer<true>(P, c, static_cast<uint32_t>(warp >> 1));
+    } else if (warp == 8 || warp == 9) {
+        if (c.rank == 0 && ptx::lane_id() == 0) mma_pv_issuer<true>(P, c, static_cast<uint32_t>(warp - 8));
+    } else if (warp == 10) {
+        key_expander(P, c);
+    } else if (warp == 11) {
+        value_expander(P, c);
+    } else {
+        softmax<true>(P, c);
     }
 
     ptx::tc_fence_before();

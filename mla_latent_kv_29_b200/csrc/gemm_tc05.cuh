@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(kThreads) absorb_kernel(const __grid_constant_
                                                           const __grid_constant__ CUtensorMap tm_w,
                                                           const uint16_t* __restrict__ q_pe, int32_t G, int32_t H,
                                                           int32_t dn, int32_t dc, int32_t dr,
-                                                          uint16_t* __restrict__ q_out) {
+                                                          uint16_t* __restrict__ q_out, int32_t q_f16) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
     const int a_bytes = static_cast<int>(absorb_a_bytes(dn));
@@ -567,18 +567,35 @@ __global__ void __launch_bounds__(kThreads) absorb_kernel(const __grid_constant_
             ptx::tmem_wait_ld();
             if (g < G) {
                 uint4* dst = reinterpret_cast<uint4*>(q_out + (static_cast<int64_t>(g) * H + h) * D + 256 * z + c0);
+                if (q_f16) {  // f16 queries for the FP8 cache's f16 MMAs
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    dst[i] = make_uint4(ptx::bf16x2(v[8 * i], v[8 * i + 1]), ptx::bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                                        ptx::bf16x2(v[8 * i + 4], v[8 * i + 5]),
-                                        ptx::bf16x2(v[8 * i + 6], v[8 * i + 7]));
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(ptx::f16x2(v[8 * i], v[8 * i + 1]), ptx::f16x2(v[8 * i + 2], v[8 * i + 3]),
+                                            ptx::f16x2(v[8 * i + 4], v[8 * i + 5]),
+                                            ptx::f16x2(v[8 * i + 6], v[8 * i + 7]));
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(ptx::bf16x2(v[8 * i], v[8 * i + 1]), ptx::bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                                            ptx::bf16x2(v[8 * i + 4], v[8 * i + 5]),
+                                            ptx::bf16x2(v[8 * i + 6], v[8 * i + 7]));
+                }
             }
         }
-        if (copy_pe) {  // the RoPE part of the query row
+        if (copy_pe) {  // the RoPE part of the query row (as f16 when q_f16)
             uint4* dst = reinterpret_cast<uint4*>(q_out + (static_cast<int64_t>(g) * H + h) * D + dc);
 #pragma unroll
-            for (int i = 0; i < kPe; ++i)
-                if (i < dr / 8) dst[i] = pe[i];
+            for (int i = 0; i < kPe; ++i) {
+                if (i >= dr / 8) continue;
+                uint4 u = pe[i];
+                if (q_f16) {
+                    auto cv = [](uint32_t w) {
+                        return ptx::f16x2(bf16_to_f32(w & 0xFFFFu), bf16_to_f32(w >> 16));
+                    };
+                    u = make_uint4(cv(u.x), cv(u.y), cv(u.z), cv(u.w));
+                }
+                dst[i] = u;
+            }
         }
     }
     ptx::tc_fence_before();

@@ -201,6 +201,68 @@ int encode_parts(CUtensorMap* m, const void* base, uint64_t dc, uint64_t H, uint
     return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// A tiled tensor map of any rank (<= 3) and element type: dims / byte strides /
+// box as cuTensorMapEncodeTiled takes them, unit element strides, L2
+// promotion 256 B, no fill.
+int encode_tiled(CUtensorMap* m, CUtensorMapDataType type, uint32_t rank, const void* base, const cuuint64_t* dims,
+                 const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swizzle) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return MLA_ERR_CUDA;
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, type, rank, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// The five maps of the FP8 cache the attention reads (fp8.cuh layout): codes
+// {row bytes, block_size, blocks} with boxes {64, 64, 1} (keys) and {64, 32, 1}
+// (values), unswizzled; the fp32 scales {block_size, blocks} with boxes
+// {64, 1} and {32, 1}; the f16 RoPE keys {64, block_size, blocks} with box
+// {64, 64, 1}, 128B-swizzled.
+struct F8Maps {
+    CUtensorMap k8, ks, kr, v8, vs;
+};
+int encode_f8_maps(F8Maps* M, const void* pool, const mla_dims_t* d, int64_t num_blocks) {
+    const uint64_t rb = static_cast<uint64_t>(fp8::row_bytes(d->kv_lora_rank, d->rope_dim));
+    const uint64_t bb = static_cast<uint64_t>(fp8::block_bytes(d->kv_lora_rank, d->rope_dim, d->block_size));
+    const uint64_t bs = static_cast<uint64_t>(d->block_size), nb = static_cast<uint64_t>(num_blocks);
+    const char* base = static_cast<const char*>(pool);
+    {
+        cuuint64_t dims[3] = {rb, bs, nb};
+        cuuint64_t strides[2] = {rb, bb};
+        cuuint32_t kbox[3] = {64, 64, 1}, vbox[3] = {64, 32, 1};
+        if (int rc = encode_tiled(&M->k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, kbox,
+                                  CU_TENSOR_MAP_SWIZZLE_NONE)) return rc;
+        if (int rc = encode_tiled(&M->v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, vbox,
+                                  CU_TENSOR_MAP_SWIZZLE_NONE)) return rc;
+    }
+    {
+        cuuint64_t dims[2] = {bs, nb};
+        cuuint64_t strides[1] = {bb};
+        cuuint32_t kbox[2] = {64, 1}, vbox[2] = {32, 1};
+        const char* sc = base + bs * rb;
+        if (int rc = encode_tiled(&M->ks, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, sc, dims, strides, kbox,
+                                  CU_TENSOR_MAP_SWIZZLE_NONE)) return rc;
+        if (int rc = encode_tiled(&M->vs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, sc, dims, strides, vbox,
+                                  CU_TENSOR_MAP_SWIZZLE_NONE)) return rc;
+    }
+    {
+        cuuint64_t dims[3] = {static_cast<cuuint64_t>(d->rope_dim), bs, nb};
+        cuuint64_t strides[2] = {rb, bb};
+        cuuint32_t box[3] = {64, 64, 1};
+        if (int rc = encode_tiled(&M->kr, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, base + d->kv_lora_rank, dims, strides,
+                                  box, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    }
+    return MLA_OK;
+}
+
+// The FP8 cache layout needs 16-byte rows, blocks and offsets (d_c a multiple
+// of 16, d_r of 8, block_size of 4).
+bool fp8_dims_ok(const mla_dims_t* d) {
+    return d->kv_lora_rank % 16 == 0 && d->rope_dim % 8 == 0 && d->block_size % 4 == 0;
+}
+
 // The tcgen05 absorb / merge / UV kernels: d_n a multiple of 64 up to 256, d_c
 // a multiple of 256 up to 512, d_r a multiple of 8 up to 64, d_v a multiple of 16 up
 // to 256, and 16-byte aligned operands.
@@ -391,12 +453,13 @@ size_t mla_append_workspace_size(const mla_dims_t* dims, int32_t n_tokens, int32
     return align_up(sizeof(float) * static_cast<size_t>(a.splits) * n_tokens * N);
 }
 
-int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t hidden, const void* w_kva,
-                  const void* rms_gamma, float rms_eps, float rope_base, const int32_t* seq_ids,
-                  const int32_t* positions, const int32_t* block_table, int32_t num_seqs,
-                  int32_t max_blocks_per_seq, void* pool, int64_t num_blocks, void* workspace,
-                  size_t workspace_bytes, void* stream) {
+static int append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t hidden, const void* w_kva,
+                     const void* rms_gamma, float rms_eps, float rope_base, const int32_t* seq_ids,
+                     const int32_t* positions, const int32_t* block_table, int32_t num_seqs,
+                     int32_t max_blocks_per_seq, void* pool, int64_t num_blocks, void* workspace,
+                     size_t workspace_bytes, void* stream, bool fp8_cache) {
     if (int rc = check_dims(dims)) return rc;
+    if (fp8_cache && !fp8_dims_ok(dims)) return MLA_ERR_UNSUPPORTED_DIMS;
     if (!x || !w_kva || !seq_ids || !positions || !block_table || !pool || !workspace) return MLA_ERR_INVALID_ARG;
     if (n_tokens < 1 || hidden < 1 || num_seqs < 1 || max_blocks_per_seq < 1 || num_blocks < 1)
         return MLA_ERR_INVALID_ARG;
@@ -425,6 +488,10 @@ int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32
     P.positions = positions;
     P.block_table = block_table;
     P.pool = static_cast<uint16_t*>(pool);
+    P.pool8 = static_cast<uint8_t*>(pool);
+    P.layout8 = fp8::Layout{fp8::row_bytes(dims->kv_lora_rank, dims->rope_dim),
+                            fp8::block_bytes(dims->kv_lora_rank, dims->rope_dim, dims->block_size), dims->block_size};
+    P.fp8 = fp8_cache ? 1 : 0;
     P.num_blocks = num_blocks;
     P.splits = splits;
     P.T = n_tokens;
@@ -436,6 +503,49 @@ int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32
     P.eps = rms_eps;
     P.rope_base = rope_base;
     if (int rc = launch(append_epilogue_kernel, n_tokens, 256, sizeof(float) * N, st, P)) return rc;
+    return launch_status();
+}
+
+int mla_append_kv(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t hidden, const void* w_kva,
+                  const void* rms_gamma, float rms_eps, float rope_base, const int32_t* seq_ids,
+                  const int32_t* positions, const int32_t* block_table, int32_t num_seqs,
+                  int32_t max_blocks_per_seq, void* pool, int64_t num_blocks, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+    return append_kv(dims, x, n_tokens, hidden, w_kva, rms_gamma, rms_eps, rope_base, seq_ids, positions,
+                     block_table, num_seqs, max_blocks_per_seq, pool, num_blocks, workspace, workspace_bytes, stream,
+                     false);
+}
+
+int mla_append_kv_fp8(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t hidden, const void* w_kva,
+                      const void* rms_gamma, float rms_eps, float rope_base, const int32_t* seq_ids,
+                      const int32_t* positions, const int32_t* block_table, int32_t num_seqs,
+                      int32_t max_blocks_per_seq, void* pool_fp8, int64_t num_blocks, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+    return append_kv(dims, x, n_tokens, hidden, w_kva, rms_gamma, rms_eps, rope_base, seq_ids, positions,
+                     block_table, num_seqs, max_blocks_per_seq, pool_fp8, num_blocks, workspace, workspace_bytes,
+                     stream, true);
+}
+
+size_t mla_fp8_block_bytes(const mla_dims_t* dims) {
+    if (check_dims(dims) || !fp8_dims_ok(dims)) return 0;
+    return static_cast<size_t>(fp8::block_bytes(dims->kv_lora_rank, dims->rope_dim, dims->block_size));
+}
+
+int mla_cache_to_fp8(const mla_dims_t* dims, const void* pool, int64_t num_blocks, void* pool_fp8, void* stream) {
+    if (int rc = check_dims(dims)) return rc;
+    if (!fp8_dims_ok(dims)) return MLA_ERR_UNSUPPORTED_DIMS;
+    if (!pool || !pool_fp8 || num_blocks < 1) return MLA_ERR_INVALID_ARG;
+    if (!aligned(pool, 16) || !aligned(pool_fp8, 16)) return MLA_ERR_INVALID_ARG;
+    if (int rc = device_ok()) return rc;
+    const int64_t rows = num_blocks * dims->block_size;
+    const fp8::Layout L{fp8::row_bytes(dims->kv_lora_rank, dims->rope_dim),
+                        fp8::block_bytes(dims->kv_lora_rank, dims->rope_dim, dims->block_size), dims->block_size};
+    const int64_t grid = (rows + 7) / 8;
+    if (grid > 0x7FFFFFFF) return MLA_ERR_INVALID_ARG;
+    if (int rc = launch(fp8::quantize_pool_kernel, static_cast<unsigned>(grid), 256, 0, as_stream(stream),
+                        static_cast<const uint16_t*>(pool), rows, dims->kv_lora_rank, dims->rope_dim, L,
+                        static_cast<uint8_t*>(pool_fp8)))
+        return rc;
     return launch_status();
 }
 
@@ -542,6 +652,8 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     const bool tc05 = tc05_dims_ok(dims) && aligned(q_nope, 16) && aligned(q_pe, 16) && aligned(w_uk, 16) &&
                       aligned(w_uv, 16) && aligned(out, 16);
     if (L.kernel == kKernelPair && !tc05) return MLA_ERR_INVALID_ARG;
+    const bool fp8_cache = opts && opts->cache_fp8;
+    if (fp8_cache && L.kernel != kKernelPair) return MLA_ERR_UNSUPPORTED_DIMS;  // only the tcgen05 kernel reads it
     const bool latent_out = opts && opts->output_latent;
     if (latent_out && !tc05) return MLA_ERR_UNSUPPORTED_DIMS;  // o_lat comes from the tensor-core merge
 
@@ -559,7 +671,8 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         const size_t smem = tc05::absorb_smem(dims->qk_nope_dim);
         if (int rc = ensure_smem(tc05::absorb_kernel, smem)) return rc;
         if (int rc = launch(tc05::absorb_kernel, dim3(H, (G + tc05::kRows - 1) / tc05::kRows, dc / 256), tc05::kThreads, smem, st,
-            tm_qn, tm_wuk, static_cast<const uint16_t*>(q_pe), G, H, dims->qk_nope_dim, dc, dr, q)) return rc;
+            tm_qn, tm_wuk, static_cast<const uint16_t*>(q_pe), G, H, dims->qk_nope_dim, dc, dr, q,
+            fp8_cache ? 1 : 0)) return rc;
     } else {
         const size_t absorb_smem = sizeof(float) * kAbsorbGroups * dims->qk_nope_dim;
         if (int rc = ensure_smem(absorb_q_kernel, absorb_smem)) return rc;
@@ -571,11 +684,16 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
 
     if (L.kernel == kKernelPair) {
         CUtensorMap tm_q, tm_k3, tm_k2, tm_v;
+        F8Maps f8;
         const uint64_t pool_rows = static_cast<uint64_t>(num_blocks) * dims->block_size;
         if (int rc = encode_row_blocks(&tm_q, q, pair::kD, static_cast<uint64_t>(G) * H, 64, pair::kQBoxes)) return rc;
-        if (int rc = encode_row_blocks(&tm_k3, pool, pair::kD, pool_rows, 64, 3)) return rc;
-        if (int rc = encode_row_blocks(&tm_k2, pool, pair::kD, pool_rows, 64, 2)) return rc;
-        if (int rc = encode_row_blocks(&tm_v, pool, pair::kD, pool_rows, 32, 4)) return rc;
+        if (fp8_cache) {
+            if (int rc = encode_f8_maps(&f8, pool, dims, num_blocks)) return rc;
+        } else {
+            if (int rc = encode_row_blocks(&tm_k3, pool, pair::kD, pool_rows, 64, 3)) return rc;
+            if (int rc = encode_row_blocks(&tm_k2, pool, pair::kD, pool_rows, 64, 2)) return rc;
+            if (int rc = encode_row_blocks(&tm_v, pool, pair::kD, pool_rows, 32, 4)) return rc;
+        }
         pair::Params PP;
         PP.hdr = hdr;
         PP.worker_group = worker_group;
@@ -594,10 +712,18 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
         PP.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
         PP.wait_ns = (opts && opts->debug_wait_limit_us) ? 1000ull * opts->debug_wait_limit_us : ptx::kWaitLimitNs;
         PP.starve = (opts && opts->debug_starve) ? 1 : 0;
+        PP.f8_block_bytes = fp8::block_bytes(dc, dr, dims->block_size);
         if (int rc = ensure_smem(pair::pair_decode_kernel, pair::kSmemBytes)) return rc;
+        if (int rc = ensure_smem(pair::pair_decode_f8_kernel, pair::kSmemBytes)) return rc;
         if (int rc = wait_hook(opts ? opts->cache_ready : nullptr, st)) return rc;
         record_hook(opts ? opts->event_attn_begin : nullptr, st);
-        if (int rc = launch(pair::pair_decode_kernel, 2 * L.workers, pair::kThreads, pair::kSmemBytes, st, tm_q, tm_k3, tm_k2, tm_v, PP)) return rc;
+        if (fp8_cache) {
+            if (int rc = launch(pair::pair_decode_f8_kernel, 2 * L.workers, pair::kF8Threads, pair::kSmemBytes, st,
+                                tm_q, f8.k8, f8.ks, f8.kr, f8.v8, f8.vs, PP)) return rc;
+        } else {
+            if (int rc = launch(pair::pair_decode_kernel, 2 * L.workers, pair::kThreads, pair::kSmemBytes, st, tm_q,
+                                tm_k3, tm_k2, tm_v, PP)) return rc;
+        }
         if (int rc = launch_status()) return rc;
         record_hook(opts ? opts->event_attn_end : nullptr, st);
     } else {

@@ -31,7 +31,7 @@ KERNEL_AUTO, KERNEL_SM100, KERNEL_GENERIC = 0, 1, 2
 EXPORTED = ("mla_append_kv", "mla_append_workspace_size", "mla_decode", "mla_decode_workspace_size",
             "mla_combine", "mla_debug_resolve_slots", "mla_get_device_error", "mla_error_string",
             "mla_version", "mla_decode_no_alloc", "mla_q_proj", "mla_q_proj_workspace_size", "mla_o_proj",
-            "mla_o_proj_workspace_size")
+            "mla_o_proj_workspace_size", "mla_append_kv_fp8", "mla_cache_to_fp8", "mla_fp8_block_bytes")
 
 
 class MLAError(RuntimeError):
@@ -50,7 +50,7 @@ class CDecodeOpts(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("num_workers", ctypes.c_int32),
                 ("event_attn_begin", ctypes.c_void_p), ("event_attn_end", ctypes.c_void_p),
                 ("cache_ready", ctypes.c_void_p), ("debug_wait_limit_us", ctypes.c_uint32),
-                ("debug_starve", ctypes.c_int32), ("output_latent", ctypes.c_int32)]
+                ("debug_starve", ctypes.c_int32), ("output_latent", ctypes.c_int32), ("cache_fp8", ctypes.c_int32)]
 
 
 _lib = None
@@ -82,6 +82,9 @@ def load():
         "mla_q_proj_workspace_size": (_SZ, [D, _I32, _I32, _I32]),
         "mla_o_proj": (_I32, [_P, _I32, _I32, _P, _I32, _P, _P, _SZ, _P]),
         "mla_o_proj_workspace_size": (_SZ, [_I32, _I32, _I32]),
+        "mla_append_kv_fp8": (_I32, [D, _P, _I32, _I32, _P, _P, _F, _F, _P, _P, _P, _I32, _I32, _P, _I64, _P, _SZ, _P]),
+        "mla_cache_to_fp8": (_I32, [D, _P, _I64, _P, _P]),
+        "mla_fp8_block_bytes": (_SZ, [D]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -108,11 +111,12 @@ def _event_handle(ev) -> Optional[int]:
 
 
 def c_opts(kernel: int = KERNEL_AUTO, num_workers: int = 0, events=None, cache_ready=None,
-           debug_wait_limit_us: int = 0, debug_starve: bool = False, output_latent: bool = False) -> CDecodeOpts:
+           debug_wait_limit_us: int = 0, debug_starve: bool = False, output_latent: bool = False,
+           cache_fp8: bool = False) -> CDecodeOpts:
     b, e = (None, None) if events is None else (_event_handle(events[0]), _event_handle(events[1]))
     r = None if cache_ready is None else _event_handle(cache_ready)
     return CDecodeOpts(int(kernel), int(num_workers), b, e, r, int(debug_wait_limit_us), int(bool(debug_starve)),
-                       int(bool(output_latent)))
+                       int(bool(output_latent)), int(bool(cache_fp8)))
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -148,22 +152,45 @@ def append_workspace_size(dims: Dims, n_tokens: int, hidden: int, softmax_scale:
 
 
 def append_kv(dims: Dims, x, w_kva, seq_ids, positions, block_table, pool, rms_gamma=None,
-              rms_eps: float = 1e-6, rope_base: float = 10000.0, workspace=None, stream=None):
+              rms_eps: float = 1e-6, rope_base: float = 10000.0, workspace=None, stream=None, fp8: bool = False):
+    """mla_append_kv into a bf16 pool, or (fp8) mla_append_kv_fp8 into an FP8 pool
+    (uint8 [num_blocks, fp8_block_bytes(dims)])."""
     lib = load()
     cd = c_dims(dims, 1.0)
     T, hidden = x.shape
     need = lib.mla_append_workspace_size(ctypes.byref(cd), T, hidden)
     if workspace is None:
         workspace = _workspace(need, x.device)
-    st = lib.mla_append_kv(
+    fn, name = (lib.mla_append_kv_fp8, "mla_append_kv_fp8") if fp8 else (lib.mla_append_kv, "mla_append_kv")
+    st = fn(
         ctypes.byref(cd), _ptr(x, torch.bfloat16, "x"), T, hidden, _ptr(w_kva, torch.bfloat16, "w_kva"),
         _ptr(rms_gamma, torch.bfloat16, "rms_gamma"), float(rms_eps), float(rope_base),
         _ptr(seq_ids, torch.int32, "seq_ids"), _ptr(positions, torch.int32, "positions"),
         _ptr(block_table, torch.int32, "block_table"), block_table.shape[0], block_table.shape[1],
-        _ptr(pool, torch.bfloat16, "pool"), pool.shape[0], _ptr(workspace, None, "workspace"),
+        _ptr(pool, torch.uint8 if fp8 else torch.bfloat16, "pool"), pool.shape[0], _ptr(workspace, None, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream))
-    _check(st, "mla_append_kv")
+    _check(st, name)
     return pool
+
+
+# ---------------------------------------------------------------- FP8 cache
+def fp8_block_bytes(dims: Dims) -> int:
+    return int(load().mla_fp8_block_bytes(ctypes.byref(c_dims(dims, 1.0))))
+
+
+def cache_to_fp8(dims: Dims, pool, out=None, stream=None):
+    """mla_cache_to_fp8: the FP8 pool (uint8 [num_blocks, fp8_block_bytes]) of a bf16 pool."""
+    lib = load()
+    nb = pool.shape[0]
+    bb = fp8_block_bytes(dims)
+    if bb == 0:
+        raise MLAError(-2, "mla_fp8_block_bytes")
+    if out is None:
+        out = torch.empty(nb, bb, dtype=torch.uint8, device=pool.device)
+    st = lib.mla_cache_to_fp8(ctypes.byref(c_dims(dims, 1.0)), _ptr(pool, torch.bfloat16, "pool"), nb,
+                              _ptr(out, torch.uint8, "pool_fp8"), _stream(stream))
+    _check(st, "mla_cache_to_fp8")
+    return out
 
 
 # -------------------------------------------------------- query projection
@@ -234,17 +261,19 @@ def decode_workspace_size(dims: Dims, softmax_scale: float, batch: int, q_len: i
 def decode(dims: Dims, softmax_scale: float, q_nope, q_pe, pool, block_table, context_lens,
            max_context_len: int, w_uk, w_uv, out=None, workspace=None, kernel: int = KERNEL_AUTO,
            num_workers: int = 0, stream=None, attn_events=None, cache_ready=None, debug_wait_limit_us: int = 0,
-           debug_starve: bool = False, output_latent: bool = False):
+           debug_starve: bool = False, output_latent: bool = False, cache_fp8: bool = False):
     """attn_events: optional (begin, end) torch.cuda.Event pair recorded around the
     attention kernel on the launch stream. cache_ready: optional torch.cuda.Event
     (already recorded once, so that it has a handle) that the attention launch
     waits for, e.g. recorded after an append_kv on another stream.
     debug_wait_limit_us / debug_starve: the failure-detection test hooks of
     mla_decode_opts_t (leave at 0 / False). output_latent: return o_lat
-    [B, Sq, H, d_c] instead of the up-projected output (w_uv is not read)."""
+    [B, Sq, H, d_c] instead of the up-projected output (w_uv is not read).
+    cache_fp8: `pool` is an FP8 pool (uint8 [num_blocks, fp8_block_bytes])."""
     lib = load()
     cd = c_dims(dims, softmax_scale)
-    o = c_opts(kernel, num_workers, attn_events, cache_ready, debug_wait_limit_us, debug_starve, output_latent)
+    o = c_opts(kernel, num_workers, attn_events, cache_ready, debug_wait_limit_us, debug_starve, output_latent,
+               cache_fp8)
     B, Sq = q_nope.shape[0], q_nope.shape[1]
     if out is None:
         width = dims.kv_lora_rank if output_latent else dims.v_head_dim
@@ -256,7 +285,8 @@ def decode(dims: Dims, softmax_scale: float, q_nope, q_pe, pool, block_table, co
         workspace = _workspace(need, q_nope.device)
     st = lib.mla_decode(
         ctypes.byref(cd), _ptr(q_nope, torch.bfloat16, "q_nope"), _ptr(q_pe, torch.bfloat16, "q_pe"), B, Sq,
-        _ptr(pool, torch.bfloat16, "pool"), pool.shape[0], _ptr(block_table, torch.int32, "block_table"),
+        _ptr(pool, torch.uint8 if cache_fp8 else torch.bfloat16, "pool"), pool.shape[0],
+        _ptr(block_table, torch.int32, "block_table"),
         block_table.shape[1], _ptr(context_lens, torch.int32, "context_lens"), int(max_context_len),
         _ptr(w_uk, torch.bfloat16, "w_uk"), _ptr(w_uv, torch.bfloat16, "w_uv"),
         _ptr(out, torch.bfloat16, "out"), _ptr(workspace, None, "workspace"),

@@ -98,8 +98,10 @@ def scale_exponent(amax: float) -> int:
 
 
 def f16_bits(v) -> np.ndarray:
-    """IEEE half bits (uint16) of exact values, rounded to nearest even."""
-    return np.asarray(v, dtype=np.float64).astype(np.float16).view(np.uint16)
+    """IEEE half bits (uint16) of exact values, rounded to nearest even; values
+    beyond the half range become +-inf, as IEEE rounding defines."""
+    with np.errstate(over="ignore"):
+        return np.asarray(v, dtype=np.float64).astype(np.float16).view(np.uint16)
 
 
 def f16_value(bits) -> np.ndarray:
