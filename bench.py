@@ -125,6 +125,8 @@ def workload_totals(w, lengths):
     G = w.batch * w.q_len
     row = d.row_width * 2  # bytes per cached token
     attn_bytes = T * row + G * d.num_heads * row  # cache rows + absorbed queries
+    # FP8 cache: d_c codes + d_r f16 + one fp32 scale per token (644 bytes for V3)
+    attn_bytes_fp8 = T * (d.kv_lora_rank + 2 * d.rope_dim + 4) + G * d.num_heads * row
     attn_flops = 2 * d.num_heads * (d.row_width + d.kv_lora_rank) * V
     w_bytes = 2 * d.num_heads * (d.qk_nope_dim + d.v_head_dim) * d.kv_lora_rank * 2
     step_bytes = T * row + w_bytes + G * d.num_heads * (d.qk_nope_dim + d.rope_dim + d.v_head_dim) * 2
@@ -133,7 +135,7 @@ def workload_totals(w, lengths):
     step_bytes += HIDDEN * d.row_width * 2 + G * HIDDEN * 2
     step_flops += 2 * G * HIDDEN * d.row_width
     return dict(T=T, V=V, G=G, attn_bytes=attn_bytes, attn_flops=attn_flops, step_bytes=step_bytes,
-                step_flops=step_flops)
+                step_flops=step_flops, attn_bytes_fp8=attn_bytes_fp8)
 
 
 Q_RANK = 1536  # q_lora_rank of the DeepSeek-V3 query path
@@ -176,12 +178,12 @@ def roofline(bytes_, flops, seconds, peaks):
 # for the kernel sources it was taken on (their SHA-256 below; the capture and
 # its command are summarised under profiles/). Any change to those sources
 # turns the reported traffic into null until a new capture is recorded here.
-KERNEL_SOURCES = ("decode_pair.cuh", "plan.cuh", "sm100.cuh", "common.cuh")
+KERNEL_SOURCES = ("decode_pair.cuh", "plan.cuh", "sm100.cuh", "common.cuh", "fp8.cuh")
 TRAFFIC = {
     # profiles/pair_decode_kernel_v3_b64_l1k_8k.md (ncu launch list of one step, the attention launch:
     # dram__bytes_read.sum + dram__bytes_write.sum)
-    "v3_b64_l1k_8k": {"bytes": 362545664 + 6273792,
-                      "sources_sha256": "22d86e39818b42247981432c84e3a295238f61a271b743e5641bb3de9301dc56"},
+    "v3_b64_l1k_8k": {"bytes": 364470016 + 6244096,
+                      "sources_sha256": "baeea80604bb1b037e1d8110b71db95da3e8396156de9ed42264571c4c8de60e"},
 }
 
 def kernel_sources_sha256() -> str:
@@ -363,10 +365,12 @@ def setup_gpu(w, device, rank):
     return st
 
 
-def make_step(w, st, kernel, overlap=True):
+def make_step(w, st, kernel, overlap=True, fp8=False):
     """One step: the append of the batch's new tokens, then the decode. With
     overlap the append runs on a side stream beside the decode's schedule and
-    query absorption, and the decode's attention waits for it (cache_ready)."""
+    query absorption, and the decode's attention waits for it (cache_ready).
+    fp8: both run on the FP8 cache st["pool8"] (mla_append_kv_fp8, and the
+    decode with cache_fp8)."""
     import torch
 
     from mla_latent_kv_29_b200 import lib
@@ -377,9 +381,11 @@ def make_step(w, st, kernel, overlap=True):
     fork.record()
     ready.record()  # the handles exist before any capture
 
+    pool = st["pool8"] if fp8 else st["pool"]
+
     def append(x_new, stream=None):
         lib.append_kv(d, st["x_new"] if x_new is None else x_new, st["w_kva"], st["new_seq"], st["new_pos"],
-                      st["table"], st["pool"], workspace=st["ws_append"], stream=stream)
+                      st["table"], pool, workspace=st["ws_append"], stream=stream, fp8=fp8)
 
     def step(x_new=None, q_nope=None, q_pe=None, events=None):
         if side is not None:
@@ -391,9 +397,9 @@ def make_step(w, st, kernel, overlap=True):
         else:
             append(x_new)
         lib.decode(d, w.softmax_scale, st["q_nope"] if q_nope is None else q_nope,
-                   st["q_pe"] if q_pe is None else q_pe, st["pool"], st["table"], st["lengths_d"], st["max_len"],
+                   st["q_pe"] if q_pe is None else q_pe, pool, st["table"], st["lengths_d"], st["max_len"],
                    st["w_uk"], st["w_uv"], out=st["out"], workspace=st["ws_decode"], kernel=kernel,
-                   attn_events=events, cache_ready=ready if side is not None else None)
+                   attn_events=events, cache_ready=ready if side is not None else None, cache_fp8=fp8)
 
     return step
 
@@ -461,21 +467,28 @@ def o_proj_lines(w, st, flush, K, warmup, device, peaks):
     return res
 
 
-def workload_summary(name, args, device, peaks, flush, K=10):
+def workload_summary(name, args, device, peaks, flush, K=10, fp8=False):
     """Step and attention times of another workload (same step as the headline:
     append of the new tokens + decode, CUDA graph replay, L2 flushed before
-    each step), for the summary of every configuration."""
+    each step), for the summary of every configuration. fp8: the same step on
+    the workload's cache converted to the FP8 format (mla_cache_to_fp8; the
+    bf16 pool is freed), appending with mla_append_kv_fp8."""
     import dataclasses
 
     import torch
 
     from mla_latent_kv_29_b200 import inputs as I
+    from mla_latent_kv_29_b200 import lib
 
     rank, _, _ = dist_env()
     w = I.WORKLOADS[name]
     w = dataclasses.replace(w, seed=rank_seed(w.seed, rank))
     st = setup_gpu(w, device, rank)
-    step = make_step(w, st, args.kernel, overlap=args.overlap)
+    if fp8:
+        st["pool8"] = lib.cache_to_fp8(st["d"], st["pool"])
+        st["pool"] = None
+        torch.cuda.synchronize(device)
+    step = make_step(w, st, args.kernel, overlap=args.overlap, fp8=fp8)
     ea = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
     ea[0].record()
     ea[1].record()
@@ -503,13 +516,15 @@ def workload_summary(name, args, device, peaks, flush, K=10):
         attn_ms.append(ea[0].elapsed_time(ea[1]))
     tot = workload_totals(w, st["lengths"].tolist())
     t_attn = statistics.median(attn_ms) / 1e3
-    roof, gbs, tfs = roofline(tot["attn_bytes"], tot["attn_flops"], t_attn, peaks)
+    attn_bytes = tot["attn_bytes_fp8"] if fp8 else tot["attn_bytes"]
+    roof, gbs, tfs = roofline(attn_bytes, tot["attn_flops"], t_attn, peaks)
+    assert lib.device_error() == 0
     del graphs, st
     torch.cuda.synchronize(device)
     return {"step_us_median": round(statistics.median(step_ms) * 1e3, 2),
             "attn_us_median": round(t_attn * 1e6, 2), "attn_bound": roof["bound"], "attn_frac": roof["frac"],
             "attn_frac_nominal": roof["frac_nominal"], "attn_gbs": round(gbs, 1), "attn_tflops": round(tfs, 2),
-            "cached_tokens": tot["T"], "new_tokens": tot["G"], "steps": K}
+            "attn_bytes": attn_bytes, "cached_tokens": tot["T"], "new_tokens": tot["G"], "steps": K}
 
 
 def run_ours(args, w):
@@ -701,6 +716,12 @@ def run_ours(args, w):
                              for n in I.WORKLOADS if n not in (w.name, "tiny_b1_l128")}
         line["workloads"]["_note"] = ("the other configurations, each timed the same way as the headline "
                                       "(median of 10 steps); tiny_b1_l128 is a correctness case only")
+    if args.fp8_lines:
+        line["fp8_cache"] = {n: workload_summary(n, args, device, peaks, flush, fp8=True)
+                             for n in (w.name, "v3_b8_l32k", "v3_b64_l8k")}
+        line["fp8_cache"]["_note"] = ("the same step on the FP8 (e4m3, per-token power-of-two scale) cache: "
+                                      "attention bytes = 644 per cached token + the f16 queries; the "
+                                      "roofline bound is whichever of HBM and tensor time is larger")
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, st["lengths"].tolist(), args.cpu_seconds)
     return line
@@ -718,7 +739,11 @@ def profile_step(args, w):
     torch.cuda.set_device(device)
     lib.load()
     st = setup_gpu(w, device, 0)
-    step = make_step(w, st, args.kernel, overlap=args.overlap)
+    fp8 = args.cache == "fp8"
+    if fp8:
+        st["pool8"] = lib.cache_to_fp8(st["d"], st["pool"])
+        st["pool"] = None
+    step = make_step(w, st, args.kernel, overlap=args.overlap, fp8=fp8)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(device)
@@ -825,12 +850,16 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--all-workloads", action=argparse.BooleanOptionalAction, default=True,
                     help="add a summary of every other configuration to the line")
+    ap.add_argument("--fp8-lines", action=argparse.BooleanOptionalAction, default=True,
+                    help="add the step on the FP8 cache for three configurations to the line")
     ap.add_argument("--overlap", action=argparse.BooleanOptionalAction, default=True,
                     help="run the append on a side stream beside the decode's query-side launches")
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="replay each step from a captured CUDA graph")
     ap.add_argument("--profile-step", action="store_true",
                     help="run one step between profiler start/stop (for ncu --profile-from-start off) and exit")
+    ap.add_argument("--cache", choices=["bf16", "fp8"], default="bf16",
+                    help="with --profile-step: the cache format of the profiled step")
     ap.add_argument("--profile-ops", action="store_true",
                     help="run one step, one query projection and the two output projections between profiler "
                          "start/stop (for ncu --profile-from-start off) and exit")
