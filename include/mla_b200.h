@@ -221,7 +221,10 @@ MLA_API int mla_append_kv_fp8(const mla_dims_t* dims, const void* x, int32_t n_t
  *            bytes, 256-byte aligned, contents need not be initialised.
  * hidden, q_rank and H * (qk_nope_dim + rope_dim) must be multiples of 64,
  * q_rank <= 2048 and rope_dim even and <= 128 (else MLA_ERR_UNSUPPORTED_DIMS). Accumulation is
- * fp32; c_q is rounded to bf16 before the second product. */
+ * fp32; c_q is rounded to bf16 before the second product. With rope_dim 64
+ * and qk_nope_dim a multiple of 64 (DeepSeek-V3) the second product writes
+ * the heads itself and q_nope and q_pe must be 16-byte aligned
+ * (MLA_ERR_INVALID_ARG otherwise). */
 MLA_API int mla_q_proj(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t hidden,
                        const void* w_qa, int32_t q_rank, const void* q_gamma, float rms_eps,
                        const void* w_qb, const int32_t* positions, float rope_base,

@@ -630,10 +630,25 @@ __host__ __device__ inline size_t row_gemm_smem(int nb) {
     return static_cast<size_t>(row_gemm_stages(nb)) * row_gemm_stage_bytes(nb) + 256 + 1024;
 }
 
+// The query projection's second product can write its heads directly: with
+// one K-range (no partials), 64-column RoPE parts and d_n a multiple of 64,
+// every 64-column piece of a tile is one piece of one head, either of its
+// non-RoPE part (rounded to bf16 into q_nope) or its whole RoPE part (rotate-
+// half pairs (i, i + 32), both in the thread's registers, rotated by
+// positions[t] * inv_freq[i] and rounded into q_pe).
+struct QHeadOut {
+    const int32_t* positions;  // null: the kernel stores fp32 partials instead
+    uint16_t* q_nope;          // [T, H, d_n]
+    uint16_t* q_pe;            // [T, H, 64]
+    int32_t dn;
+    double inv_freq[32];       // base^(-2i/64), computed on the host in double
+};
+
 __global__ void __launch_bounds__(kThreads, 1) row_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
                                                               const __grid_constant__ CUtensorMap tm_w, int32_t T,
                                                               int32_t N, int32_t k_blocks, int32_t k_per_cta,
-                                                              int32_t nb, float* __restrict__ part) {
+                                                              int32_t nb, float* __restrict__ part,
+                                                              const __grid_constant__ QHeadOut qo) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
     const int stage_bytes = row_gemm_stage_bytes(nb), n_stages = row_gemm_stages(nb);
@@ -719,8 +734,54 @@ __global__ void __launch_bounds__(kThreads, 1) row_gemm_kernel(const __grid_cons
     ptx::tc_fence_after();
     const int t = static_cast<int>(threadIdx.x);
     const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    if (qo.positions) {  // the head split: each 64-column piece of the tile is one piece of one head
+        const int D = qo.dn + 64, H = N / D;
+        const int64_t row = m0 + t;
 #pragma unroll 1
-    for (int c0 = 0; c0 < ncols; c0 += 32) {
+        for (int pc = 0; pc < nb; ++pc) {
+            float v[64];
+            {
+                float (&v0)[32] = *reinterpret_cast<float(*)[32]>(&v[0]);
+                float (&v1)[32] = *reinterpret_cast<float(*)[32]>(&v[32]);
+                ptx::tmem_ld32(tl + 64 * pc, v0);
+                ptx::tmem_ld32(tl + 64 * pc + 32, v1);
+                ptx::tmem_wait_ld();
+            }
+            if (!ok || nk == 0) {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) v[i] = 0.f;
+            }
+            const int n = n0 + 64 * pc;
+            const int h = n / D, off = n - h * D;
+            if (row >= T) continue;
+            uint4* dst;
+            if (off < qo.dn) {
+                dst = reinterpret_cast<uint4*>(qo.q_nope + (row * H + h) * qo.dn + off);
+            } else {
+                dst = reinterpret_cast<uint4*>(qo.q_pe + (row * H + h) * 64);
+                const double pos = static_cast<double>(qo.positions[row]);
+#pragma unroll 1
+                for (int i = 0; i < 32; ++i) {
+                    // angle reduced to [-pi, pi] in double with a two-term 2 pi, so that the
+                    // float sine and cosine stay on their short-argument path
+                    const double angle = pos * qo.inv_freq[i];
+                    const double k = rint(angle * 0.15915494309189535);  // 1 / (2 pi)
+                    const double reduced = fma(-k, 2.4492935982947064e-16, fma(-k, 6.283185307179586, angle));
+                    float sn, cs;
+                    sincosf(static_cast<float>(reduced), &sn, &cs);
+                    const float x1 = v[i], x2 = v[i + 32];
+                    v[i] = x1 * cs - x2 * sn;
+                    v[i + 32] = x2 * cs + x1 * sn;
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                dst[c] = make_uint4(ptx::bf16x2(v[8 * c], v[8 * c + 1]), ptx::bf16x2(v[8 * c + 2], v[8 * c + 3]),
+                                    ptx::bf16x2(v[8 * c + 4], v[8 * c + 5]), ptx::bf16x2(v[8 * c + 6], v[8 * c + 7]));
+        }
+    }
+#pragma unroll 1
+    for (int c0 = 0; c0 < (qo.positions ? 0 : ncols); c0 += 32) {
         float v[32];
         ptx::tmem_ld32(tl + c0, v);
         ptx::tmem_wait_ld();

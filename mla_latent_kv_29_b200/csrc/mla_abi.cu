@@ -375,8 +375,10 @@ AppendPlan append_plan(int32_t n_tokens, int32_t hidden, int32_t N) {
 // tcgen05 row GEMM: x bf16 [T, K], w bf16 [K, N], K and N multiples of 64,
 // x and w 16-byte aligned.
 int launch_row_gemm(const void* x, int32_t T, int32_t K, const void* w, int32_t N, const AppendPlan& ap,
-                    float* part, cudaStream_t st) {
+                    float* part, cudaStream_t st, const tc05::QHeadOut* qo = nullptr) {
     if (!aligned(x, 16) || !aligned(w, 16)) return MLA_ERR_INVALID_ARG;
+    tc05::QHeadOut none{};
+    if (!qo) qo = &none;
     CUtensorMap tm_x, tm_w;
     if (int rc = encode_2d(&tm_x, x, K, T, tc05::kRows)) return rc;
     if (int rc = encode_2d(&tm_w, w, N, K, 64)) return rc;
@@ -384,8 +386,12 @@ int launch_row_gemm(const void* x, int32_t T, int32_t K, const void* w, int32_t 
     if (int rc = ensure_smem(tc05::row_gemm_kernel, smem)) return rc;
     const dim3 grid(N / (64 * ap.nb), (T + tc05::kRows - 1) / tc05::kRows, ap.splits);
     return launch(tc05::row_gemm_kernel, grid, tc05::kThreads, smem, st, tm_x, tm_w, T, N, K / 64, ap.k_per_split,
-                  ap.nb, part);
+                  ap.nb, part, *qo);
 }
+
+// The second product of the query projection writes q_nope / q_pe itself
+// (tc05::QHeadOut) when every 64-column tile is one piece of one head.
+bool q_heads_fused(const mla_dims_t* d) { return d->rope_dim == 64 && d->qk_nope_dim % 64 == 0; }
 
 // ---- query projection workspace: GEMM 1 partials | c_q bf16 | GEMM 2 partials
 struct QProjLayout {
@@ -403,6 +409,13 @@ int q_proj_layout(const mla_dims_t* d, int32_t T, int32_t hidden, int32_t R, QPr
         return MLA_ERR_UNSUPPORTED_DIMS;
     L->g1 = append_plan(T, hidden, R);
     L->g2 = append_plan(T, R, static_cast<int32_t>(N2));
+    if (q_heads_fused(d)) {
+        // one K-range and the widest tile that divides N2: 256 columns per CTA stream
+        // W_qb's rows in 512-byte pieces (measured 52 us against 64 for 64-column
+        // tiles at 64 tokens on V3 dims)
+        const int nb = N2 % 256 == 0 ? 4 : (N2 % 128 == 0 ? 2 : 1);
+        L->g2 = AppendPlan{true, 1, R / 64, nb};
+    }
     size_t off = 0;
     L->part1 = off; off = align_up(off + sizeof(float) * static_cast<size_t>(L->g1.splits) * T * R);
     L->cq = off; off = align_up(off + sizeof(uint16_t) * static_cast<size_t>(T) * R);
@@ -576,6 +589,17 @@ int mla_q_proj(const mla_dims_t* dims, const void* x, int32_t n_tokens, int32_t 
     if (int rc = launch(q_norm_kernel, n_tokens, kQNormThreads, sizeof(float) * q_rank, st, part1, L.g1.splits,
                         n_tokens, q_rank, static_cast<const uint16_t*>(q_gamma), rms_eps, cq)) return rc;
     // q = c_q . W_qb, then the per-head split and the RoPE of the rope part
+    if (q_heads_fused(dims)) {
+        if (!aligned(q_nope, 16) || !aligned(q_pe, 16)) return MLA_ERR_INVALID_ARG;
+        tc05::QHeadOut qo;
+        qo.positions = positions;
+        qo.q_nope = static_cast<uint16_t*>(q_nope);
+        qo.q_pe = static_cast<uint16_t*>(q_pe);
+        qo.dn = dn;
+        for (int i = 0; i < 32; ++i) qo.inv_freq[i] = std::pow(static_cast<double>(rope_base), -2.0 * i / 64.0);
+        if (int rc = launch_row_gemm(cq, n_tokens, q_rank, w_qb, N2, L.g2, part2, st, &qo)) return rc;
+        return launch_status();
+    }
     if (int rc = launch_row_gemm(cq, n_tokens, q_rank, w_qb, N2, L.g2, part2, st)) return rc;
     QSplitParams P;
     P.part = part2;

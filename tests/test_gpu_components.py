@@ -154,6 +154,9 @@ def test_append_tiny_dims_uses_the_cuda_core_path():
 @pytest.mark.parametrize("case", [
     ("small", I.Dims(num_heads=4, kv_lora_rank=64, rope_dim=32, qk_nope_dim=32, v_head_dim=32, block_size=64),
      5, 256, 128, True),
+    # RoPE width 64 and d_n a multiple of 64: the second product writes the heads itself
+    ("small_heads_in_gemm", I.Dims(num_heads=4, kv_lora_rank=64, rope_dim=64, qk_nope_dim=64, v_head_dim=32,
+                                   block_size=64), 5, 256, 128, True),
     ("v3", I.WORKLOADS["v3_b64_l1k_8k"].dims, 64, 7168, 1536, True),
     ("v3_ragged_no_gamma", I.WORKLOADS["v3_b64_l1k_8k"].dims, 130, 7168, 1536, False),
 ])
