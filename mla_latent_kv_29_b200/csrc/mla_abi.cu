@@ -279,6 +279,7 @@ int decode_layout(const mla_dims_t* d, int32_t batch, int32_t q_len, int32_t max
     if (batch < 1 || q_len < 1 || max_len < q_len) return MLA_ERR_INVALID_ARG;
     const int kernel = pick_kernel(d, o);
     if (kernel < 0) return MLA_ERR_UNSUPPORTED_DIMS;
+    if (o && o->cache_fp8 && kernel != kKernelPair) return MLA_ERR_UNSUPPORTED_DIMS;  // only it reads FP8
     L->kernel = kernel;
     L->tile = kernel == kKernelPair ? pair::kTile : kGenTokens;
     const int64_t G = static_cast<int64_t>(batch) * q_len;
@@ -676,8 +677,7 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_pe, int
     const bool tc05 = tc05_dims_ok(dims) && aligned(q_nope, 16) && aligned(q_pe, 16) && aligned(w_uk, 16) &&
                       aligned(w_uv, 16) && aligned(out, 16);
     if (L.kernel == kKernelPair && !tc05) return MLA_ERR_INVALID_ARG;
-    const bool fp8_cache = opts && opts->cache_fp8;
-    if (fp8_cache && L.kernel != kKernelPair) return MLA_ERR_UNSUPPORTED_DIMS;  // only the tcgen05 kernel reads it
+    const bool fp8_cache = opts && opts->cache_fp8;  // decode_layout admits it with the tcgen05 kernel only
     const bool latent_out = opts && opts->output_latent;
     if (latent_out && !tc05) return MLA_ERR_UNSUPPORTED_DIMS;  // o_lat comes from the tensor-core merge
 

@@ -142,6 +142,28 @@ def _check(status: int, what: str):
         raise MLAError(status, what)
 
 
+_nvtx = False
+
+
+def set_nvtx(on: bool = True) -> None:
+    """Mark every library call with an NVTX range named after its C entry point
+    (visible in Nsight timelines); off by default, which costs nothing."""
+    global _nvtx
+    _nvtx = bool(on)
+
+
+def _call(name: str, *args) -> int:
+    """Calls C entry point `name`, inside an NVTX range of that name when enabled."""
+    fn = getattr(load(), name)
+    if not _nvtx:
+        return fn(*args)
+    torch.cuda.nvtx.range_push(name)
+    try:
+        return fn(*args)
+    finally:
+        torch.cuda.nvtx.range_pop()
+
+
 def _workspace(nbytes: int, device) -> torch.Tensor:
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
@@ -161,9 +183,9 @@ def append_kv(dims: Dims, x, w_kva, seq_ids, positions, block_table, pool, rms_g
     need = lib.mla_append_workspace_size(ctypes.byref(cd), T, hidden)
     if workspace is None:
         workspace = _workspace(need, x.device)
-    fn, name = (lib.mla_append_kv_fp8, "mla_append_kv_fp8") if fp8 else (lib.mla_append_kv, "mla_append_kv")
-    st = fn(
-        ctypes.byref(cd), _ptr(x, torch.bfloat16, "x"), T, hidden, _ptr(w_kva, torch.bfloat16, "w_kva"),
+    name = "mla_append_kv_fp8" if fp8 else "mla_append_kv"
+    st = _call(
+        name, ctypes.byref(cd), _ptr(x, torch.bfloat16, "x"), T, hidden, _ptr(w_kva, torch.bfloat16, "w_kva"),
         _ptr(rms_gamma, torch.bfloat16, "rms_gamma"), float(rms_eps), float(rope_base),
         _ptr(seq_ids, torch.int32, "seq_ids"), _ptr(positions, torch.int32, "positions"),
         _ptr(block_table, torch.int32, "block_table"), block_table.shape[0], block_table.shape[1],
@@ -187,7 +209,7 @@ def cache_to_fp8(dims: Dims, pool, out=None, stream=None):
         raise MLAError(-2, "mla_fp8_block_bytes")
     if out is None:
         out = torch.empty(nb, bb, dtype=torch.uint8, device=pool.device)
-    st = lib.mla_cache_to_fp8(ctypes.byref(c_dims(dims, 1.0)), _ptr(pool, torch.bfloat16, "pool"), nb,
+    st = _call("mla_cache_to_fp8", ctypes.byref(c_dims(dims, 1.0)), _ptr(pool, torch.bfloat16, "pool"), nb,
                               _ptr(out, torch.uint8, "pool_fp8"), _stream(stream))
     _check(st, "mla_cache_to_fp8")
     return out
@@ -214,7 +236,7 @@ def q_proj(dims: Dims, x, w_qa, w_qb, positions, q_gamma=None, rms_eps: float = 
         q_nope = torch.empty(T, dims.num_heads, dims.qk_nope_dim, dtype=torch.bfloat16, device=x.device)
     if q_pe is None:
         q_pe = torch.empty(T, dims.num_heads, dims.rope_dim, dtype=torch.bfloat16, device=x.device)
-    st = lib.mla_q_proj(
+    st = _call("mla_q_proj",
         ctypes.byref(cd), _ptr(x, torch.bfloat16, "x"), T, hidden, _ptr(w_qa, torch.bfloat16, "w_qa"), q_rank,
         _ptr(q_gamma, torch.bfloat16, "q_gamma"), float(rms_eps), _ptr(w_qb, torch.bfloat16, "w_qb"),
         _ptr(positions, torch.int32, "positions"), float(rope_base), _ptr(q_nope, torch.bfloat16, "q_nope"),
@@ -243,7 +265,7 @@ def o_proj(x, w, y=None, workspace=None, stream=None):
         workspace = _workspace(need, x.device)
     if y is None:
         y = torch.empty(T, n, dtype=torch.bfloat16, device=x.device)
-    st = lib.mla_o_proj(_ptr(x2, torch.bfloat16, "x"), T, k, _ptr(w, torch.bfloat16, "w"), n,
+    st = _call("mla_o_proj", _ptr(x2, torch.bfloat16, "x"), T, k, _ptr(w, torch.bfloat16, "w"), n,
                         _ptr(y, torch.bfloat16, "y"), _ptr(workspace, None, "workspace"),
                         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "mla_o_proj")
@@ -283,7 +305,7 @@ def decode(dims: Dims, softmax_scale: float, q_nope, q_pe, pool, block_table, co
         raise MLAError(-2, "mla_decode_workspace_size")
     if workspace is None:
         workspace = _workspace(need, q_nope.device)
-    st = lib.mla_decode(
+    st = _call("mla_decode",
         ctypes.byref(cd), _ptr(q_nope, torch.bfloat16, "q_nope"), _ptr(q_pe, torch.bfloat16, "q_pe"), B, Sq,
         _ptr(pool, torch.uint8 if cache_fp8 else torch.bfloat16, "pool"), pool.shape[0],
         _ptr(block_table, torch.int32, "block_table"),
@@ -305,7 +327,7 @@ def decode_no_alloc(dims: Dims, softmax_scale: float, q_nope, q_pe, pool, block_
     B, Sq = q_nope.shape[0], q_nope.shape[1]
     if out is None:
         out = torch.empty(B, Sq, dims.num_heads, dims.v_head_dim, dtype=torch.bfloat16, device=q_nope.device)
-    st = lib.mla_decode_no_alloc(
+    st = _call("mla_decode_no_alloc",
         ctypes.byref(cd), _ptr(q_nope, torch.bfloat16, "q_nope"), _ptr(q_pe, torch.bfloat16, "q_pe"), B, Sq,
         _ptr(pool, torch.bfloat16, "pool"), pool.shape[0], _ptr(block_table, torch.int32, "block_table"),
         block_table.shape[1], _ptr(context_lens, torch.int32, "context_lens"), int(max_context_len),
@@ -322,7 +344,7 @@ def combine(dims: Dims, o_part, lse_part, part_offsets, o_lat=None, lse_out=None
     G = part_offsets.numel() - 1
     if o_lat is None:
         o_lat = torch.empty(G, dims.num_heads, dims.kv_lora_rank, dtype=torch.float32, device=o_part.device)
-    st = lib.mla_combine(ctypes.byref(cd), _ptr(o_part, torch.float32, "o_part"),
+    st = _call("mla_combine", ctypes.byref(cd), _ptr(o_part, torch.float32, "o_part"),
                          _ptr(lse_part, torch.float32, "lse_part"), _ptr(part_offsets, torch.int32, "part_offsets"),
                          G, _ptr(o_lat, torch.float32, "o_lat"), _ptr(lse_out, torch.float32, "lse_out"),
                          _stream(stream))

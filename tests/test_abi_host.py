@@ -111,6 +111,25 @@ def test_q_proj_validation(so):
     assert call(ws_bytes=16) == -3
 
 
+def test_fp8_cache_validation(so):
+    d = _dims()
+    assert so.mla_fp8_block_bytes(ctypes.byref(d)) == 64 * 640 + 256  # 41216: 644 bytes per token
+    assert so.mla_fp8_block_bytes(ctypes.byref(_dims(kv_lora_rank=520))) == 0  # latent not a multiple of 16
+    assert so.mla_fp8_block_bytes(ctypes.byref(_dims(block_size=62))) == 0  # scales not 16-byte aligned
+    fake = ctypes.c_void_p(1 << 20)
+    assert so.mla_cache_to_fp8(ctypes.byref(d), None, 10, fake, None) == -1
+    assert so.mla_cache_to_fp8(ctypes.byref(d), fake, 0, fake, None) == -1
+    assert so.mla_cache_to_fp8(ctypes.byref(d), ctypes.c_void_p((1 << 20) + 8), 10, fake, None) == -1  # unaligned
+    assert so.mla_cache_to_fp8(ctypes.byref(_dims(rope_dim=4)), fake, 10, fake, None) == -2
+    assert so.mla_append_kv_fp8(ctypes.byref(_dims(rope_dim=4)), fake, 64, 7168, fake, None, 1e-6, 1e4, fake, fake,
+                                fake, 16, 1, fake, 10, fake, 1 << 30, None) == -2
+    assert so.mla_append_kv_fp8(ctypes.byref(d), fake, 64, 7168, fake, None, 1e-6, 1e4, fake, fake, fake, 16, 1,
+                                fake, 10, fake, 16, None) == -3
+    # an FP8 decode needs the tensor-core kernel: the CUDA-core kernel refuses it before any launch
+    opts = L.c_opts(kernel=2, cache_fp8=True)
+    assert _decode(so, d, opts=opts) == -2
+
+
 def test_valid_call_without_gpu_reports_no_device(so):
     import torch
 
@@ -130,3 +149,21 @@ def test_python_binding_has_no_cpu_path():
     q = torch.zeros(1, 1, 16, 32, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         L.decode(w.dims, w.softmax_scale, q, q, q, q, q, 128, q, q)
+
+
+def test_nvtx_ranges_wrap_the_calls(monkeypatch):
+    """With NVTX on, each entry point runs inside a range of its own name, and the
+    range is closed even when the call fails."""
+    import torch
+
+    pushed, popped = [], []
+    monkeypatch.setattr(torch.cuda.nvtx, "range_push", lambda n: pushed.append(n))
+    monkeypatch.setattr(torch.cuda.nvtx, "range_pop", lambda: popped.append(1))
+    L.set_nvtx(True)
+    try:
+        st = L._call("mla_combine", ctypes.byref(_dims()), None, None, None, 4, None, None, None)
+    finally:
+        L.set_nvtx(False)
+    assert st == -1 and pushed == ["mla_combine"] and len(popped) == 1
+    L._call("mla_combine", ctypes.byref(_dims()), None, None, None, 4, None, None, None)
+    assert pushed == ["mla_combine"]  # off again: no range

@@ -64,6 +64,16 @@ def test_cache_to_fp8_is_bit_exact():
     assert bad.size == 0, f"{len(bad)} bytes differ, first at {bad[:4].tolist()}"
 
 
+def test_cache_to_fp8_other_dims_is_bit_exact():
+    """The conversion is not tied to V3 dims: latent 64, RoPE 16, 128-token blocks."""
+    L = _lib()
+    d = I.WORKLOADS["tiny_b1_l128"].dims
+    g = torch.Generator().manual_seed(6)
+    pool = (torch.randn(3, d.block_size, d.row_width, generator=g) * 3.0).to(torch.bfloat16)
+    got = L.cache_to_fp8(d, pool.cuda()).cpu().numpy()
+    assert np.array_equal(got, F.quantize_pool(_f64(pool), d))
+
+
 @pytest.mark.parametrize("n_seqs,per_seq,hidden", [(3, 1, 256), (5, 4, 7168), (2, 40, 512)])
 def test_append_fp8_matches_oracle_and_touches_only_its_rows(n_seqs, per_seq, hidden):
     L = _lib()
