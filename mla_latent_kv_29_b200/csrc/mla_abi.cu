@@ -966,7 +966,7 @@ extern "C" int mla_decode_no_alloc(const mla_dims_t* dims, const void* q_nope, c
                                    int32_t max_context_len, const void* w_uk, const void* w_uv, void* out,
                                    const mla_decode_opts_t* opts, void* stream) {
     const size_t need = mla_decode_workspace_size(dims, batch, q_len, max_context_len, opts);
-    if (need == 0) {  // same validation verdict as mla_decode
+    if (need == 0) {  // the same validation result as mla_decode
         DecodeLayout L;
         const int rc = decode_layout(dims, batch, q_len, max_context_len, opts, &L);
         return rc ? rc : MLA_ERR_INVALID_ARG;
