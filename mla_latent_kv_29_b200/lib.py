@@ -319,17 +319,18 @@ def decode(dims: Dims, softmax_scale: float, q_nope, q_pe, pool, block_table, co
 
 def decode_no_alloc(dims: Dims, softmax_scale: float, q_nope, q_pe, pool, block_table, context_lens,
                     max_context_len: int, w_uk, w_uv, out=None, kernel: int = KERNEL_AUTO, num_workers: int = 0,
-                    stream=None):
+                    stream=None, cache_fp8: bool = False):
     """mla_decode with the library's built-in scratch buffer (no workspace argument)."""
     lib = load()
     cd = c_dims(dims, softmax_scale)
-    o = c_opts(kernel, num_workers)
+    o = c_opts(kernel, num_workers, cache_fp8=cache_fp8)
     B, Sq = q_nope.shape[0], q_nope.shape[1]
     if out is None:
         out = torch.empty(B, Sq, dims.num_heads, dims.v_head_dim, dtype=torch.bfloat16, device=q_nope.device)
     st = _call("mla_decode_no_alloc",
         ctypes.byref(cd), _ptr(q_nope, torch.bfloat16, "q_nope"), _ptr(q_pe, torch.bfloat16, "q_pe"), B, Sq,
-        _ptr(pool, torch.bfloat16, "pool"), pool.shape[0], _ptr(block_table, torch.int32, "block_table"),
+        _ptr(pool, torch.uint8 if cache_fp8 else torch.bfloat16, "pool"), pool.shape[0],
+        _ptr(block_table, torch.int32, "block_table"),
         block_table.shape[1], _ptr(context_lens, torch.int32, "context_lens"), int(max_context_len),
         _ptr(w_uk, torch.bfloat16, "w_uk"), _ptr(w_uv, torch.bfloat16, "w_uv"),
         _ptr(out, torch.bfloat16, "out"), ctypes.byref(o), _stream(stream))

@@ -247,3 +247,57 @@ def test_fp8_full_size_sampled():
     ref = O.decode_paged(data["q_nope"], data["q_pe"], deq.reshape(-1, d.block_size, d.row_width), tab,
                          data["lengths"], data["w_uk"], data["w_uv"], d, w.softmax_scale, batch_ids=ids)
     _check(got, ref, ids=ids)
+
+
+def test_fp8_bounded_wait_expiry_reports_timeout_and_context_survives():
+    """The FP8 kernel's waits give up too: with its load warps starved and a 1 ms
+    limit, every role (expansion warps included) drains and the call reports
+    MLA_ERR_DEVICE_TIMEOUT; an ordinary FP8 decode afterwards still matches."""
+    L = _lib()
+    w, lengths = _v3("f8_wait_expiry", 1, 1, [100])
+    data = build(w, lengths=lengths)
+    pool8, deq = _fp8_pools(w, data)
+    dd = to_device(data)
+    L.device_error()  # clear
+    L.decode(w.dims, w.softmax_scale, dd["q_nope"], dd["q_pe"], pool8, dd["table"], dd["lengths"], 100,
+             dd["w_uk"], dd["w_uv"], kernel=1, debug_wait_limit_us=1000, debug_starve=True, cache_fp8=True)
+    assert L.device_error() == -6
+    assert L.device_error() == 0
+    got = _decode8(w, dd, pool8)
+    ref = O.decode_paged(data["q_nope"], data["q_pe"], deq, data["table"].numpy(), data["lengths"], data["w_uk"],
+                         data["w_uv"], w.dims, w.softmax_scale)
+    _check(got, ref)
+
+
+def test_fp8_decode_latent_output():
+    """With output_latent the FP8 decode returns o_lat: the oracle's latent decode
+    on the dequantised cache."""
+    L = _lib()
+    w, lengths = _v3("f8_latent", 3, 2, [300, 77, 129])
+    data = build(w, lengths=lengths)
+    pool8, deq = _fp8_pools(w, data)
+    dd = to_device(data)
+    o_lat = L.decode(w.dims, w.softmax_scale, dd["q_nope"], dd["q_pe"], pool8, dd["table"], dd["lengths"], 300,
+                     dd["w_uk"], dd["w_uv"], output_latent=True, cache_fp8=True)
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    ref = O.decode_latent_paged(data["q_nope"], data["q_pe"], deq, data["table"].numpy(), data["lengths"],
+                                data["w_uk"], w.dims, w.softmax_scale)
+    _check(o_lat.float().cpu().numpy(), ref)
+
+
+def test_fp8_decode_without_a_workspace():
+    """mla_decode_no_alloc reads the FP8 cache too (its scratch is the library's
+    own buffer); against the oracle on the dequantised cache."""
+    L = _lib()
+    w, lengths = _v3("f8_no_alloc", 4, 2, [63, 64, 65, 129])
+    data = build(w, lengths=lengths)
+    pool8, deq = _fp8_pools(w, data)
+    dd = to_device(data)
+    got = L.decode_no_alloc(w.dims, w.softmax_scale, dd["q_nope"], dd["q_pe"], pool8, dd["table"], dd["lengths"],
+                            129, dd["w_uk"], dd["w_uv"], cache_fp8=True)
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    ref = O.decode_paged(data["q_nope"], data["q_pe"], deq, data["table"].numpy(), data["lengths"], data["w_uk"],
+                         data["w_uv"], w.dims, w.softmax_scale)
+    _check(got.float().cpu().numpy(), ref)
