@@ -642,6 +642,7 @@ def run_ours(args, w):
     torch.cuda.synchronize(device)
     barrier(device)
     e2e_ms = [a.elapsed_time(b) for a, b in e2e_ev]
+    t_e2e_pipe = e2e_pipelined(args, step, st, pieces, offs, total, h_in, K, device)
 
     t_step = max_over_ranks(statistics.mean(step_ms), device)
     t_attn = max_over_ranks(statistics.mean(attn_ms), device)
@@ -672,6 +673,7 @@ def run_ours(args, w):
     assert lib.device_error() == 0, "device fault in the query projection"
     t_q = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in q_ev), device)
     t_e2e = max_over_ranks(statistics.mean(e2e_ms), device)
+    t_e2e_pipe = max_over_ranks(t_e2e_pipe, device)
     if rank != 0:
         return None
     tot = workload_totals(w, st["lengths"].tolist())
@@ -700,9 +702,17 @@ def run_ours(args, w):
         "decode_tokens_per_s": round(world * tot["G"] / (t_step / 1e3), 1),
         "step_roofline_nominal_us": round(nominal_step * 1e6, 2),
         "step_frac_of_nominal_roofline": round(nominal_step / (t_step / 1e3), 4),
-        "e2e": {"value": round(t_e2e * 1e3, 2), "unit": UNIT,
+        "e2e": {"value": round(t_e2e_pipe * 1e3, 2), "unit": UNIT,
                 "h2d_bytes_per_step": h_in.numel(),
-                "d2h_bytes_per_step": h_out.numel() * 2},
+                "d2h_bytes_per_step": h_out.numel() * 2,
+                "timing": "K steps back to back through the public calls: each step copies its inputs from pinned "
+                          "host memory and its output back; two staging and output buffers let step k's copies "
+                          "overlap steps k - 1 and k + 1 (copy streams in, compute, copy streams out); total time / "
+                          "K, no L2 flush between steps (the cache exceeds L2, but the layer's 42 MB of weights stay "
+                          "in L2 from one step to the next, which is why this can come out below the flushed "
+                          "device-timed step)",
+                "serial_value": round(t_e2e * 1e3, 2),
+                "serial_timing": "each step alone: L2 flush, copy in, step, copy out, CUDA events around the three"},
         "gpu_launches": launches_per_step * K,
         "q_proj": q_proj_line(w, t_q, peaks),
         "o_proj": o_proj_lines(w, st, flush, min(K, 20), args.warmup, device, peaks),
@@ -725,6 +735,95 @@ def run_ours(args, w):
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, st["lengths"].tolist(), args.cpu_seconds)
     return line
+
+
+def e2e_pipelined(args, step, st, pieces, offs, total, h_in0, K, device):
+    """Mean ms per step of K back-to-back steps through the public calls, each
+    copying its inputs in from pinned host memory and its output back, with
+    two staging / output buffer sets so that a step's copies overlap its
+    neighbours' compute: H2D of step k on one stream (after step k - 2 is done
+    with the buffers), the step on the compute stream, D2H on a third."""
+    import torch
+
+    sets = []
+    for i in range(2):
+        h_in = h_in0 if i == 0 else h_in0.clone().pin_memory()
+        d_in = torch.empty(total, dtype=torch.uint8, device=device)
+        views = [d_in[o:o + t_.numel() * t_.element_size()].view(t_.dtype).view(t_.shape)
+                 for t_, o in zip(pieces, offs)]
+        out = torch.empty_like(st["out"])
+        h_out = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+        sets.append(dict(h_in=h_in, d_in=d_in, views=views, out=out, h_out=h_out, graph=None))
+    saved = (st["new_seq"], st["new_pos"], st["out"])
+
+    def bind(S):
+        st["new_seq"], st["new_pos"], st["out"] = S["views"][3], S["views"][4], S["out"]
+
+    def run_step(S):
+        if S["graph"] is not None:
+            S["graph"].replay()
+        else:
+            bind(S)
+            step(x_new=S["views"][0], q_nope=S["views"][1], q_pe=S["views"][2])
+
+    if args.graph:
+        for S in sets:
+            bind(S)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(x_new=S["views"][0], q_nope=S["views"][1], q_pe=S["views"][2])
+            S["graph"] = g
+        torch.cuda.synchronize(device)
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    s_c = torch.cuda.current_stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_c = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for i in range(2):  # every event recorded once before its first wait
+        ev_in[i].record(s_in)
+        ev_c[i].record(s_c)
+        ev_out[i].record(s_out)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):  # warm-up of the pipelined loop itself
+        for k in range(2):
+            S = sets[k]
+            with torch.cuda.stream(s_in):
+                S["d_in"].copy_(S["h_in"], non_blocking=True)
+            s_c.wait_stream(s_in)
+            run_step(S)
+            with torch.cuda.stream(s_out):
+                s_out.wait_stream(s_c)
+                S["h_out"].copy_(S["out"], non_blocking=True)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    t0.record(s_c)
+    s_in.wait_event(t0)
+    s_out.wait_event(t0)
+    for k in range(K):
+        i = k % 2
+        S = sets[i]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_c[i])  # step k - 2 has read this staging buffer
+            S["d_in"].copy_(S["h_in"], non_blocking=True)
+            ev_in[i].record(s_in)
+        s_c.wait_event(ev_in[i])
+        s_c.wait_event(ev_out[i])  # step k - 2's output has been copied out
+        run_step(S)
+        ev_c[i].record(s_c)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_c[i])
+            S["h_out"].copy_(S["out"], non_blocking=True)
+            ev_out[i].record(s_out)
+    s_c.wait_stream(s_out)
+    s_c.wait_stream(s_in)
+    t1.record(s_c)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    st["new_seq"], st["new_pos"], st["out"] = saved
+    for S in sets:
+        S["graph"] = None
+    return t0.elapsed_time(t1) / K
 
 
 def profile_step(args, w):
