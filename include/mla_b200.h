@@ -78,7 +78,11 @@ typedef struct mla_dims {
 typedef struct mla_decode_opts {
     int32_t kernel;      /* 0 auto; 1 sm100 tensor-core kernel (V3 dims only);
                             2 CUDA-core kernel (any supported dims) */
-    int32_t num_workers; /* 0 auto; else the number of split-KV workers the
+    int32_t num_workers; /* 0 auto (tensor-core kernel: one worker per SM
+                            pair, but at most half of the problem's 128-token
+                            tiles, batch * q_len * ceil(max_context_len / 128),
+                            so that a small problem keeps about two tiles per
+                            worker); else the number of split-KV workers the
                             balanced schedule targets (>= 1) */
     void* event_attn_begin; /* NULL or a cudaEvent_t recorded on `stream` right
                                before the split-KV attention kernel */
