@@ -58,7 +58,8 @@ def test_e4m3_encode_saturates_and_ties_to_even():
     assert F.e4m3_encode([1.1875])[0] == 0x3A  # halfway 1.125 and 1.25: even mantissa 2
     assert F.e4m3_encode([2.0 ** -10])[0] == 0x00  # half the smallest subnormal -> 0 (even)
     assert F.e4m3_encode([3 * 2.0 ** -10])[0] == 0x02  # halfway codes 1 and 2 -> 2
-    assert F.e4m3_encode([math.nan])[0] == F.E4M3_NAN
+    assert F.e4m3_encode([math.nan])[0] == 0x7F  # S.1111.111, the code torch's cast gives too
+    assert torch.tensor([math.nan]).to(torch.float8_e4m3fn).view(torch.uint8).item() == 0x7F
 
 
 def test_scale_exponent_closed_form():
