@@ -108,6 +108,21 @@ def test_prefill_chunk(kernel, workers):
 
 
 @pytest.mark.parametrize("kernel", list(KERNELS))
+@pytest.mark.parametrize("workers", [0, 3])
+def test_pages_of_128_tokens(kernel, workers):
+    """block_size 128 (the tensor-core kernel takes any multiple of 64): a
+    128-token tile is half of a page, so both halves of a pair read the same
+    pool block."""
+    import dataclasses
+
+    w, lengths = small_v3("pages128", 3, 2, [70, 260, 385])
+    w = dataclasses.replace(w, dims=dataclasses.replace(w.dims, block_size=128))
+    data = build(w, lengths=lengths)
+    got = run_decode(w, to_device(data), kernel=KERNELS[kernel], num_workers=workers)
+    check(got, oracle_out(w, data))
+
+
+@pytest.mark.parametrize("kernel", list(KERNELS))
 def test_nan_in_unused_rows_and_blocks(kernel):
     w, lengths = small_v3("nan_fill", 3, 2, [70, 5, 200], spare=3)
     data = build(w, fill=float("nan"), lengths=lengths)

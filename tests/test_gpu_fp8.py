@@ -301,3 +301,18 @@ def test_fp8_decode_without_a_workspace():
     ref = O.decode_paged(data["q_nope"], data["q_pe"], deq, data["table"].numpy(), data["lengths"], data["w_uk"],
                          data["w_uv"], w.dims, w.softmax_scale)
     _check(got.float().cpu().numpy(), ref)
+
+
+def test_fp8_decode_pages_of_128_tokens():
+    """The FP8 maps address (slot, block): 128-token pages put a tile's halves
+    at slots 0 and 64 of one block."""
+    import dataclasses
+
+    w, lengths = _v3("f8_pages128", 3, 2, [70, 260, 385])
+    w = dataclasses.replace(w, dims=dataclasses.replace(w.dims, block_size=128))
+    data = build(w, lengths=lengths)
+    pool8, deq = _fp8_pools(w, data)
+    got = _decode8(w, to_device(data), pool8, workers=3)
+    ref = O.decode_paged(data["q_nope"], data["q_pe"], deq, data["table"].numpy(), data["lengths"], data["w_uk"],
+                         data["w_uv"], w.dims, w.softmax_scale)
+    _check(got, ref)
