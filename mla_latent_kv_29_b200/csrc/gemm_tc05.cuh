@@ -477,7 +477,9 @@ __global__ void __launch_bounds__(kMuvThreads, 1) merge_uv_kernel(const __grid_c
 // [H * d_n rows, d_c columns], box {64, d_n} (MN-major B: the latent index is
 // contiguous). Each CTA loads its d_n / 64 A boxes and the 4 B boxes of its
 // 256 output columns at once (d_n = 128: 96 KB, two CTAs per SM), then runs
-// d_n / 16 MMAs of N = 256 into 256 TMEM columns.
+// d_n / 16 MMAs of N = 256 into 256 TMEM columns. With q_f16 set, Q is written
+// as IEEE half instead of bf16 (q_pe converted too): the operand type of the
+// attention over the FP8 cache, whose MMAs run on f16.
 // grid (H, ceil(G / 128), d_c / 256); block 128; dynamic smem absorb_smem(d_n).
 __host__ __device__ inline size_t absorb_a_bytes(int dn) { return static_cast<size_t>(dn / 64) * kRows * kBoxBytes; }
 __host__ __device__ inline size_t absorb_smem(int dn) {
