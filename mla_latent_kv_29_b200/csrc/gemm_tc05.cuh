@@ -9,8 +9,10 @@
 //               then multiplied (uv_kernel)
 //   row GEMM:   y = x W (fp32 partials over K ranges) for x [T, K] and W
 //               [K, N] (row_gemm_kernel): the cache append's x W_kva, the
-//               query projection's x W_qa and c_q W_qb, and the output
-//               projection (sum_partials_kernel adds its partials into bf16).
+//               query projection's x W_qa and c_q W_qb (the latter, with one
+//               K range, writing q_nope and the rotated q_pe itself), and the
+//               output projection (sum_partials_kernel adds its partials into
+//               bf16).
 //
 // Roles of the 128-thread kernels: lane 0 of warp 0 issues the TMA loads,
 // lane 0 of warp 1 the MMAs (M = 128, cta_group::1), warp 2 owns the TMEM
