@@ -3,8 +3,9 @@
 // (q_b_proj), each head's qk_head_dim values split into the d_n non-RoPE part
 // and the d_r RoPE part, the latter rotated (rotate-half RoPE of
 // "一次讲透MHA、GQA、MQA、MLA", "MLA的实现") at the token's position.
-// The two GEMMs run on tc05::row_gemm_kernel (fp32 partials); the kernels here
-// are the row normalisation between them and the split + RoPE after them.
+// The two GEMMs run on tc05::row_gemm_kernel; the kernels here are the row
+// normalisation between them and, for RoPE widths other than 64, the split +
+// RoPE after them (with 64 the second GEMM writes the heads itself).
 // Both run once per CTA, so their loops stay rolled.
 #pragma once
 
